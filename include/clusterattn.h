@@ -1,0 +1,114 @@
+/*
+ * libclusterattn: cluster-attention forward pass for NVIDIA B200 (sm_100a).
+ *
+ * The operation (model card "Hooshaai/distilbert-sst2-cluster-attention",
+ * Architecture Overview and Mathematical Formulation section 1; model card
+ * "Hooshaai/svd-sst2-roberta-cluster", sections 2.1 and 3), per (batch b,
+ * head h), with Q, K, V the [L, d] slices of that head and s = 1 / sqrt(d):
+ *
+ *   1. strided init   mu_k = Q[floor(k L / K)],                k = 0..K-1
+ *   2. for t = 1..iters (batch Lloyd's k-means on the queries):
+ *        D_ik = |Q_i|^2 + |mu_k|^2 - 2 Q_i . mu_k
+ *        c_i  = argmin_k D_ik                     (ties: lowest k)
+ *        mu_k = sum_{c_i = k} Q_i / max(1, count_k) (empty cluster: zero)
+ *      with iters == 0: c_i = 0 and mu stays at init;
+ *   3. centroid attention  V_cent = softmax(mu K^T s) V            [K, d]
+ *   4. gather             g_i = V_cent[c_i]
+ *   5. window attention   o_i = softmax_{j : |i-j| <= floor(W/2), 0 <= j < L}
+ *                                 (s Q_i . K_j) V_j
+ *   6. convex fusion      O_i = (1 - alpha) g_i + alpha o_i.
+ *
+ * Precision.  Arithmetic is fp32 with fp32 accumulation; O is rounded once to
+ * the input type.  Centroids are kept in fp32 (the cards' module measures
+ * distances on centroids cast to float): each is the exact member sum divided
+ * by the count in fp64 and rounded once to fp32.  The argmin is decided on
+ * those fp32 centroids exactly: an fp32 pass with a rigorous error bound
+ * settles almost every token, and the few whose two best candidates lie
+ * within that bound are re-measured in fp64, in the expanded form above with
+ * index-order sums.
+ *
+ * Conventions for every entry point below:
+ *   - Tensors are dense, row-major [B, H, L, d] (d fastest), as produced by
+ *     the cards' projection + view(B, L, H, d).transpose(1, 2); assign_out is
+ *     [B, H, L] int32, centroids_out [B, H, K, d] fp32.
+ *   - Pointers are DEVICE pointers owned by the caller (except ca_forward_host
+ *     and ca_forward_host_bf16, which take HOST pointers), 16-byte aligned;
+ *     out must not overlap q, k or v.  The library keeps no pointer after a
+ *     call returns.
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Device entry points are asynchronous on that stream; their
+ *     scratch memory comes from cudaMallocAsync / cudaFreeAsync on it.
+ *   - assign_out and centroids_out may be NULL (not written).
+ *   - Validation happens on the host before any launch and returns a status;
+ *     nothing is launched on a non-OK status.  Launch failures return
+ *     CA_ERR_CUDA.  Device-side problems are reported by ca_sync_status.
+ *   - Supported: d == 64; 1 <= K <= min(L, 128); iters >= 0; W >= 0;
+ *     0 <= alpha <= 1 (finite); B, H, L >= 1; B*H*L*d < 2^31.
+ *   - Results are deterministic: the same inputs give bitwise-identical
+ *     outputs on the same GPU.
+ */
+#ifndef CLUSTERATTN_H_
+#define CLUSTERATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CA_OK = 0,
+    CA_ERR_INVALID_ARG = 1, /* a size, pointer or scalar argument is out of range   */
+    CA_ERR_UNSUPPORTED = 2, /* a valid request this build does not handle (e.g. d)  */
+    CA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed          */
+    CA_ERR_TIMEOUT = 4,     /* a bounded device-side wait ran out                   */
+    CA_ERR_DEVICE = 5       /* a kernel recorded an internal consistency failure    */
+} ca_status;
+
+/* fp32 Q, K, V and out.  Steps 1-6 above for all B*H heads. */
+ca_status ca_forward(const float *q, const float *k, const float *v, int B, int H, int L, int d,
+                     int K, int iters, int W, float alpha, float *out, int32_t *assign_out,
+                     float *centroids_out, void *stream);
+
+/* bf16 Q, K, V and out, as raw uint16 bit patterns; centroids_out stays fp32. */
+ca_status ca_forward_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int H,
+                          int L, int d, int K, int iters, int W, float alpha, uint16_t *out,
+                          int32_t *assign_out, float *centroids_out, void *stream);
+
+/* As ca_forward / ca_forward_bf16 (dtype 0 = fp32, 1 = bf16), and also writes
+ * the assignment of every iteration to assign_hist [B, H, iters, L] int32
+ * (device pointer, may be NULL).  Used to check each Lloyd step on its own. */
+ca_status ca_forward_trace(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                           int L, int d, int K, int iters, int W, float alpha, void *out,
+                           int32_t *assign_out, float *centroids_out, int32_t *assign_hist,
+                           void *stream);
+
+/* End-to-end form for callers holding HOST buffers (dtype 0 = fp32 with float
+ * arrays, 1 = bf16 with uint16 arrays): copies q, k, v to the device, runs the
+ * forward on stream, copies out (and assign_out / centroids_out when non-NULL)
+ * back and synchronizes the stream before returning.  Host buffers should be
+ * pinned for full copy bandwidth; pageable buffers work but copy slower.
+ * Device buffers are stream-ordered allocations released before return. */
+ca_status ca_forward_host(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                          int L, int d, int K, int iters, int W, float alpha, void *out,
+                          int32_t *assign_out, float *centroids_out, void *stream);
+
+/* Synchronizes stream, then reports (and clears) the first device-side error
+ * recorded by a kernel of this library on the current device, or a pending
+ * CUDA error.  CA_OK when nothing went wrong. */
+ca_status ca_sync_status(void *stream);
+
+/* Static description of a status code. */
+const char *ca_status_string(ca_status s);
+
+/* Thread-local detail of the last non-OK status returned on this thread. */
+const char *ca_last_error(void);
+
+/* Library version string. */
+const char *ca_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CLUSTERATTN_H_ */
