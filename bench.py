@@ -1,0 +1,332 @@
+#!/usr/bin/env python
+"""Benchmark of the cluster-attention forward pass (libclusterattn on B200).
+
+One step = one full forward (k-means, centroid attention, gather, window
+attention, blend) over one batch of a seeded synthetic workload, inputs
+already resident in HBM.  L2 is flushed (a 256 MiB write, outside the timed
+event pairs) before every timed step.  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle arm
+
+Under torchrun (N > 1) every rank runs its own full copy of the workload on
+its own GPU (independent heads, no data-path collective: weak scaling); the
+step time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "cluster-attention fwd tokens/s (B·H·L/s) and achieved HBM GB/s vs ~8 TB/s"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "l512_bf16"
+FALLBACK_HBM_GBS = 6650.0
+# Kernel whose launches the roofline object reports, per workload.
+DOMINANT = {"small_f32": "kmeans_assign", "card_gmm_f32": "kmeans_assign", "l512_bf16": "kmeans_assign",
+            "l4k_gmm_bf16": "kmeans_assign", "l32k_dup_bf16": "kmeans_assign"}
+
+
+def workload_desc(w) -> dict:
+    src = {"normal": "N(0,1)", "gmm": f"Q {w.gmm_components}-component Gaussian mixture (means N(0,4I), std {w.gmm_std}), K,V N(0,1)"}[w.q_kind]
+    if w.dup_frac:
+        src += f", {int(w.dup_frac * 100)}% of tokens duplicated (forced ties / empty clusters)"
+    return {"workload": f"{w.name}: B={w.B}, H={w.H}, L={w.L}, d={w.d}, K={w.K}, iters={w.iters}, "
+                        f"W={w.W}, alpha={w.alpha}; {w.dtype} {src}, seed 0",
+            "B": w.B, "H": w.H, "L": w.L, "d": w.d, "K": w.K, "iters": w.iters, "W": w.W,
+            "alpha": w.alpha, "io_dtype": w.dtype, "tokens_per_step": w.tokens,
+            "l2": "flushed before every timed step (256 MiB write outside the timed events)"}
+
+
+def dist_info():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
+    None when there is none or the kernel sources changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[workload][kernel]
+        from means_cluster_attention_b200.build import source_hash
+        if e.get("source_hash") != source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.strip().split(", ") for r in f if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_rate(w, target_s: float, max_heads=None):
+    """Time the fp64 oracle (as it stands) on a bounded head sample of the
+    workload on this host's cores.  Returns (tokens/s, cores, sample text)."""
+    import oracle
+    from means_cluster_attention_b200.inputs import make_inputs
+    cores = oracle.default_threads()
+    # calibrate on one head, then size the sample to about target_s
+    x1 = make_inputs(w, heads=1)
+    t0 = time.perf_counter()
+    oracle.forward(x1["q64"], x1["k64"], x1["v64"], K=w.K, iters=w.iters, W=w.W, alpha=w.alpha, nthreads=1)
+    t1 = max(time.perf_counter() - t0, 1e-4)
+    heads = int(max(1, min(w.heads, (target_s / t1) * cores)))
+    if max_heads:
+        heads = min(heads, max_heads)
+    heads = max(1, (heads // cores) * cores) if heads >= cores else heads
+    x = make_inputs(w, heads=heads)
+    used = min(cores, heads)
+    t0 = time.perf_counter()
+    oracle.forward(x["q64"], x["k64"], x["v64"], K=w.K, iters=w.iters, W=w.W, alpha=w.alpha, nthreads=used)
+    dt = time.perf_counter() - t0
+    toks = heads * w.L
+    sample = (f"{heads} of {w.heads} heads (L={w.L}) of {w.name}, same recipe and sizes, "
+              f"{toks} tokens in {dt:.2f} s on {used} threads")
+    return toks / dt, used, sample, dt
+
+
+def run_reference(args, w):
+    ws, rank, local = dist_info()
+    if rank != 0:
+        return 0
+    # Each step: a bounded head sample sized so warmup + steps end within ~3 min.
+    per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    rates = []
+    cores = sample = None
+    for i in range(args.warmup + args.steps):
+        rate, cores, sample, dt = cpu_oracle_rate(w, per_step)
+        if i >= args.warmup:
+            rates.append(rate)
+    value = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * w.tokens / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_desc(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, w):
+    import numpy as np
+    import torch
+    import means_cluster_attention_b200 as ca
+    from means_cluster_attention_b200 import _lib
+    from means_cluster_attention_b200.inputs import make_inputs
+
+    ws, rank, local = dist_info()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    x = make_inputs(w, seed=0)
+    if w.dtype == "f32":
+        conv = lambda a: torch.from_numpy(a).to(dev)
+    else:
+        conv = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    q, k, v = conv(x["q"]), conv(x["k"]), conv(x["v"])
+    out = torch.empty_like(q)
+    assign = torch.empty((w.B, w.H, w.L), dtype=torch.int32, device=dev)
+    cent = torch.empty((w.B, w.H, w.K, w.d), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        ca.forward(q, k, v, w.K, w.iters, w.W, w.alpha, out=out, assign=assign, centroids=cent)
+
+    for _ in range(args.warmup):
+        step()
+        flush.zero_()
+    ca.sync_status()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    dom = args.profile_kernel or DOMINANT.get(w.name, "kmeans_assign")
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    _lib.profile_start(dom)
+    n0 = _lib.launch_count()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record()
+        step()
+        ends[i].record()
+    torch.cuda.synchronize()
+    n_launch = _lib.launch_count() - n0
+    kstat = _lib.profile_stop()
+    if pg:
+        pg.barrier()
+    clk = clocks.stop()
+    ca.sync_status()
+    ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms_step = sum(ms) / len(ms)
+    k_ms = kstat.total_ms / max(1, kstat.launches)
+    if pg:
+        t = torch.tensor([ms_step, k_ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_step, k_ms = float(t[0]), float(t[1])
+    value = w.tokens * ws / (ms_step / 1e3)
+
+    # End to end through the C ABI with host buffers (pinned), copies included.
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        oh = torch.empty_like(qh).pin_memory()
+        n_e2e = max(3, min(args.steps, 10))
+        for _ in range(2):
+            ca.forward_host(qh, kh, vh, w.K, w.iters, w.W, w.alpha, out=oh)
+        e_ms = []
+        for _ in range(n_e2e):
+            s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s_ev.record()
+            ca.forward_host(qh, kh, vh, w.K, w.iters, w.W, w.alpha, out=oh)
+            e_ev.record()
+            torch.cuda.synchronize()
+            e_ms.append(s_ev.elapsed_time(e_ev))
+        e_step = sum(e_ms) / len(e_ms)
+        if pg:
+            t = torch.tensor([e_step], device=dev, dtype=torch.float64)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e_step = float(t[0])
+        nbytes = q.numel() * q.element_size()
+        e2e = {"value": w.tokens * ws / (e_step / 1e3), "unit": UNIT, "h2d_bytes_per_step": 3 * nbytes,
+               "d2h_bytes_per_step": nbytes, "ms_per_step": e_step}
+
+    peak, peak_kind = measured_peak()
+    achieved = (kstat.algorithmic_bytes / max(1, kstat.launches)) / (k_ms / 1e3) / 1e9 if k_ms > 0 else 0.0
+    step_bytes = 4.0 * w.tokens * w.d * w.elem_bytes
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_kind": peak_kind,
+                "traffic": ncu_traffic(dom, w.name),
+                "kernel_ms_per_launch": k_ms, "launches_timed": int(kstat.launches),
+                "alg_bytes_per_launch": kstat.algorithmic_bytes / max(1, kstat.launches),
+                "step_alg_bytes": step_bytes, "step_achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+                "step_frac": step_bytes / (ms_step / 1e3) / 1e9 / peak, "step_frac_of_8tbs": step_bytes / (ms_step / 1e3) / 8e12}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_desc(w),
+        "roofline": roofline, "e2e": e2e, "gpu_launches": int(n_launch), "clocks": clk,
+        "step_ms_min": min(ms), "step_ms_median": statistics.median(ms),
+    }
+    if pg:
+        line["config"]["parallelism"] = f"replicas x{ws} (independent heads, no collective)"
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        rate, cores, sample, _ = cpu_oracle_rate(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    from means_cluster_attention_b200.inputs import WORKLOADS
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--profile-kernel", default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -31,8 +31,8 @@
  *   - Tensors are dense, row-major [B, H, L, d] (d fastest), as produced by
  *     the cards' projection + view(B, L, H, d).transpose(1, 2); assign_out is
  *     [B, H, L] int32, centroids_out [B, H, K, d] fp32.
- *   - Pointers are DEVICE pointers owned by the caller (except ca_forward_host
- *     and ca_forward_host_bf16, which take HOST pointers), 16-byte aligned;
+ *   - Pointers are DEVICE pointers owned by the caller (ca_forward_host takes
+ *     HOST pointers instead), 16-byte aligned;
  *     out must not overlap q, k or v.  The library keeps no pointer after a
  *     call returns.
  *   - stream is a cudaStream_t passed as void* (NULL = legacy default
@@ -43,7 +43,8 @@
  *     nothing is launched on a non-OK status.  Launch failures return
  *     CA_ERR_CUDA.  Device-side problems are reported by ca_sync_status.
  *   - Supported: d == 64; 1 <= K <= min(L, 128); iters >= 0; W >= 0;
- *     0 <= alpha <= 1 (finite); B, H, L >= 1; B*H*L*d < 2^31.
+ *     0 <= alpha <= 1 (finite); B, H, L >= 1; B*H <= 65535; B*H*L*d < 2^31.
+ *     Inputs must be finite.
  *   - Results are deterministic: the same inputs give bitwise-identical
  *     outputs on the same GPU.
  */
@@ -106,6 +107,26 @@ const char *ca_last_error(void);
 
 /* Library version string. */
 const char *ca_version(void);
+
+/* Measurement support.  Every kernel launch of the library is counted
+ * (ca_launch_count, process-wide, monotonic).  Between ca_profile_start and
+ * ca_profile_stop, each launch of the kernel named kernel_name (NULL or ""
+ * selects none) is bracketed by two CUDA events recorded on its launching
+ * stream.  ca_profile_stop waits for those events and fills *stat with the
+ * number of timed launches, their summed duration and their summed
+ * algorithmic HBM bytes (one read of every input and one write of every
+ * output the kernel must touch).  Kernel names: "kmeans_init",
+ * "kmeans_assign", "kmeans_update", "centroid_attn", "centroid_combine",
+ * "window_blend". */
+typedef struct {
+    long long launches;
+    double total_ms;
+    double algorithmic_bytes;
+} ca_kernel_stat;
+
+ca_status ca_profile_start(const char *kernel_name);
+ca_status ca_profile_stop(ca_kernel_stat *stat);
+long long ca_launch_count(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,322 @@
+// libclusterattn host layer: argument validation, stream-ordered scratch,
+// kernel launches.  The C ABI is declared in include/clusterattn.h.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include "clusterattn.h"
+#include "common.cuh"
+#include "kmeans.cuh"
+#include "attention.cuh"
+#include "profile.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+ca_status fail(ca_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+ca_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(CA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+#define CA_CUDA(call)                                          \
+    do {                                                       \
+        cudaError_t e_ = (call);                               \
+        if (e_ != cudaSuccess) return cuda_fail(e_, #call);    \
+    } while (0)
+
+struct Problem {
+    int B, H, L, d, K, iters, W;
+    float alpha;
+    int64_t heads() const { return (int64_t)B * H; }
+};
+
+ca_status validate(const void *q, const void *k, const void *v, const void *out, const Problem &p) {
+    if (!q || !k || !v || !out) return fail(CA_ERR_INVALID_ARG, "q, k, v and out must be non-null");
+    if (p.B < 1 || p.H < 1 || p.L < 1)
+        return fail(CA_ERR_INVALID_ARG, "B, H, L must be >= 1 (got %d, %d, %d)", p.B, p.H, p.L);
+    if (p.d < 1) return fail(CA_ERR_INVALID_ARG, "d must be >= 1 (got %d)", p.d);
+    if (p.d != ca::kD) return fail(CA_ERR_UNSUPPORTED, "only d == 64 is supported (got %d)", p.d);
+    if (p.K < 1 || p.K > p.L)
+        return fail(CA_ERR_INVALID_ARG, "K must satisfy 1 <= K <= L (got K=%d, L=%d)", p.K, p.L);
+    if (p.K > ca::kMaxK) return fail(CA_ERR_UNSUPPORTED, "K must be <= %d (got %d)", ca::kMaxK, p.K);
+    if (p.iters < 0) return fail(CA_ERR_INVALID_ARG, "iters must be >= 0 (got %d)", p.iters);
+    if (p.W < 0) return fail(CA_ERR_INVALID_ARG, "W must be >= 0 (got %d)", p.W);
+    if (!std::isfinite(p.alpha) || p.alpha < 0.f || p.alpha > 1.f)
+        return fail(CA_ERR_INVALID_ARG, "alpha must be finite and in [0, 1]");
+    if (p.heads() > 65535) return fail(CA_ERR_UNSUPPORTED, "B*H must be <= 65535 (got %lld)", (long long)p.heads());
+    const int64_t elems = p.heads() * (int64_t)p.L * p.d;
+    if (elems >= (int64_t(1) << 31)) return fail(CA_ERR_INVALID_ARG, "B*H*L*d must be < 2^31");
+    const uintptr_t a = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)out;
+    if (a & 15u) return fail(CA_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+    return CA_OK;
+}
+
+// Stream-ordered scratch, released on the same stream when the object dies.
+struct Scratch {
+    cudaStream_t st;
+    void *ptrs[8] = {};
+    int n = 0;
+    explicit Scratch(cudaStream_t s) : st(s) {}
+    ~Scratch() {
+        for (int i = 0; i < n; ++i) cudaFreeAsync(ptrs[i], st);
+    }
+    cudaError_t get(void **p, size_t bytes) {
+        cudaError_t e = cudaMallocAsync(p, bytes, st);
+        if (e == cudaSuccess) ptrs[n++] = *p;
+        return e;
+    }
+};
+
+template <typename T>
+ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *out,
+                      int32_t *assign_out, float *cent_out, int32_t *hist, cudaStream_t st) {
+    using namespace ca;
+    const int64_t NH = p.heads();
+    const int L = p.L, K = p.K;
+    const float scale = 1.0f / sqrtf((float)p.d);
+
+    Scratch s(st);
+    float *mu = nullptr, *vcent = nullptr, *part = nullptr;
+    double *sums = nullptr;
+    int32_t *counts = nullptr, *assign = assign_out;
+    const int n_chunks = (L + kCaChunk - 1) / kCaChunk;
+    CA_CUDA(s.get((void **)&mu, sizeof(float) * NH * K * kD));
+    CA_CUDA(s.get((void **)&vcent, sizeof(float) * NH * K * kD));
+    CA_CUDA(s.get((void **)&part, sizeof(float) * NH * n_chunks * K * (kD + 2)));
+    CA_CUDA(s.get((void **)&sums, sizeof(double) * NH * K * kD));
+    CA_CUDA(s.get((void **)&counts, sizeof(int32_t) * NH * K));
+    if (!assign) CA_CUDA(s.get((void **)&assign, sizeof(int32_t) * NH * L));
+
+    const double esz = (double)sizeof(T);
+    const double head_bytes = (double)NH * L * kD * esz;  // one read of Q (or K, V, O)
+
+    // 1. strided init (and c = 0 for iters == 0)
+    {
+        Launch pl("kmeans_init", st, 0.0);
+        kmeans_init_kernel<T><<<(unsigned)NH, 256, 0, st>>>(q, L, K, mu);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+    if (p.iters == 0) {
+        CA_CUDA(cudaMemsetAsync(assign, 0, sizeof(int32_t) * NH * L, st));
+        if (cent_out) CA_CUDA(cudaMemcpyAsync(cent_out, mu, sizeof(float) * NH * K * kD, cudaMemcpyDeviceToDevice, st));
+    }
+    CA_CUDA(cudaMemsetAsync(sums, 0, sizeof(double) * NH * K * kD, st));
+    CA_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * NH * K, st));
+
+    // 2. Lloyd iterations
+    const int tokens_per_cta = 1024;
+    const size_t asmem = AssignSmem::bytes(K);
+    CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asmem));
+    const dim3 agrid((L + tokens_per_cta - 1) / tokens_per_cta, (unsigned)NH);
+    for (int t = 0; t < p.iters; ++t) {
+        int32_t *hist_t = hist ? hist + (int64_t)t * L : nullptr;
+        {
+            Launch pl("kmeans_assign", st, head_bytes);
+            kmeans_assign_kernel<T><<<agrid, kAssignThreads, asmem, st>>>(
+                q, L, K, tokens_per_cta, mu, assign, hist_t, (int64_t)p.iters * L, sums, counts);
+            pl.after();
+        }
+        CA_CUDA(cudaGetLastError());
+        {
+            Launch pl("kmeans_update", st, 0.0);
+            kmeans_update_kernel<<<(unsigned)NH, 256, 0, st>>>(K, sums, counts, mu,
+                                                                t == p.iters - 1 ? cent_out : nullptr);
+            pl.after();
+        }
+        CA_CUDA(cudaGetLastError());
+    }
+
+    // 3. centroid attention
+    const size_t csmem = centroid_attn_smem_bytes(K);
+    CA_CUDA(cudaFuncSetAttribute(centroid_attn_partial_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem));
+    {
+        Launch pl("centroid_attn", st, 2.0 * head_bytes);
+        centroid_attn_partial_kernel<T><<<dim3(n_chunks, (unsigned)NH), kCaThreads, csmem, st>>>(
+            k, v, L, K, scale, mu, n_chunks, part);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+    {
+        Launch pl("centroid_combine", st, 0.0);
+        centroid_attn_combine_kernel<<<(unsigned)NH, 256, 0, st>>>(K, n_chunks, part, vcent);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+
+    // 4-6. gather + window attention + blend
+    const size_t wsmem = window_smem_bytes();
+    CA_CUDA(cudaFuncSetAttribute(window_blend_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem));
+    {
+        Launch pl("window_blend", st, 4.0 * head_bytes);
+        window_blend_kernel<T><<<dim3((L + kWinQ - 1) / kWinQ, (unsigned)NH), kWinThreads, wsmem, st>>>(
+            q, k, v, L, K, p.W / 2, scale, p.alpha, vcent, assign, out);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+    return CA_OK;
+}
+
+ca_status dispatch(const void *q, const void *k, const void *v, int dtype, const Problem &p,
+                   void *out, int32_t *assign_out, float *cent_out, int32_t *hist, void *stream) {
+    ca_status s = validate(q, k, v, out, p);
+    if (s != CA_OK) return s;
+    if (((uintptr_t)cent_out & 15u) || ((uintptr_t)assign_out & 3u) || ((uintptr_t)hist & 3u))
+        return fail(CA_ERR_INVALID_ARG, "centroids_out must be 16-byte aligned, assign buffers 4-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == 0)
+        return run_forward<float>((const float *)q, (const float *)k, (const float *)v, p, (float *)out,
+                                  assign_out, cent_out, hist, st);
+    if (dtype == 1)
+        return run_forward<__nv_bfloat16>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
+                                          (const __nv_bfloat16 *)v, p, (__nv_bfloat16 *)out,
+                                          assign_out, cent_out, hist, st);
+    return fail(CA_ERR_INVALID_ARG, "dtype must be 0 (fp32) or 1 (bf16), got %d", dtype);
+}
+
+}  // namespace
+
+extern "C" {
+
+ca_status ca_forward(const float *q, const float *k, const float *v, int B, int H, int L, int d,
+                     int K, int iters, int W, float alpha, float *out, int32_t *assign_out,
+                     float *centroids_out, void *stream) {
+    Problem p{B, H, L, d, K, iters, W, alpha};
+    return dispatch(q, k, v, 0, p, out, assign_out, centroids_out, nullptr, stream);
+}
+
+ca_status ca_forward_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int H,
+                          int L, int d, int K, int iters, int W, float alpha, uint16_t *out,
+                          int32_t *assign_out, float *centroids_out, void *stream) {
+    Problem p{B, H, L, d, K, iters, W, alpha};
+    return dispatch(q, k, v, 1, p, out, assign_out, centroids_out, nullptr, stream);
+}
+
+ca_status ca_forward_trace(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                           int L, int d, int K, int iters, int W, float alpha, void *out,
+                           int32_t *assign_out, float *centroids_out, int32_t *assign_hist,
+                           void *stream) {
+    Problem p{B, H, L, d, K, iters, W, alpha};
+    return dispatch(q, k, v, dtype, p, out, assign_out, centroids_out, assign_hist, stream);
+}
+
+ca_status ca_forward_host(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                          int L, int d, int K, int iters, int W, float alpha, void *out,
+                          int32_t *assign_out, float *centroids_out, void *stream) {
+    Problem p{B, H, L, d, K, iters, W, alpha};
+    if (!q || !k || !v || !out) return fail(CA_ERR_INVALID_ARG, "q, k, v and out must be non-null");
+    if (dtype != 0 && dtype != 1) return fail(CA_ERR_INVALID_ARG, "dtype must be 0 or 1");
+    ca_status s = validate((const void *)16, (const void *)16, (const void *)16, (void *)16, p);
+    if (s != CA_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t esz = dtype == 0 ? 4 : 2;
+    const size_t n = (size_t)p.heads() * p.L * p.d;
+    void *dq = nullptr, *dk = nullptr, *dv = nullptr, *dout = nullptr, *dcent = nullptr;
+    int32_t *dassign = nullptr;
+    {
+        Scratch sc(st);
+        CA_CUDA(sc.get(&dq, n * esz));
+        CA_CUDA(sc.get(&dk, n * esz));
+        CA_CUDA(sc.get(&dv, n * esz));
+        CA_CUDA(sc.get(&dout, n * esz));
+        if (assign_out) CA_CUDA(sc.get((void **)&dassign, sizeof(int32_t) * p.heads() * p.L));
+        if (centroids_out) CA_CUDA(sc.get(&dcent, sizeof(float) * p.heads() * p.K * p.d));
+        CA_CUDA(cudaMemcpyAsync(dq, q, n * esz, cudaMemcpyHostToDevice, st));
+        CA_CUDA(cudaMemcpyAsync(dk, k, n * esz, cudaMemcpyHostToDevice, st));
+        CA_CUDA(cudaMemcpyAsync(dv, v, n * esz, cudaMemcpyHostToDevice, st));
+        s = dispatch(dq, dk, dv, dtype, p, dout, dassign, (float *)dcent, nullptr, stream);
+        if (s != CA_OK) return s;
+        CA_CUDA(cudaMemcpyAsync(out, dout, n * esz, cudaMemcpyDeviceToHost, st));
+        if (assign_out)
+            CA_CUDA(cudaMemcpyAsync(assign_out, dassign, sizeof(int32_t) * p.heads() * p.L, cudaMemcpyDeviceToHost, st));
+        if (centroids_out)
+            CA_CUDA(cudaMemcpyAsync(centroids_out, dcent, sizeof(float) * p.heads() * p.K * p.d, cudaMemcpyDeviceToHost, st));
+    }
+    CA_CUDA(cudaStreamSynchronize(st));
+    return CA_OK;
+}
+
+ca_status ca_sync_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int code = 0, where = 0;
+    e = cudaMemcpyFromSymbol(&code, ca::g_dev_error, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol");
+    if (code != 0) {
+        cudaMemcpyFromSymbol(&where, ca::g_dev_error_where, sizeof(int));
+        const int zero = 0;
+        cudaMemcpyToSymbol(ca::g_dev_error, &zero, sizeof(int));
+        return fail((ca_status)code, "device-side error %d recorded at site %d", code, where);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "pending CUDA error");
+    return CA_OK;
+}
+
+const char *ca_status_string(ca_status s) {
+    switch (s) {
+        case CA_OK: return "CA_OK";
+        case CA_ERR_INVALID_ARG: return "CA_ERR_INVALID_ARG: an argument is out of range";
+        case CA_ERR_UNSUPPORTED: return "CA_ERR_UNSUPPORTED: valid request not handled by this build";
+        case CA_ERR_CUDA: return "CA_ERR_CUDA: a CUDA call or launch failed";
+        case CA_ERR_TIMEOUT: return "CA_ERR_TIMEOUT: a bounded device-side wait ran out";
+        case CA_ERR_DEVICE: return "CA_ERR_DEVICE: a kernel recorded an internal consistency failure";
+    }
+    return "unknown ca_status";
+}
+
+const char *ca_last_error(void) { return g_last_error.c_str(); }
+
+const char *ca_version(void) { return "libclusterattn 0.1 (sm_100a)"; }
+
+ca_status ca_profile_start(const char *kernel_name) {
+    ca::ProfileState &p = ca::profile();
+    std::lock_guard<std::mutex> g(p.mu);
+    if (p.active) return fail(CA_ERR_INVALID_ARG, "profiling already started");
+    p.selected = kernel_name ? kernel_name : "";
+    p.pairs.clear();
+    p.active = true;
+    return CA_OK;
+}
+
+ca_status ca_profile_stop(ca_kernel_stat *stat) {
+    ca::ProfileState &p = ca::profile();
+    std::lock_guard<std::mutex> g(p.mu);
+    if (!p.active) return fail(CA_ERR_INVALID_ARG, "profiling not started");
+    p.active = false;
+    ca_kernel_stat r{0, 0.0, 0.0};
+    ca_status status = CA_OK;
+    for (auto &pr : p.pairs) {
+        float ms = 0.f;
+        cudaError_t e = cudaEventSynchronize(pr.b);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, pr.a, pr.b);
+        if (e != cudaSuccess && status == CA_OK) status = cuda_fail(e, "cudaEventElapsedTime");
+        r.launches += 1;
+        r.total_ms += ms;
+        r.algorithmic_bytes += pr.bytes;
+        p.pool.push_back(pr.a);
+        p.pool.push_back(pr.b);
+    }
+    p.pairs.clear();
+    if (stat) *stat = r;
+    return status;
+}
+
+long long ca_launch_count(void) { return ca::profile().launches.load(); }
+
+}  // extern "C"

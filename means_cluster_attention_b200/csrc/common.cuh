@@ -1,0 +1,75 @@
+// Shared device helpers for the cluster-attention kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ca {
+
+// Head dimension handled by this build.
+constexpr int kD = 64;
+// Largest cluster count accepted at the boundary.
+constexpr int kMaxK = 128;
+
+// First device-side error recorded by any kernel of the library (0 = none).
+// Codes match ca_status; the host reads and clears it in ca_sync_status.
+__device__ int g_dev_error;
+__device__ int g_dev_error_where;
+
+__device__ __forceinline__ void record_error(int code, int where) {
+    if (atomicCAS(&g_dev_error, 0, code) == 0) g_dev_error_where = where;
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Load one 64-element row (16-byte aligned) into fp32 registers.
+__device__ __forceinline__ void load_row64(const float *__restrict__ p, float (&r)[kD]) {
+    const float4 *p4 = reinterpret_cast<const float4 *>(p);
+#pragma unroll
+    for (int i = 0; i < kD / 4; ++i) {
+        float4 t = __ldg(p4 + i);
+        r[4 * i + 0] = t.x;
+        r[4 * i + 1] = t.y;
+        r[4 * i + 2] = t.z;
+        r[4 * i + 3] = t.w;
+    }
+}
+
+__device__ __forceinline__ void load_row64(const __nv_bfloat16 *__restrict__ p, float (&r)[kD]) {
+    const uint4 *p4 = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < kD / 8; ++i) {
+        uint4 t = __ldg(p4 + i);
+        const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            r[8 * i + 2 * e + 0] = __uint_as_float(w[e] << 16);
+            r[8 * i + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+        }
+    }
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
+}  // namespace ca

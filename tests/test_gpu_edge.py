@@ -1,0 +1,98 @@
+"""GPU edge cases against the oracle: ragged and tiny sequence lengths, K at
+1, at L and at its maximum, zero iterations, zero and very wide windows,
+alpha at both ends, both dtypes; plus determinism, the host-buffer entry
+point, and device status after a clean run."""
+
+import numpy as np
+import pytest
+
+import oracle
+from means_cluster_attention_b200.inputs import Workload, make_inputs
+from helpers import TOL, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # L, K, iters, W, alpha, B, H
+    (1, 1, 3, 32, 0.5, 1, 2),
+    (2, 2, 1, 0, 0.5, 1, 1),
+    (63, 7, 4, 1, 0.25, 2, 3),
+    (65, 65, 2, 33, 0.0, 1, 2),
+    (100, 1, 3, 400, 1.0, 2, 1),
+    (129, 128, 3, 16, 0.7, 1, 1),
+    (1000, 13, 0, 32, 0.5, 1, 2),
+    (1025, 100, 2, 64, 0.3, 1, 2),
+    (2049, 32, 3, 129, 0.6, 1, 1),
+]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("L,K,iters,W,alpha,B,H", CASES)
+def test_edge_case_parity(dtype, L, K, iters, W, alpha, B, H):
+    w = Workload("edge", B, H, L, 64, K, iters, W, alpha, dtype, "normal")
+    x = make_inputs(w, seed=L * 31 + K)
+    g = run_gpu(x, dtype, K, iters, W, alpha, hist=iters > 0)
+    ref_out, ref_assign, ref_cent, ref_hist = oracle.forward(
+        x["q64"], x["k64"], x["v64"], K=K, iters=iters, W=W, alpha=alpha, hist=True)
+    np.testing.assert_array_equal(g["assign"], ref_assign)
+    if iters > 0:
+        np.testing.assert_array_equal(g["hist"], ref_hist)
+    np.testing.assert_array_equal(g["cent"], ref_cent)
+    err = float(np.abs(g["out"] - ref_out).max())
+    assert err <= TOL[dtype], err
+
+
+def test_gmm_with_tiny_clusters_and_exact_ties():
+    # Mixture data with more clusters than components: duplicated centroids,
+    # empty clusters and zero centroids all appear.
+    w = Workload("gmm_edge", 2, 4, 300, 64, 40, 4, 32, 0.5, "bf16", "gmm", gmm_components=8,
+                 gmm_std=0.05)
+    x = make_inputs(w, seed=5)
+    g = run_gpu(x, "bf16", w.K, w.iters, w.W, w.alpha, hist=True)
+    _, ref_assign, ref_cent, ref_hist = oracle.forward(x["q64"], x["k64"], x["v64"], K=w.K,
+                                                      iters=w.iters, W=w.W, alpha=w.alpha, hist=True)
+    np.testing.assert_array_equal(g["hist"], ref_hist)
+    np.testing.assert_array_equal(g["cent"], ref_cent)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_deterministic(dtype):
+    import torch
+    import means_cluster_attention_b200 as ca
+    from helpers import to_device
+    w = Workload("det", 2, 4, 3000, 64, 24, 3, 40, 0.5, dtype, "normal")
+    x = make_inputs(w, seed=11)
+    q, k, v = to_device(x, dtype)
+    o1, a1, c1 = ca.forward(q, k, v, w.K, w.iters, w.W, w.alpha)
+    o2, a2, c2 = ca.forward(q, k, v, w.K, w.iters, w.W, w.alpha)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(a1, a2) and torch.equal(c1, c2)
+    ca.sync_status()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_host_entry_point_matches_device_path(dtype):
+    import torch
+    import means_cluster_attention_b200 as ca
+    from helpers import to_device
+    w = Workload("host", 2, 3, 777, 64, 16, 3, 32, 0.5, dtype, "normal")
+    x = make_inputs(w, seed=3)
+    q, k, v = to_device(x, dtype)
+    o_dev, a_dev, c_dev = ca.forward(q, k, v, w.K, w.iters, w.W, w.alpha, sync_check=True)
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    o_h = torch.empty_like(qh).pin_memory()
+    a_h = torch.empty((2, 3, 777), dtype=torch.int32).pin_memory()
+    c_h = torch.empty((2, 3, 16, 64), dtype=torch.float32).pin_memory()
+    ca.forward_host(qh, kh, vh, w.K, w.iters, w.W, w.alpha, out=o_h, assign=a_h, centroids=c_h)
+    assert torch.equal(o_h, o_dev.cpu())
+    assert torch.equal(a_h, a_dev.cpu())
+    assert torch.equal(c_h, c_dev.cpu())
+
+
+def test_invalid_call_launches_nothing_and_status_stays_clean():
+    import torch
+    import means_cluster_attention_b200 as ca
+    q = torch.zeros((1, 1, 8, 64), device="cuda")
+    with pytest.raises(ca.ClusterAttnError):
+        ca.forward(q, q, q, 4, -1, 4, 0.5)
+    ca.sync_status()
