@@ -93,7 +93,7 @@ def _call(lib, fn="ca_forward", q=P, k=P, v=P, out=P, assign=None, cent=None, **
     (dict(alpha=-0.1), 1),
     (dict(alpha=float("nan")), 1),
     (dict(alpha=float("inf")), 1),
-    (dict(B=1 << 10, H=1 << 7, L=1 << 8), 1),  # B*H*L*d >= 2^31
+    (dict(B=255, H=256, L=1 << 11), 1),        # B*H*L*d >= 2^31
     (dict(B=1 << 10, H=1 << 7, L=16), 2),      # B*H above 65535
 ])
 @pytest.mark.parametrize("fn", ["ca_forward", "ca_forward_bf16"])
