@@ -7,12 +7,14 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "clusterattn.h"
 #include "common.cuh"
 #include "kmeans.cuh"
 #include "attention.cuh"
+#include "fused.cuh"
 #include "profile.cuh"
 
 namespace {
@@ -66,7 +68,36 @@ ca_status validate(const void *q, const void *k, const void *v, const void *out,
     return CA_OK;
 }
 
-// Stream-ordered scratch, released on the same stream when the object dies.
+// One stream-ordered memory pool per device, owned by the library.  Its
+// release threshold is set to the maximum so that memory freed at the end of
+// a call stays mapped for the next one (no OS round trip per call).
+cudaError_t library_pool(cudaMemPool_t *out) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> g(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t p = nullptr;
+        e = cudaMemPoolCreate(&p, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t thr = ~0ull;
+        e = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &thr);
+        if (e != cudaSuccess) return e;
+        pools[dev] = p;
+    }
+    *out = pools[dev];
+    return cudaSuccess;
+}
+
+// Stream-ordered scratch from the library pool, released on the same stream
+// when the object dies.
 struct Scratch {
     cudaStream_t st;
     void *ptrs[8] = {};
@@ -76,11 +107,55 @@ struct Scratch {
         for (int i = 0; i < n; ++i) cudaFreeAsync(ptrs[i], st);
     }
     cudaError_t get(void **p, size_t bytes) {
-        cudaError_t e = cudaMallocAsync(p, bytes, st);
+        cudaMemPool_t pool;
+        cudaError_t e = library_pool(&pool);
+        if (e != cudaSuccess) return e;
+        e = cudaMallocFromPoolAsync(p, bytes, pool, st);
         if (e == cudaSuccess) ptrs[n++] = *p;
         return e;
     }
 };
+
+// The fused one-CTA-per-head kernel handles bf16 heads with L <= 512,
+// K <= 64 and a window radius floor(W/2) <= 16.
+bool fused_eligible(int dtype, const Problem &p) {
+    return dtype == 1 && p.L <= ca::fused::kMaxL && p.K <= ca::fused::kMaxK && p.W / 2 <= ca::fused::kMaxR;
+}
+
+ca_status run_fused(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v, const Problem &p,
+                    __nv_bfloat16 *out, int32_t *assign_out, float *cent_out, int32_t *hist, cudaStream_t st) {
+    using namespace ca;
+    const fused::Layout lay(p.L, p.K, p.W / 2);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    CA_CUDA(cudaGetDevice(&dev));
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        CA_CUDA(cudaFuncSetAttribute(fused::fused_forward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+        attr_set[dev] = true;
+    }
+    fused::Params P;
+    P.q = q;
+    P.k = k;
+    P.v = v;
+    P.out = out;
+    P.assign = assign_out;
+    P.cent = cent_out;
+    P.hist = hist;
+    P.L = p.L;
+    P.K = p.K;
+    P.iters = p.iters;
+    P.r = p.W / 2;
+    P.alpha = p.alpha;
+    P.scale = 1.0f / sqrtf((float)p.d);
+    const double bytes = 4.0 * (double)p.heads() * p.L * kD * sizeof(__nv_bfloat16);
+    {
+        Launch pl("fused_forward", st, bytes);
+        fused::fused_forward_kernel<<<(unsigned)p.heads(), fused::kThreads, lay.total, st>>>(P);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+    return CA_OK;
+}
 
 template <typename T>
 ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *out,
@@ -179,6 +254,9 @@ ca_status dispatch(const void *q, const void *k, const void *v, int dtype, const
     if (((uintptr_t)cent_out & 15u) || ((uintptr_t)assign_out & 3u) || ((uintptr_t)hist & 3u))
         return fail(CA_ERR_INVALID_ARG, "centroids_out must be 16-byte aligned, assign buffers 4-byte aligned");
     cudaStream_t st = (cudaStream_t)stream;
+    if (fused_eligible(dtype, p))
+        return run_fused((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, p,
+                         (__nv_bfloat16 *)out, assign_out, cent_out, hist, st);
     if (dtype == 0)
         return run_forward<float>((const float *)q, (const float *)k, (const float *)v, p, (float *)out,
                                   assign_out, cent_out, hist, st);

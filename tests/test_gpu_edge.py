@@ -96,3 +96,55 @@ def test_invalid_call_launches_nothing_and_status_stays_clean():
     with pytest.raises(ca.ClusterAttnError):
         ca.forward(q, q, q, 4, -1, 4, 0.5)
     ca.sync_status()
+
+
+# Shapes served by the fused one-CTA-per-head kernel (bf16, L <= 512, K <= 64,
+# floor(W/2) <= 16): ragged lengths, K at the 16/32/64 padding boundaries,
+# windows at the radius limit.
+FUSED_CASES = [
+    # L, K, iters, W, alpha, B, H
+    (1, 1, 2, 32, 0.5, 1, 3),
+    (17, 5, 3, 33, 0.4, 2, 2),
+    (64, 16, 0, 2, 0.5, 1, 2),
+    (100, 17, 5, 31, 0.9, 1, 2),
+    (255, 33, 3, 32, 0.5, 2, 1),
+    (256, 64, 3, 16, 0.1, 1, 2),
+    (300, 48, 2, 1, 0.5, 1, 2),
+    (511, 16, 4, 32, 0.5, 2, 2),
+    (512, 64, 5, 33, 0.5, 1, 3),
+]
+
+
+@pytest.mark.parametrize("L,K,iters,W,alpha,B,H", FUSED_CASES)
+def test_fused_path_parity(L, K, iters, W, alpha, B, H):
+    from means_cluster_attention_b200 import _lib
+    w = Workload("fused", B, H, L, 64, K, iters, W, alpha, "bf16", "normal")
+    x = make_inputs(w, seed=L * 7 + K)
+    _lib.profile_start("fused_forward")
+    g = run_gpu(x, "bf16", K, iters, W, alpha, hist=iters > 0)
+    stat = _lib.profile_stop()
+    assert stat.launches == 1, "the fused kernel did not run"
+    ref_out, ref_assign, ref_cent, ref_hist = oracle.forward(
+        x["q64"], x["k64"], x["v64"], K=K, iters=iters, W=W, alpha=alpha, hist=True)
+    if iters > 0:
+        np.testing.assert_array_equal(g["hist"], ref_hist)
+    np.testing.assert_array_equal(g["assign"], ref_assign)
+    np.testing.assert_array_equal(g["cent"], ref_cent)
+    err = float(np.abs(g["out"] - ref_out).max())
+    assert err <= TOL["bf16"], err
+
+
+def test_fused_gmm_forced_ties():
+    # Mixture data plus duplicated rows at the strided start positions: exact
+    # ties, empty and zero centroids inside the fused kernel.
+    from means_cluster_attention_b200 import _lib
+    w = Workload("fused_dup", 2, 3, 400, 64, 40, 4, 32, 0.5, "bf16", "gmm", gmm_components=6,
+                 gmm_std=0.05, dup_frac=0.1)
+    x = make_inputs(w, seed=9)
+    _lib.profile_start("fused_forward")
+    g = run_gpu(x, "bf16", w.K, w.iters, w.W, w.alpha, hist=True)
+    assert _lib.profile_stop().launches == 1
+    _, ref_assign, ref_cent, ref_hist = oracle.forward(x["q64"], x["k64"], x["v64"], K=w.K,
+                                                      iters=w.iters, W=w.W, alpha=w.alpha, hist=True)
+    np.testing.assert_array_equal(g["hist"], ref_hist)
+    np.testing.assert_array_equal(g["cent"], ref_cent)
