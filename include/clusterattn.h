@@ -94,6 +94,26 @@ ca_status ca_forward_host(const void *q, const void *k, const void *v, int dtype
                           int L, int d, int K, int iters, int W, float alpha, void *out,
                           int32_t *assign_out, float *centroids_out, void *stream);
 
+/* Allocation-free form of ca_forward_trace (without the trace; dtype 0 =
+ * fp32, 1 = bf16).  The model cards have no counterpart: this exists for
+ * callers that cannot let a library allocate device memory, such as runtimes
+ * that reserve the GPU for their own allocator up front, or serving loops
+ * that allow no allocation call on their hot path.  The caller passes inputs
+ * and outputs as usual; all other working memory comes from one fixed 16 MiB
+ * device array inside the library (held on every GPU that loads the library,
+ * until the process exits).  Problems whose working memory exceeds 16 MiB
+ * are rejected with CA_ERR_INVALID_ARG and a message giving the size needed
+ * (for example B*H = 384 heads of L = 128 with K = 16 fit; the working
+ * memory grows with B*H*K and, when assign_out is NULL, with B*H*L).  The
+ * call makes no cudaMalloc, cudaMallocAsync or cudaFree call.  Its first call
+ * on each device looks up the array's device address (the device must be
+ * current); make that first call before any stream capture.  Every call
+ * reuses the same array, so calls that overlap on the GPU (on two streams,
+ * or from two threads) race with each other; serialize them. */
+ca_status ca_forward_noalloc(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                             int L, int d, int K, int iters, int W, float alpha, void *out,
+                             int32_t *assign_out, float *centroids_out, void *stream);
+
 /* Synchronizes stream, then reports (and clears) the first device-side error
  * recorded by a kernel of this library on the current device, or a pending
  * CUDA error.  CA_OK when nothing went wrong. */

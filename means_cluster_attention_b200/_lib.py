@@ -25,6 +25,7 @@ SIGNATURES = {
     "ca_forward_bf16": ([_vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp], _ci),
     "ca_forward_trace": ([_vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp, _vp], _ci),
     "ca_forward_host": ([_vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp], _ci),
+    "ca_forward_noalloc": ([_vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp], _ci),
     "ca_sync_status": ([_vp], _ci),
     "ca_status_string": ([_ci], ctypes.c_char_p),
     "ca_last_error": ([], ctypes.c_char_p),

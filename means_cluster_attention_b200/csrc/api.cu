@@ -398,3 +398,163 @@ ca_status ca_profile_stop(ca_kernel_stat *stat) {
 long long ca_launch_count(void) { return ca::profile().launches.load(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point.
+//
+// Some callers cannot let a library allocate device memory: runtimes that
+// reserve the whole GPU for their own allocator up front (a new driver
+// allocation would fail, or fragment memory they manage), and serving loops
+// with hard latency budgets where an allocation call on the hot path is not
+// acceptable.  ca_forward_noalloc serves them: it runs the multi-kernel path
+// with its working memory taken from one fixed array that lives in this file.
+//
+//   - The array holds kNoAllocScratchBytes (16 MiB).  It is part of the
+//     library's device image, so every GPU that loads the library holds it
+//     until the process exits.
+//   - Host code cannot use the array's name as a device address.  The first
+//     call on each device looks up the real address with
+//     cudaGetSymbolAddress, with that device current, and caches it; make
+//     that first call before any stream capture.
+//   - Every call shares the array and it keeps the previous call's contents:
+//     the running sums and counts are cleared on each call before use.  Calls
+//     that overlap on the GPU (two streams, or two threads) race on it.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+ca_status noalloc_scratch_address(unsigned char **out) {
+    static std::mutex mu;
+    static unsigned char *addr[64] = {};
+    int dev = 0;
+    CA_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(CA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> g(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
+        addr[dev] = static_cast<unsigned char *>(p);
+    }
+    *out = addr[dev];
+    return CA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <typename T>
+ca_status run_forward_noalloc(const T *q, const T *k, const T *v, const Problem &p, T *out,
+                              int32_t *assign_out, float *cent_out, cudaStream_t st) {
+    using namespace ca;
+    const int64_t NH = p.heads();
+    const int L = p.L, K = p.K;
+    const float scale = 1.0f / sqrtf((float)p.d);
+    const int n_chunks = (L + kCaChunk - 1) / kCaChunk;
+
+    // Carve the working buffers out of the fixed array.
+    const size_t b_mu = align256(sizeof(float) * NH * K * kD);
+    const size_t b_vc = b_mu;
+    const size_t b_part = align256(sizeof(float) * NH * n_chunks * K * (kD + 2));
+    const size_t b_sums = align256(sizeof(double) * NH * K * kD);
+    const size_t b_cnt = align256(sizeof(int32_t) * NH * K);
+    const size_t b_asg = assign_out ? 0 : align256(sizeof(int32_t) * NH * L);
+    const size_t need = b_mu + b_vc + b_part + b_sums + b_cnt + b_asg;
+    if (need > kNoAllocScratchBytes)
+        return fail(CA_ERR_INVALID_ARG,
+                    "problem needs %zu bytes of working memory; the allocation-free entry point holds %zu",
+                    need, kNoAllocScratchBytes);
+    unsigned char *base = nullptr;
+    ca_status s = noalloc_scratch_address(&base);
+    if (s != CA_OK) return s;
+    float *mu = reinterpret_cast<float *>(base);
+    float *vcent = reinterpret_cast<float *>(base + b_mu);
+    float *part = reinterpret_cast<float *>(base + b_mu + b_vc);
+    double *sums = reinterpret_cast<double *>(base + b_mu + b_vc + b_part);
+    int32_t *counts = reinterpret_cast<int32_t *>(base + b_mu + b_vc + b_part + b_sums);
+    int32_t *assign = assign_out ? assign_out
+                                 : reinterpret_cast<int32_t *>(base + b_mu + b_vc + b_part + b_sums + b_cnt);
+    const double head_bytes = (double)NH * L * kD * sizeof(T);
+
+    {
+        Launch pl("kmeans_init", st, 0.0);
+        kmeans_init_kernel<T><<<(unsigned)NH, 256, 0, st>>>(q, L, K, mu);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+    if (p.iters == 0) {
+        CA_CUDA(cudaMemsetAsync(assign, 0, sizeof(int32_t) * NH * L, st));
+        if (cent_out) CA_CUDA(cudaMemcpyAsync(cent_out, mu, sizeof(float) * NH * K * kD, cudaMemcpyDeviceToDevice, st));
+    }
+    // The array keeps the last call's contents: clear the running sums.
+    CA_CUDA(cudaMemsetAsync(sums, 0, sizeof(double) * NH * K * kD, st));
+    CA_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * NH * K, st));
+
+    const int tokens_per_cta = 1024;
+    const size_t asmem = AssignSmem::bytes(K);
+    CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asmem));
+    const dim3 agrid((L + tokens_per_cta - 1) / tokens_per_cta, (unsigned)NH);
+    for (int t = 0; t < p.iters; ++t) {
+        {
+            Launch pl("kmeans_assign", st, head_bytes);
+            kmeans_assign_kernel<T><<<agrid, kAssignThreads, asmem, st>>>(
+                q, L, K, tokens_per_cta, mu, assign, nullptr, (int64_t)p.iters * L, sums, counts);
+            pl.after();
+        }
+        CA_CUDA(cudaGetLastError());
+        {
+            Launch pl("kmeans_update", st, 0.0);
+            kmeans_update_kernel<<<(unsigned)NH, 256, 0, st>>>(K, sums, counts, mu,
+                                                                t == p.iters - 1 ? cent_out : nullptr);
+            pl.after();
+        }
+        CA_CUDA(cudaGetLastError());
+    }
+    const size_t csmem = centroid_attn_smem_bytes(K);
+    CA_CUDA(cudaFuncSetAttribute(centroid_attn_partial_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem));
+    {
+        Launch pl("centroid_attn", st, 2.0 * head_bytes);
+        centroid_attn_partial_kernel<T><<<dim3(n_chunks, (unsigned)NH), kCaThreads, csmem, st>>>(
+            k, v, L, K, scale, mu, n_chunks, part);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+    {
+        Launch pl("centroid_combine", st, 0.0);
+        centroid_attn_combine_kernel<<<(unsigned)NH, 256, 0, st>>>(K, n_chunks, part, vcent);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+    const size_t wsmem = window_smem_bytes();
+    CA_CUDA(cudaFuncSetAttribute(window_blend_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem));
+    {
+        Launch pl("window_blend", st, 4.0 * head_bytes);
+        window_blend_kernel<T><<<dim3((L + kWinQ - 1) / kWinQ, (unsigned)NH), kWinThreads, wsmem, st>>>(
+            q, k, v, L, K, p.W / 2, scale, p.alpha, vcent, assign, out);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+    return CA_OK;
+}
+
+}  // namespace
+
+extern "C" ca_status ca_forward_noalloc(const void *q, const void *k, const void *v, int dtype, int B,
+                                        int H, int L, int d, int K, int iters, int W, float alpha,
+                                        void *out, int32_t *assign_out, float *centroids_out,
+                                        void *stream) {
+    Problem p{B, H, L, d, K, iters, W, alpha};
+    ca_status s = validate(q, k, v, out, p);
+    if (s != CA_OK) return s;
+    if (((uintptr_t)centroids_out & 15u) || ((uintptr_t)assign_out & 3u))
+        return fail(CA_ERR_INVALID_ARG, "centroids_out must be 16-byte aligned, assign_out 4-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == 0)
+        return run_forward_noalloc<float>((const float *)q, (const float *)k, (const float *)v, p, (float *)out,
+                                          assign_out, centroids_out, st);
+    if (dtype == 1)
+        return run_forward_noalloc<__nv_bfloat16>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
+                                                  (const __nv_bfloat16 *)v, p, (__nv_bfloat16 *)out,
+                                                  assign_out, centroids_out, st);
+    return fail(CA_ERR_INVALID_ARG, "dtype must be 0 (fp32) or 1 (bf16), got %d", dtype);
+}
