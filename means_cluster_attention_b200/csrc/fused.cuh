@@ -2,11 +2,11 @@
 // bf16 inputs.  Every step of the path runs inside this kernel:
 //
 //   Q (resident in shared memory, loaded once)
-//     -> strided init, I Lloyd iterations (distances on tensor cores, exact
-//        argmin, exact fp64 member sums)            [k-means]
-//   K, V (streamed in 64-key tiles through a 2-stage cp.async ring)
-//     -> V_cent = softmax(mu K^T / sqrt(d)) V        [centroid attention]
-//   Q, K, V blocks of 128 queries (second read, from L2)
+//     -> strided init, I Lloyd iterations: distances on tensor cores with an
+//        exact argmin, exact fp64 member sums          [k-means]
+//   K, V (64-key tiles, up to five in flight)
+//     -> V_cent = softmax(mu K^T / sqrt(d)) V           [centroid attention]
+//   K, V blocks of 128 queries + halo (second read, from L2, double buffered)
 //     -> clipped window attention, gather V_cent[c_i], convex blend, store O.
 //
 // Model card "Hooshaai/distilbert-sst2-cluster-attention": Architecture
@@ -25,6 +25,12 @@
 // lowest k with the smallest distance wins.  Centroids that are bitwise
 // copies of a lower-index centroid can never win (their distances are equal
 // and the lower index takes the tie) and are excluded up front.
+//
+// Member sums: tokens are ordered by cluster with a stable counting sort;
+// each warp walks a contiguous slice of the sorted tokens, turning bf16
+// values into doubles with integer operations and adding in fp64.  Those sums are exact for any input
+// whose non-zero magnitudes lie within 2^-27 .. 16, so the centroid
+// mu_k = fp32(sum / max(1, count)) does not depend on the order of the adds.
 #pragma once
 
 #include "common.cuh"
@@ -39,30 +45,38 @@ constexpr int kMaxL = 512;
 constexpr int kMaxK = 64;
 constexpr int kMaxR = 16;
 constexpr int kTile = 64;       // keys per centroid-attention tile
+constexpr int kSlots = 5;       // centroid-attention tiles in flight
 constexpr int kWinBlock = 128;  // queries per window block (8 warps x 16)
 constexpr int kMaxNT = (16 + 2 * kMaxR + 14) / 8;  // key n-tiles per window m-tile
 constexpr float kEps = 1.220703125e-04f;           // 2^-13
 constexpr float kLog2e = 1.4426950408889634f;
 
-struct Layout {
-    int Lp, Kp, r, win_rows;
-    uint32_t q_off, ring_off, mu_off, hi_off, lo_off, vc_off, mm_off, hash_off, c_off, list_off,
-        misc_off, ml_off, total;
+__host__ __device__ inline uint32_t up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+__host__ __device__ inline uint32_t umax(uint32_t a, uint32_t b) { return a > b ? a : b; }
 
-    __host__ __device__ static uint32_t up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+struct Layout {
+    int Lp, Kp, r, nT, win_rows;
+    uint32_t big_off, sums_off, mu_off, hi_off, lo_off, vc_off, mm_off, hash_off, dead_off, c_off,
+        list_off, perm_off, sc_off, table_off, cnt_off, base_off, misc_off, ml_off, win_stage, total;
 
     __host__ __device__ Layout(int L, int K, int r_) {
         Lp = (int)up((uint32_t)L, 64);
         Kp = K <= 16 ? 16 : (K <= 32 ? 32 : 64);
         r = r_;
-        win_rows = (int)up((uint32_t)(kWinBlock + 2 * r + 8), 8);
+        nT = Lp / kTile;
+        const uint32_t wr = up((uint32_t)(kWinBlock + 2 * r + 8), 8);
+        win_rows = (int)(wr < (uint32_t)Lp + 8 ? wr : (uint32_t)Lp + 8);
+        win_stage = 2u * (uint32_t)win_rows * 128u;
         const uint32_t q_bytes = (uint32_t)Lp * 128u;
-        const uint32_t win_bytes = (uint32_t)kWinBlock * 128u + 2u * (uint32_t)win_rows * 128u;
+        const uint32_t sums_bytes = (uint32_t)Kp * 64u * 8u;
+        const uint32_t slots = (uint32_t)(nT < kSlots ? nT : kSlots);
+        uint32_t big = umax(q_bytes + sums_bytes, slots * 2u * kTile * 128u);
+        big = umax(big, 2u * win_stage);
+        big = umax(big, (uint32_t)kWarps * 16u * 64u * 4u);  // centroid-phase combine scratch
         uint32_t o = 0;
-        q_off = o;
-        o += up(q_bytes > win_bytes ? q_bytes : win_bytes, 1024);
-        ring_off = o;
-        o += 2u * 2u * kTile * 128u;  // 2 stages x (K tile, V tile); also combine scratch
+        big_off = o;
+        sums_off = q_bytes;
+        o += up(big, 1024);
         mu_off = o;
         o += up((uint32_t)Kp * 65u * 4u, 128);
         hi_off = o;
@@ -75,10 +89,22 @@ struct Layout {
         o += (uint32_t)Kp * 4u;
         hash_off = o;
         o += (uint32_t)Kp * 4u;
+        cnt_off = o;
+        o += (uint32_t)Kp * 4u;
+        base_off = o;
+        o += (uint32_t)Kp * 4u;
+        dead_off = o;
+        o += up((uint32_t)Kp, 16);
         c_off = o;
+        o += up((uint32_t)Lp, 16);
+        sc_off = o;
         o += up((uint32_t)Lp, 16);
         list_off = o;
         o += up((uint32_t)Lp * 2u, 16);
+        perm_off = o;
+        o += up((uint32_t)Lp * 2u, 16);
+        table_off = o;
+        o += up((uint32_t)(Lp / 32) * (uint32_t)Kp * 2u, 16);
         misc_off = o;
         o += 64;
         ml_off = o;
@@ -97,20 +123,17 @@ struct Params {
     float alpha, scale;
 };
 
-// Row state for the running argmin: smallest value, its index, second value.
+// Running argmin of one row: smallest value, its index, second value.
 struct Best {
     float m1, m2;
     int k1;
 };
 
 __device__ __forceinline__ void best_push(Best &b, float s, int k) {
-    if (s < b.m1) {
-        b.m2 = b.m1;
-        b.m1 = s;
-        b.k1 = k;
-    } else {
-        b.m2 = fminf(b.m2, s);
-    }
+    const bool lt = s < b.m1;
+    b.m2 = fminf(b.m2, fmaxf(b.m1, s));
+    b.k1 = lt ? k : b.k1;
+    b.m1 = fminf(b.m1, s);
 }
 
 __device__ __forceinline__ Best best_merge(const Best &a, const Best &b) {
@@ -134,26 +157,56 @@ __device__ __forceinline__ Best best_quad(Best b) {
     return b;
 }
 
-// Issue the cp.async copies of `rows` rows of a [*, 64] bf16 matrix starting
-// at global row g0 into a swizzled 128-byte-row buffer; rows at or beyond
-// `valid` are zero-filled.
+// cp.async copies of `rows` rows of a [*, 64] bf16 matrix starting at global
+// row g0 into a swizzled 128-byte-row buffer; rows at or beyond `valid` are
+// zero-filled.
 __device__ __forceinline__ void load_rows(uint32_t dst, const __nv_bfloat16 *src, int g0, int rows, int valid) {
     for (int e = threadIdx.x; e < rows * 8; e += kThreads) {
         const int row = e >> 3, ch = e & 7;
-        const int g = g0 + row;
-        const bool ok = g >= 0 && g < valid;
-        const __nv_bfloat16 *s = src + (size_t)(ok ? g : 0) * kD + ch * 8;
+        const int gr = g0 + row;
+        const bool ok = gr >= 0 && gr < valid;
+        const __nv_bfloat16 *s = src + (size_t)(ok ? gr : 0) * kD + ch * 8;
         cp_async16(dst + swz(row, ch), s, ok ? 16 : 0);
     }
+}
+
+// 2^x with the MUFU instruction (relative error about 2^-22; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Exact fp64 value of a bf16 bit pattern (low 16 bits of b) built with
+// integer operations: the 8-bit exponent is rebiased (+896) into the 11-bit
+// field and the 7 fraction bits become the top fraction bits.  Zero and
+// subnormal inputs take the (exact) conversion path.  Inputs are finite.
+__device__ __forceinline__ double bf16_to_f64(uint32_t b) {
+    if ((b & 0x7F80u) == 0u) return (double)__uint_as_float(b << 16);
+    const uint32_t hi = ((b & 0x8000u) << 16) | (((b & 0x7FFFu) << 13) + 0x38000000u);
+    return __hiloint2double((int)hi, 0);
+}
+
+// Both bf16 halves of a 32-bit word as exact doubles, for words whose two
+// exponent fields are non-zero (the caller checks; see bf16_to_f64).
+__device__ __forceinline__ void bf16x2_to_f64_normal(uint32_t w, double &lo, double &hi) {
+    const uint32_t h0 = ((w << 16) & 0x80000000u) | (((w & 0x7FFFu) << 13) + 0x38000000u);
+    const uint32_t h1 = (w & 0x80000000u) | (((w >> 3) & 0x0FFFE000u) + 0x38000000u);
+    lo = __hiloint2double((int)h0, 0);
+    hi = __hiloint2double((int)h1, 0);
+}
+
+__device__ __forceinline__ bool bf16x2_has_zero_exp(uint32_t w) {
+    return ((w & 0x7F80u) == 0u) || ((w & 0x7F800000u) == 0u);
+}
+
 __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const Layout lay(P.L, P.K, P.r);
-    const int L = P.L, K = P.K, Lp = lay.Lp, Kp = lay.Kp;
+    const int L = P.L, K = P.K, Lp = lay.Lp, Kp = lay.Kp, nT = lay.nT;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int64_t head = blockIdx.x;
@@ -162,38 +215,39 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     const __nv_bfloat16 *vh = P.v + head * (int64_t)L * kD;
 
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t q_s = sbase + lay.q_off, ring_s = sbase + lay.ring_off;
+    const uint32_t big_s = sbase + lay.big_off;  // Q during k-means, then K/V staging
     const uint32_t hi_s = sbase + lay.hi_off, lo_s = sbase + lay.lo_off;
-    float *mu = reinterpret_cast<float *>(smem + lay.mu_off);   // [Kp][65]
-    float *vc = reinterpret_cast<float *>(smem + lay.vc_off);   // [Kp][64]
-    float *mm = reinterpret_cast<float *>(smem + lay.mm_off);   // [Kp]
+    unsigned char *qbytes = smem + lay.big_off;
+    float *mu = reinterpret_cast<float *>(smem + lay.mu_off);                     // [Kp][65]
+    float *vc = reinterpret_cast<float *>(smem + lay.vc_off);                     // [Kp][64]
+    float *mm = reinterpret_cast<float *>(smem + lay.mm_off);                     // [Kp]
     uint32_t *hsh = reinterpret_cast<uint32_t *>(smem + lay.hash_off);
-    uint8_t *cs = smem + lay.c_off;                             // [Lp]
+    int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
+    int *base_s = reinterpret_cast<int *>(smem + lay.base_off);
+    double *sums = reinterpret_cast<double *>(smem + lay.big_off + lay.sums_off);  // [Kp][64]
+    uint8_t *dead = smem + lay.dead_off;
+    uint8_t *cs = smem + lay.c_off;                                              // [Lp]
+    uint8_t *sc = smem + lay.sc_off;                                             // [Lp] sorted cluster ids
     uint16_t *list = reinterpret_cast<uint16_t *>(smem + lay.list_off);
+    uint16_t *perm = reinterpret_cast<uint16_t *>(smem + lay.perm_off);
+    int16_t *table = reinterpret_cast<int16_t *>(smem + lay.table_off);           // [Lp/32][Kp]
     int *misc = reinterpret_cast<int *>(smem + lay.misc_off);  // 0 refine count, 1 mm_max, 2 mun_max
     float *ml = reinterpret_cast<float *>(smem + lay.ml_off);
 
-    // ---- prologue: Q, then the first two K/V tiles --------------------------
-    load_rows(q_s, qh, 0, Lp, L);
+    // ---- prologue: Q ------------------------------------------------------
+    load_rows(big_s, qh, 0, Lp, L);
     cp_async_commit();
-    const int nT = Lp / kTile;
-    for (int s = 0; s < 2; ++s) {
-        if (s < nT) {
-            load_rows(ring_s + s * 2 * kTile * 128, kh, s * kTile, kTile, L);
-            load_rows(ring_s + s * 2 * kTile * 128 + kTile * 128, vh, s * kTile, kTile, L);
-        }
-        cp_async_commit();
-    }
     for (int i = threadIdx.x; i < Lp; i += kThreads) cs[i] = i < L ? 0 : 0xFF;
     if (threadIdx.x == 0) misc[0] = 0;
-    cp_async_wait<2>();
+    cp_async_wait<0>();
     __syncthreads();
 
     // |Q_i| for the rows this thread sees in the k-means epilogue.
     const int n_mt = Lp / 16;
-    float qn[kMaxL / 16 / kWarps][2];
+    constexpr int kMtPerWarp = kMaxL / 16 / kWarps;  // 4
+    float qn[kMtPerWarp][2];
 #pragma unroll
-    for (int j = 0; j < kMaxL / 16 / kWarps; ++j) {
+    for (int j = 0; j < kMtPerWarp; ++j) {
         const int mt = warp + j * kWarps;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -202,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                 const int row = mt * 16 + g + 8 * h;
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(smem + lay.q_off + swz(row, 2 * t + c));
+                    const uint4 w = *reinterpret_cast<const uint4 *>(qbytes + swz(row, 2 * t + c));
                     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -217,8 +271,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         }
     }
 
-    // ---- centroid finalisation: fp32 row -> hi/lo bf16, |mu|^2, hash -------
-    // Called by one warp per centroid, lane holding coordinates 2*lane, 2*lane+1.
+    // One warp per centroid row: lane holds coordinates 2*lane, 2*lane+1.
     auto finalize_row = [&](int kk, float x0, float x1) {
         mu[kk * 65 + 2 * lane] = x0;
         mu[kk * 65 + 2 * lane + 1] = x1;
@@ -227,12 +280,15 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         const __nv_bfloat16 l1 = __float2bfloat16_rn(x1 - __bfloat162float(h1));
         const uint32_t off = swz(kk, lane >> 2) + (lane & 3) * 4;
         __nv_bfloat162 hv, lv;
-        hv.x = h0; hv.y = h1;
-        lv.x = l0; lv.y = l1;
+        hv.x = h0;
+        hv.y = h1;
+        lv.x = l0;
+        lv.y = l1;
         *reinterpret_cast<__nv_bfloat162 *>(smem + lay.hi_off + off) = hv;
         *reinterpret_cast<__nv_bfloat162 *>(smem + lay.lo_off + off) = lv;
         float sq = fmaf(x0, x0, x1 * x1);
         uint32_t hv32 = (__float_as_uint(x0) * 0x9E3779B1u) ^ (__float_as_uint(x1) * 0x85EBCA77u + (uint32_t)lane * 0xC2B2AE3Du);
+#pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             sq += __shfl_xor_sync(0xffffffffu, sq, o);
             hv32 += __shfl_xor_sync(0xffffffffu, hv32, o);
@@ -243,41 +299,50 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         }
     };
 
-    // After every centroid row is final: mark duplicates and padding with
-    // +inf, and take max |mu|, max |mu|^2 over the live centroids.
+    // After every centroid row is final: mark padding and bitwise duplicates
+    // of a lower-index centroid dead (+inf), and take max |mu|^2, max |mu|
+    // over the live centroids.
     auto finalize_set = [&]() {
         __syncthreads();
         const int kk = threadIdx.x;
-        bool dead = true;
         if (kk < Kp) {
-            dead = kk >= K;
-            for (int a = 0; a < kk && !dead; ++a) {
+            bool dd = kk >= K;
+            for (int a = 0; a < kk && !dd; ++a) {
                 if (hsh[a] != hsh[kk]) continue;
                 bool same = true;
                 for (int j = 0; j < kD && same; ++j)
                     same = __float_as_uint(mu[a * 65 + j]) == __float_as_uint(mu[kk * 65 + j]);
-                dead = same;
+                dd = same;
             }
-            if (!dead) {
-                atomicMax(&misc[1], __float_as_int(mm[kk]));
-                atomicMax(&misc[2], __float_as_int(sqrtf(mm[kk])));
+            dead[kk] = dd ? 1 : 0;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            float mx = 0.f;
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                const int k2 = lane + 32 * s;
+                if (k2 < Kp) {
+                    if (dead[k2]) mm[k2] = INFINITY;
+                    else mx = fmaxf(mx, mm[k2]);
+                }
+            }
+            mx = warp_max(mx);
+            if (lane == 0) {
+                misc[1] = __float_as_int(mx);
+                misc[2] = __float_as_int(sqrtf(mx));
+                misc[0] = 0;
             }
         }
         __syncthreads();
-        if (kk < Kp && dead) mm[kk] = INFINITY;
-        __syncthreads();
     };
 
-    // ---- strided init: mu_k = Q[floor(k L / K)] -----------------------------
-    if (threadIdx.x == 0) {
-        misc[1] = 0;
-        misc[2] = 0;
-    }
+    // ---- strided init: mu_k = Q[floor(k L / K)] -------------------------------
     for (int kk = warp; kk < Kp; kk += kWarps) {
         float x0 = 0.f, x1 = 0.f;
         if (kk < K) {
             const int row = (int)(((int64_t)kk * L) / K);
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(smem + lay.q_off + swz(row, lane >> 2) + (lane & 3) * 4);
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(qbytes + swz(row, lane >> 2) + (lane & 3) * 4);
             x0 = bf16lo(w);
             x1 = bf16hi(w);
         }
@@ -285,90 +350,128 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     }
     finalize_set();
 
-    // ---- Lloyd iterations ----------------------------------------------------
+    const int nch = Lp / 32;
+    // ---- Lloyd iterations -----------------------------------------------------
     for (int it = 0; it < P.iters; ++it) {
         const float mm_max = __int_as_float(misc[1]), mun_max = __int_as_float(misc[2]);
-        // assignment: tensor-core distances + certified argmin
+        // (1) assignment: tensor-core distances + certified argmin, two m-tiles at a time
 #pragma unroll
-        for (int j = 0; j < kMaxL / 16 / kWarps; ++j) {
-            const int mt = warp + j * kWarps;
-            if (mt >= n_mt) break;
-            uint32_t a[4][4];
+        for (int jp = 0; jp < kMtPerWarp; jp += 2) {
+            const int mt0 = warp + jp * kWarps, mt1 = mt0 + kWarps;
+            if (mt0 >= n_mt) break;
+            const bool two = mt1 < n_mt;
+            uint32_t a0[4][4], a1[4][4];
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const int m = lane >> 3;
-                const int row = mt * 16 + (lane & 7) + ((m & 1) ? 8 : 0);
-                ldmatrix_x4(a[ks], q_s + swz(row, 2 * ks + (m >> 1)));
+                const int rr = (lane & 7) + ((m & 1) ? 8 : 0);
+                ldmatrix_x4(a0[ks], big_s + swz(mt0 * 16 + rr, 2 * ks + (m >> 1)));
+                if (two) ldmatrix_x4(a1[ks], big_s + swz(mt1 * 16 + rr, 2 * ks + (m >> 1)));
+                else a1[ks][0] = a1[ks][1] = a1[ks][2] = a1[ks][3] = 0u;
             }
-            Best b0{INFINITY, INFINITY, 0}, b1{INFINITY, INFINITY, 0};
+            Best b[2][2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) b[u][h] = Best{INFINITY, INFINITY, 0};
             for (int nt = 0; nt < Kp / 8; ++nt) {
-                float ch[4] = {0.f, 0.f, 0.f, 0.f}, cl[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t bh[2][4], bl[2][4];
 #pragma unroll
                 for (int kp = 0; kp < 2; ++kp) {
-                    uint32_t bh[4], bl[4];
                     const int row = nt * 8 + (lane & 7);
                     const int chunk = 4 * kp + (lane >> 3);
-                    ldmatrix_x4(bh, hi_s + swz(row, chunk));
-                    ldmatrix_x4(bl, lo_s + swz(row, chunk));
-                    mma_16816(ch, a[2 * kp], bh[0], bh[1]);
-                    mma_16816(ch, a[2 * kp + 1], bh[2], bh[3]);
-                    mma_16816(cl, a[2 * kp], bl[0], bl[1]);
-                    mma_16816(cl, a[2 * kp + 1], bl[2], bl[3]);
+                    ldmatrix_x4(bh[kp], hi_s + swz(row, chunk));
+                    ldmatrix_x4(bl[kp], lo_s + swz(row, chunk));
+                }
+                float acc[2][2][4];
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int s = 0; s < 2; ++s)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[u][s][e] = 0.f;
+#pragma unroll
+                for (int kp = 0; kp < 2; ++kp) {
+                    mma_16816(acc[0][0], a0[2 * kp], bh[kp][0], bh[kp][1]);
+                    mma_16816(acc[0][1], a0[2 * kp], bl[kp][0], bl[kp][1]);
+                    mma_16816(acc[1][0], a1[2 * kp], bh[kp][0], bh[kp][1]);
+                    mma_16816(acc[1][1], a1[2 * kp], bl[kp][0], bl[kp][1]);
+                    mma_16816(acc[0][0], a0[2 * kp + 1], bh[kp][2], bh[kp][3]);
+                    mma_16816(acc[0][1], a0[2 * kp + 1], bl[kp][2], bl[kp][3]);
+                    mma_16816(acc[1][0], a1[2 * kp + 1], bh[kp][2], bh[kp][3]);
+                    mma_16816(acc[1][1], a1[2 * kp + 1], bl[kp][2], bl[kp][3]);
                 }
                 const int c0 = nt * 8 + 2 * t;
                 const float m0 = mm[c0], m1 = mm[c0 + 1];
-                best_push(b0, fmaf(-2.f, ch[0] + cl[0], m0), c0);
-                best_push(b0, fmaf(-2.f, ch[1] + cl[1], m1), c0 + 1);
-                best_push(b1, fmaf(-2.f, ch[2] + cl[2], m0), c0);
-                best_push(b1, fmaf(-2.f, ch[3] + cl[3], m1), c0 + 1);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    best_push(b[u][0], fmaf(-2.f, acc[u][0][0] + acc[u][1][0], m0), c0);
+                    best_push(b[u][0], fmaf(-2.f, acc[u][0][1] + acc[u][1][1], m1), c0 + 1);
+                    best_push(b[u][1], fmaf(-2.f, acc[u][0][2] + acc[u][1][2], m0), c0);
+                    best_push(b[u][1], fmaf(-2.f, acc[u][0][3] + acc[u][1][3], m1), c0 + 1);
+                }
             }
-            b0 = best_quad(b0);
-            b1 = best_quad(b1);
-            if (t == 0) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int mt = u ? mt1 : mt0;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const Best &b = h ? b1 : b0;
+                    const Best bb = best_quad(b[u][h]);
                     const int row = mt * 16 + g + 8 * h;
-                    if (row < L) {
-                        const float E = kEps * fmaf(qn[j][h], mun_max, mm_max);
-                        cs[row] = (uint8_t)b.k1;
-                        if (b.m2 <= b.m1 + 2.f * E) list[atomicAdd(&misc[0], 1)] = (uint16_t)row;
+                    if (t == 0 && (u == 0 || two) && row < L) {
+                        const float E = kEps * fmaf(qn[jp + u][h], mun_max, mm_max);
+                        cs[row] = (uint8_t)bb.k1;
+                        if (bb.m2 <= bb.m1 + 2.f * E) list[atomicAdd(&misc[0], 1)] = (uint16_t)row;
                     }
                 }
             }
         }
         __syncthreads();
-        // exact re-measure of ambiguous tokens, one warp per token
+        // (2) exact re-measure of ambiguous tokens, one warp per token
         const int n_ref = misc[0];
         for (int e = warp; e < n_ref; e += kWarps) {
             const int row = list[e];
-            double qq = 0.0;
-            double qm[2] = {0.0, 0.0}, m2[2] = {0.0, 0.0};
-            for (int j = 0; j < kD; ++j) {
-                const uint16_t bits = *reinterpret_cast<const uint16_t *>(smem + lay.q_off + swz(row, j >> 3) + (j & 7) * 2);
-                const double qj = (double)__uint_as_float((uint32_t)bits << 16);
-                qq = __dadd_rn(qq, __dmul_rn(qj, qj));
+            double qq = 0.0, qm0 = 0.0, qm1 = 0.0, m20 = 0.0, m21 = 0.0;
+            const int k0 = lane, k1 = lane + 32;
+            const bool v0 = k0 < Kp, v1 = k1 < Kp;
+#pragma unroll 2
+            for (int jb = 0; jb < kD; jb += 8) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(qbytes + swz(row, jb >> 3));
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                double qj[8], mj0[8], mj1[8];
 #pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    const int kk = lane + 32 * s;
-                    const double mj = kk < Kp ? (double)mu[kk * 65 + j] : 0.0;
-                    qm[s] = __dadd_rn(qm[s], __dmul_rn(qj, mj));
-                    m2[s] = __dadd_rn(m2[s], __dmul_rn(mj, mj));
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    qj[2 * e2] = bf16_to_f64(ws[e2] & 0xffffu);
+                    qj[2 * e2 + 1] = bf16_to_f64(ws[e2] >> 16);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    mj0[u] = v0 ? (double)mu[k0 * 65 + jb + u] : 0.0;
+                    mj1[u] = v1 ? (double)mu[k1 * 65 + jb + u] : 0.0;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    qq = __dadd_rn(qq, __dmul_rn(qj[u], qj[u]));
+                    qm0 = __dadd_rn(qm0, __dmul_rn(qj[u], mj0[u]));
+                    m20 = __dadd_rn(m20, __dmul_rn(mj0[u], mj0[u]));
+                    qm1 = __dadd_rn(qm1, __dmul_rn(qj[u], mj1[u]));
+                    m21 = __dadd_rn(m21, __dmul_rn(mj1[u], mj1[u]));
                 }
             }
             double bd = INFINITY;
             int bk = 0x7fffffff;
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                const int kk = lane + 32 * s;
-                if (kk < Kp && !(mm[kk] == INFINITY)) {
-                    const double D = __dsub_rn(__dadd_rn(qq, m2[s]), __dmul_rn(2.0, qm[s]));
-                    if (D < bd) {
-                        bd = D;
-                        bk = kk;
-                    }
+            if (v0 && !dead[k0]) {
+                bd = __dsub_rn(__dadd_rn(qq, m20), __dmul_rn(2.0, qm0));
+                bk = k0;
+            }
+            if (v1 && !dead[k1]) {
+                const double D = __dsub_rn(__dadd_rn(qq, m21), __dmul_rn(2.0, qm1));
+                if (D < bd) {
+                    bd = D;
+                    bk = k1;
                 }
             }
+#pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 const double od = __shfl_xor_sync(0xffffffffu, bd, o);
                 const int ok = __shfl_xor_sync(0xffffffffu, bk, o);
@@ -390,45 +493,124 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
             int32_t *hrow = P.hist + (head * P.iters + it) * (int64_t)L;
             for (int i = threadIdx.x; i < L; i += kThreads) hrow[i] = cs[i];
         }
-        if (threadIdx.x == 0) {
-            misc[0] = 0;
-            misc[1] = 0;
-            misc[2] = 0;
+        // (3) stable counting sort of the tokens by cluster
+        for (int i = threadIdx.x; i < nch * Kp; i += kThreads) table[i] = 0;
+        __syncthreads();
+        int my_c[2], my_rank[2];
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            const int ch = warp + s * kWarps;
+            my_c[s] = 0xFF;
+            my_rank[s] = 0;
+            if (ch < nch) {
+                const int c = cs[ch * 32 + lane];
+                const unsigned peers = __match_any_sync(0xffffffffu, c);
+                my_c[s] = c;
+                my_rank[s] = __popc(peers & ((1u << lane) - 1u));
+                if (c != 0xFF && lane == __ffs(peers) - 1) table[ch * Kp + c] = (int16_t)__popc(peers);
+            }
         }
-        // update: exact fp64 member sums, one warp per cluster
-        const bool last = it == P.iters - 1;
-        for (int kk = warp; kk < Kp; kk += kWarps) {
-            double s0[4] = {0.0, 0.0, 0.0, 0.0}, s1[4] = {0.0, 0.0, 0.0, 0.0};
-            int cnt = 0;
-            if (kk < K) {
-                for (int base = 0; base < Lp; base += 32) {
-                    uint32_t m = __ballot_sync(0xffffffffu, cs[base + lane] == kk);
-                    cnt += __popc(m);
-                    while (m) {
-                        int rows[4];
+        __syncthreads();
+        if (threadIdx.x < Kp) {
+            int run = 0;
+            for (int ch = 0; ch < nch; ++ch) {
+                const int v = table[ch * Kp + threadIdx.x];
+                table[ch * Kp + threadIdx.x] = (int16_t)run;
+                run += v;
+            }
+            cnt_s[threadIdx.x] = run;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int c0 = lane < Kp ? cnt_s[lane] : 0, c1 = lane + 32 < Kp ? cnt_s[lane + 32] : 0;
+            int s0 = c0, s1 = c1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int x0 = __shfl_up_sync(0xffffffffu, s0, o), x1 = __shfl_up_sync(0xffffffffu, s1, o);
+                if (lane >= o) {
+                    s0 += x0;
+                    s1 += x1;
+                }
+            }
+            const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
+            if (lane < Kp) base_s[lane] = s0 - c0;
+            if (lane + 32 < Kp) base_s[lane + 32] = tot0 + s1 - c1;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            const int ch = warp + s * kWarps;
+            if (ch < nch && my_c[s] != 0xFF) {
+                const int pos = base_s[my_c[s]] + table[ch * Kp + my_c[s]] + my_rank[s];
+                perm[pos] = (uint16_t)(ch * 32 + lane);
+                sc[pos] = (uint8_t)my_c[s];
+            }
+        }
+        __syncthreads();
+        // (4) exact member sums: each warp walks a contiguous slice of the
+        // sorted tokens run by run (one cluster per run), lane holding
+        // coordinates 2*lane and 2*lane+1, four independent accumulators; a
+        // run's sum is added into the cluster's row with an (exact) fp64
+        // shared-memory atomic, so runs split between warps combine exactly.
+        for (int i = threadIdx.x; i < Kp * kD; i += kThreads) sums[i] = 0.0;
+        __syncthreads();
+        {
+            const int seg = (L + kWarps - 1) / kWarps;
+            const int p1 = min(L, (warp + 1) * seg);
+            int p = warp * seg;
+            while (p < p1) {
+                const int c = sc[p];
+                double s0[4] = {0.0, 0.0, 0.0, 0.0}, s1[4] = {0.0, 0.0, 0.0, 0.0};
+                for (;;) {
+                    const int q = p + lane;
+                    const unsigned same = __ballot_sync(0xffffffffu, q < p1 && sc[q] == c);
+                    const int n = __ffs(~same) ? __ffs(~same) - 1 : 32;
+                    const int rowl = (lane < n) ? perm[p + lane] : 0;
+                    for (int j = 0; j < n; j += 4) {
+                        uint32_t w[4];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            if (m) {
-                                rows[u] = base + __ffs(m) - 1;
-                                m &= m - 1;
-                            } else {
-                                rows[u] = -1;
-                            }
+                            const int rr = __shfl_sync(0xffffffffu, rowl, (j + u) & 31);
+                            w[u] = (j + u < n) ? *reinterpret_cast<const uint32_t *>(qbytes + swz(rr, lane >> 2) + (lane & 3) * 4) : 0u;
                         }
+                        bool slow = false;
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            if (rows[u] >= 0) {
-                                const uint32_t w = *reinterpret_cast<const uint32_t *>(smem + lay.q_off + swz(rows[u], lane >> 2) + (lane & 3) * 4);
-                                s0[u] += (double)bf16lo(w);
-                                s1[u] += (double)bf16hi(w);
+                        for (int u = 0; u < 4; ++u) slow |= (j + u < n) && bf16x2_has_zero_exp(w[u]);
+                        if (__any_sync(0xffffffffu, slow)) {
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                if (j + u < n) {
+                                    s0[u] += bf16_to_f64(w[u] & 0xffffu);
+                                    s1[u] += bf16_to_f64(w[u] >> 16);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                if (j + u < n) {
+                                    double d0, d1;
+                                    bf16x2_to_f64_normal(w[u], d0, d1);
+                                    s0[u] += d0;
+                                    s1[u] += d1;
+                                }
                             }
                         }
                     }
+                    p += n;
+                    if (n < 32) break;
                 }
+                atomicAdd(&sums[c * kD + 2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
+                atomicAdd(&sums[c * kD + 2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
             }
+        }
+        __syncthreads();
+        // (5) mu_k = fp32(sum_k / max(1, count_k)), one warp per centroid
+        const bool last = it == P.iters - 1;
+        for (int kk = warp; kk < Kp; kk += kWarps) {
+            const int cnt = kk < K ? cnt_s[kk] : 0;
             const double den = (double)(cnt > 1 ? cnt : 1);
-            const float x0 = __double2float_rn(((s0[0] + s0[1]) + (s0[2] + s0[3])) / den);
-            const float x1 = __double2float_rn(((s1[0] + s1[1]) + (s1[2] + s1[3])) / den);
+            const float x0 = kk < K ? __double2float_rn(sums[kk * kD + 2 * lane] / den) : 0.f;
+            const float x1 = kk < K ? __double2float_rn(sums[kk * kD + 2 * lane + 1] / den) : 0.f;
             finalize_row(kk, x0, x1);
             if (last && P.cent && kk < K) {
                 float2 *dst = reinterpret_cast<float2 *>(P.cent + (head * K + kk) * kD);
@@ -444,12 +626,21 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         for (int i = threadIdx.x; i < L; i += kThreads) P.assign[head * L + i] = cs[i];
     }
 
-    // ---- centroid attention over streamed K/V tiles --------------------------
+    // ---- centroid attention over K/V tiles, up to kSlots in flight ------------
     const int n_cm = Kp / 16;          // centroid m-tiles: 1, 2 or 4
     const int G = kWarps / n_cm;       // warps sharing one m-tile: 8, 4 or 2
     const int cm = warp / G, kb = warp % G;
     const int keys_w = kTile / G;      // keys per warp per tile: 8, 16 or 32
     const float csc = P.scale * kLog2e;
+    __syncthreads();  // Q is no longer read: the big region becomes K/V slots
+    for (int s = 0; s < kSlots; ++s) {
+        if (s < nT) {
+            const uint32_t slot = big_s + s * 2 * kTile * 128;
+            load_rows(slot, kh, s * kTile, kTile, L);
+            load_rows(slot + kTile * 128, vh, s * kTile, kTile, L);
+        }
+        cp_async_commit();
+    }
     uint32_t ahi[4][4], alo[4][4];
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
@@ -466,9 +657,9 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     float rm[2] = {-INFINITY, -INFINITY}, rl[2] = {0.f, 0.f};
 
     for (int tt = 0; tt < nT; ++tt) {
-        cp_async_wait<1>();
+        cp_async_wait<kSlots - 1>();
         __syncthreads();
-        const uint32_t kt = ring_s + (tt & 1) * 2 * kTile * 128;
+        const uint32_t kt = big_s + (tt % kSlots) * 2 * kTile * 128;
         const uint32_t vt = kt + kTile * 128;
         float sacc[4][4];
 #pragma unroll
@@ -489,16 +680,14 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                 mma_16816(sacc[n], alo[2 * kp + 1], bk[2], bk[3]);
             }
         }
-        // online softmax over this warp's keys of the tile
         float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
             if (n * 8 >= keys_w) break;
             const int key = tt * kTile + kb * keys_w + n * 8 + 2 * t;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int e = 0; e < 4; ++e)
                 if (key + (e & 1) >= L) sacc[n][e] = -INFINITY;
-            }
             tmax[0] = fmaxf(tmax[0], fmaxf(sacc[n][0], sacc[n][1]));
             tmax[1] = fmaxf(tmax[1], fmaxf(sacc[n][2], sacc[n][3]));
         }
@@ -508,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
             tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 1));
             tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 2));
             const float mn = fmaxf(rm[h], tmax[h]);
-            corr[h] = (mn == -INFINITY) ? 1.f : exp2f((rm[h] - mn) * csc);
+            corr[h] = (mn == -INFINITY) ? 1.f : ex2((rm[h] - mn) * csc);
             rm[h] = mn;
             rl[h] *= corr[h];
         }
@@ -522,19 +711,19 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         uint32_t pa[4][2];
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
+            pa[n][0] = pa[n][1] = 0u;
             if (n * 8 >= keys_w) break;
             float p[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float mh = rm[e >> 1];
-                p[e] = (mh == -INFINITY) ? 0.f : exp2f((sacc[n][e] - mh) * csc);
+                p[e] = (mh == -INFINITY) ? 0.f : ex2((sacc[n][e] - mh) * csc);
             }
             rl[0] += p[0] + p[1];
             rl[1] += p[2] + p[3];
             pa[n][0] = pack_bf16(p[0], p[1]);
             pa[n][1] = pack_bf16(p[2], p[3]);
         }
-        // O += P V
         if (keys_w == 8) {
             const int key0 = kb * keys_w;
 #pragma unroll
@@ -561,16 +750,16 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
             }
         }
         __syncthreads();
-        if (tt + 2 < nT) {
-            load_rows(kt, kh, (tt + 2) * kTile, kTile, L);
-            load_rows(vt, vh, (tt + 2) * kTile, kTile, L);
+        if (tt + kSlots < nT) {
+            load_rows(kt, kh, (tt + kSlots) * kTile, kTile, L);
+            load_rows(vt, vh, (tt + kSlots) * kTile, kTile, L);
         }
         cp_async_commit();
     }
     cp_async_wait<0>();
-    // combine the G partial states of each centroid m-tile (ring reused)
+    // combine the G partial states of each centroid m-tile (big region reused)
     {
-        float *part = reinterpret_cast<float *>(smem + lay.ring_off);  // [warp][16][64]
+        float *part = reinterpret_cast<float *>(smem + lay.big_off);  // [warp][16][64]
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             rl[h] += __shfl_xor_sync(0xffffffffu, rl[h], 1);
@@ -601,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
             float num = 0.f, den = 0.f;
             for (int w = mt * G; w < mt * G + G; ++w) {
                 const float mw = ml[(w * 16 + rr) * 2];
-                const float f = (mw == -INFINITY) ? 0.f : exp2f((mw - M) * csc);
+                const float f = (mw == -INFINITY) ? 0.f : ex2((mw - M) * csc);
                 den = fmaf(ml[(w * 16 + rr) * 2 + 1], f, den);
                 num = fmaf(part[(w * 16 + rr) * 64 + col], f, num);
             }
@@ -610,32 +799,54 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         __syncthreads();
     }
 
-    // ---- window attention + gather + blend, 128 queries per block ------------
+    // ---- window attention + gather + blend: blocks of 128 queries, K/V
+    // double buffered, Q fragments straight from global memory (L2) ---------
     const int r = P.r;
-    const uint32_t qb_s = q_s, kw_s = q_s + kWinBlock * 128, vw_s = kw_s + lay.win_rows * 128;
-    for (int qb = 0; qb < L; qb += kWinBlock) {
-        const int ks0 = max(0, qb - r) & ~7;
-        const int ke = min(L - 1, qb + kWinBlock - 1 + r);
-        const int nrows = (ke - ks0 + 1 + 7) & ~7;
-        load_rows(qb_s, qh, qb, kWinBlock, L);
-        load_rows(kw_s, kh, ks0, nrows, ke + 1);
-        load_rows(vw_s, vh, ks0, nrows, ke + 1);
+    const int nblk = (L + kWinBlock - 1) / kWinBlock;
+    auto issue_block = [&](int b) {
+        if (b < nblk) {
+            const int qb = b * kWinBlock;
+            const int ks0 = max(0, qb - r) & ~7;
+            const int ke = min(L - 1, qb + kWinBlock - 1 + r);
+            const int nrows = (ke - ks0 + 1 + 7) & ~7;
+            const uint32_t st = big_s + (b & 1) * lay.win_stage;
+            load_rows(st, kh, ks0, nrows, ke + 1);
+            load_rows(st + lay.win_rows * 128, vh, ks0, nrows, ke + 1);
+        }
         cp_async_commit();
-        cp_async_wait<0>();
-        __syncthreads();
-        const int i0 = qb + warp * 16;
-        if (i0 < L) {
-            uint32_t a[4][4];
+    };
+    issue_block(0);
+    issue_block(1);
+    __nv_bfloat16 *oh = P.out + head * (int64_t)L * kD;
+    // Q fragments of this warp's 16 rows of a block, read from global memory
+    // (L2); fetched one block ahead.
+    uint32_t a[4][4];
+    auto fetch_q = [&](int b) {
+        const int i0b = b * kWinBlock + warp * 16;
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const int m = lane >> 3;
-                const int row = warp * 16 + (lane & 7) + ((m & 1) ? 8 : 0);
-                ldmatrix_x4(a[ks], qb_s + swz(row, 2 * ks + (m >> 1)));
+        for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int row = i0b + g + ((e & 1) ? 8 : 0);
+                const int col = 16 * ks + 2 * t + ((e & 2) ? 8 : 0);
+                a[ks][e] = (b < nblk && row < L) ? __ldg(reinterpret_cast<const unsigned int *>(qh + (int64_t)row * kD + col)) : 0u;
             }
+        }
+    };
+    fetch_q(0);
+    for (int b = 0; b < nblk; ++b) {
+        const int qb = b * kWinBlock;
+        const int ks0 = max(0, qb - r) & ~7;
+        const int i0 = qb + warp * 16;
+        cp_async_wait<1>();
+        __syncthreads();
+        const uint32_t kw_s = big_s + (b & 1) * lay.win_stage;
+        const uint32_t vw_s = kw_s + lay.win_rows * 128;
+        if (i0 < L) {
             const int kst = max(0, i0 - r) & ~7;
             const int kend = min(L - 1, i0 + 15 + r);
             const int nt = (kend - kst) / 8 + 1;
-            const int lr0 = kst - ks0;  // local row of the first key
+            const int lr0 = kst - ks0;
             float sacc[kMaxNT][4];
 #pragma unroll
             for (int n = 0; n < kMaxNT; ++n) {
@@ -681,7 +892,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float mh = mx[e >> 1];
-                        p[e] = (mh == -INFINITY) ? 0.f : exp2f((sacc[n][e] - mh) * csc);
+                        p[e] = (mh == -INFINITY) ? 0.f : ex2((sacc[n][e] - mh) * csc);
                     }
                     sum[0] += p[0] + p[1];
                     sum[1] += p[2] + p[3];
@@ -721,7 +932,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                     }
                 }
             }
-            // gather + blend, staged into this warp's own Q rows
+            // gather + blend, stored straight to global memory
             const float inv0 = sum[0] > 0.f ? 1.f / sum[0] : 0.f, inv1 = sum[1] > 0.f ? 1.f / sum[1] : 0.f;
             const int ia = i0 + g, ib = i0 + g + 8;
             const int ca = ia < L ? cs[ia] : 0, cb = ib < L ? cs[ib] : 0;
@@ -729,28 +940,23 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
 #pragma unroll
             for (int d = 0; d < 8; ++d) {
                 const int col = 8 * d + 2 * t;
-                const float y0 = be * vc[ca * kD + col] + al * (oacc[d][0] * inv0);
-                const float y1 = be * vc[ca * kD + col + 1] + al * (oacc[d][1] * inv0);
-                const float y2 = be * vc[cb * kD + col] + al * (oacc[d][2] * inv1);
-                const float y3 = be * vc[cb * kD + col + 1] + al * (oacc[d][3] * inv1);
-                *reinterpret_cast<uint32_t *>(smem + lay.q_off + swz(warp * 16 + g, d) + 4 * t) = pack_bf16(y0, y1);
-                *reinterpret_cast<uint32_t *>(smem + lay.q_off + swz(warp * 16 + g + 8, d) + 4 * t) = pack_bf16(y2, y3);
-            }
-            __syncwarp();
-            __nv_bfloat16 *oh = P.out + head * (int64_t)L * kD;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = lane + 32 * u;
-                const int rr = e >> 3, ch = e & 7;
-                const int i = i0 + rr;
-                if (i < L) {
-                    const uint4 val = *reinterpret_cast<const uint4 *>(smem + lay.q_off + swz(warp * 16 + rr, ch));
-                    *reinterpret_cast<uint4 *>(oh + (int64_t)i * kD + ch * 8) = val;
+                if (ia < L) {
+                    const float y0 = be * vc[ca * kD + col] + al * (oacc[d][0] * inv0);
+                    const float y1 = be * vc[ca * kD + col + 1] + al * (oacc[d][1] * inv0);
+                    *reinterpret_cast<uint32_t *>(oh + (int64_t)ia * kD + col) = pack_bf16(y0, y1);
+                }
+                if (ib < L) {
+                    const float y2 = be * vc[cb * kD + col] + al * (oacc[d][2] * inv1);
+                    const float y3 = be * vc[cb * kD + col + 1] + al * (oacc[d][3] * inv1);
+                    *reinterpret_cast<uint32_t *>(oh + (int64_t)ib * kD + col) = pack_bf16(y2, y3);
                 }
             }
         }
+        fetch_q(b + 1);
         __syncthreads();
+        issue_block(b + 2);
     }
+    cp_async_wait<0>();
 }
 
 }  // namespace fused
