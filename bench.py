@@ -33,8 +33,8 @@ UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "l512_bf16"
 FALLBACK_HBM_GBS = 6650.0
 # Kernel whose launches the roofline object reports, per workload.
-DOMINANT = {"small_f32": "kmeans_assign", "card_gmm_f32": "kmeans_assign", "l512_bf16": "fused_forward",
-            "l4k_gmm_bf16": "kmeans_assign", "l32k_dup_bf16": "kmeans_assign"}
+DOMINANT = {"small_f32": "window_blend", "card_gmm_f32": "window_blend", "l512_bf16": "fused_forward",
+            "l4k_gmm_bf16": "tiled_assign", "l32k_dup_bf16": "tiled_assign"}
 
 
 def workload_desc(w) -> dict:

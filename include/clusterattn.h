@@ -135,8 +135,12 @@ const char *ca_version(void);
  * stream.  ca_profile_stop waits for those events and fills *stat with the
  * number of timed launches, their summed duration and their summed
  * algorithmic HBM bytes (one read of every input and one write of every
- * output the kernel must touch).  Kernel names: "kmeans_init",
- * "kmeans_assign", "kmeans_update", "centroid_attn", "centroid_combine",
+ * output the kernel must touch).  Kernel names: the fused one-CTA-per-head
+ * kernel (bf16, L <= 512, K <= 64, floor(W/2) <= 16) is "fused_forward";
+ * the tiled bf16 path (K <= 64, floor(W/2) <= 128) launches "tiled_init",
+ * "tiled_assign", "tiled_update", "tiled_centroid", "tiled_combine" and
+ * "tiled_window"; every other case runs the general path "kmeans_init",
+ * "kmeans_assign", "kmeans_update", "centroid_attn", "centroid_combine" and
  * "window_blend". */
 typedef struct {
     long long launches;

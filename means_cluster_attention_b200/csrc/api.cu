@@ -15,6 +15,7 @@
 #include "kmeans.cuh"
 #include "attention.cuh"
 #include "fused.cuh"
+#include "tiled.cuh"
 #include "profile.cuh"
 
 namespace {
@@ -100,7 +101,7 @@ cudaError_t library_pool(cudaMemPool_t *out) {
 // when the object dies.
 struct Scratch {
     cudaStream_t st;
-    void *ptrs[8] = {};
+    void *ptrs[16] = {};
     int n = 0;
     explicit Scratch(cudaStream_t s) : st(s) {}
     ~Scratch() {
@@ -151,6 +152,151 @@ ca_status run_fused(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     {
         Launch pl("fused_forward", st, bytes);
         fused::fused_forward_kernel<<<(unsigned)p.heads(), fused::kThreads, lay.total, st>>>(P);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+    return CA_OK;
+}
+
+// The tiled bf16 path serves the heads the fused kernel does not take, for
+// K <= 64 and a window radius floor(W/2) <= 128.
+bool tiled_eligible(int dtype, const Problem &p) {
+    return dtype == 1 && p.K <= 64 && p.W / 2 <= ca::tiled::kMaxR;
+}
+
+ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v, const Problem &p,
+                    __nv_bfloat16 *out, int32_t *assign_out, float *cent_out, int32_t *hist, cudaStream_t st) {
+    using namespace ca;
+    const int64_t NH = p.heads();
+    const int L = p.L, K = p.K, Kp = tiled::kpad(K);
+    const int n_tiles = (L + tiled::kTileQ - 1) / tiled::kTileQ;
+    const int n_chunks = (L + tiled::kChunk - 1) / tiled::kChunk;
+    const float scale = 1.0f / sqrtf((float)p.d);
+    Scratch s(st);
+    float *mu = nullptr, *mm = nullptr, *cpart = nullptr, *vcent = nullptr;
+    __nv_bfloat16 *hi = nullptr, *lo = nullptr;
+    uint32_t *hash = nullptr;
+    double *psum = nullptr;
+    int *pcnt = nullptr;
+    int32_t *assign = assign_out;
+    CA_CUDA(s.get((void **)&mu, sizeof(float) * NH * Kp * kD));
+    CA_CUDA(s.get((void **)&hi, sizeof(__nv_bfloat16) * NH * Kp * kD));
+    CA_CUDA(s.get((void **)&lo, sizeof(__nv_bfloat16) * NH * Kp * kD));
+    CA_CUDA(s.get((void **)&mm, sizeof(float) * NH * Kp));
+    CA_CUDA(s.get((void **)&hash, sizeof(uint32_t) * NH * Kp));
+    CA_CUDA(s.get((void **)&psum, sizeof(double) * NH * n_tiles * Kp * kD));
+    CA_CUDA(s.get((void **)&pcnt, sizeof(int) * NH * n_tiles * Kp));
+    CA_CUDA(s.get((void **)&cpart, sizeof(float) * NH * n_chunks * K * (kD + 2)));
+    CA_CUDA(s.get((void **)&vcent, sizeof(float) * NH * K * kD));
+    if (!assign) CA_CUDA(s.get((void **)&assign, sizeof(int32_t) * NH * L));
+
+    static bool attr_set[64] = {};
+    int dev = 0;
+    CA_CUDA(cudaGetDevice(&dev));
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+        CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+        CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+        attr_set[dev] = true;
+    }
+    const double head_bytes = (double)NH * L * kD * sizeof(__nv_bfloat16);
+
+    tiled::MuParams mp{};
+    mp.q = q;
+    mp.part_sum = psum;
+    mp.part_cnt = pcnt;
+    mp.mu = mu;
+    mp.hi = hi;
+    mp.lo = lo;
+    mp.mm = mm;
+    mp.hash = hash;
+    mp.L = L;
+    mp.K = K;
+    mp.Kp = Kp;
+    mp.n_tiles = n_tiles;
+    mp.init = 1;
+    mp.cent_out = p.iters == 0 ? cent_out : nullptr;
+    {
+        Launch pl("tiled_init", st, 0.0);
+        tiled::tiled_mu_kernel<<<dim3(Kp, (unsigned)NH), 64, 0, st>>>(mp);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+    if (p.iters == 0) CA_CUDA(cudaMemsetAsync(assign, 0, sizeof(int32_t) * NH * L, st));
+
+    const tiled::AssignLayout alay(K);
+    tiled::AssignParams ap{};
+    ap.q = q;
+    ap.mu = mu;
+    ap.hi = hi;
+    ap.lo = lo;
+    ap.mm = mm;
+    ap.hash = hash;
+    ap.assign = assign;
+    ap.hist_stride = (int64_t)p.iters * L;
+    ap.part_sum = psum;
+    ap.part_cnt = pcnt;
+    ap.L = L;
+    ap.K = K;
+    ap.n_tiles = n_tiles;
+    mp.init = 0;
+    for (int t = 0; t < p.iters; ++t) {
+        ap.hist = hist ? hist + (int64_t)t * L : nullptr;
+        {
+            Launch pl("tiled_assign", st, head_bytes);
+            tiled::tiled_assign_kernel<<<dim3(n_tiles, (unsigned)NH), tiled::kThreads, alay.total, st>>>(ap);
+            pl.after();
+        }
+        CA_CUDA(cudaGetLastError());
+        mp.cent_out = t == p.iters - 1 ? cent_out : nullptr;
+        {
+            Launch pl("tiled_update", st, 0.0);
+            tiled::tiled_mu_kernel<<<dim3(Kp, (unsigned)NH), 64, 0, st>>>(mp);
+            pl.after();
+        }
+        CA_CUDA(cudaGetLastError());
+    }
+
+    const tiled::CentroidLayout clay(K);
+    tiled::CentroidParams cp{};
+    cp.k = k;
+    cp.v = v;
+    cp.hi = hi;
+    cp.lo = lo;
+    cp.part = cpart;
+    cp.L = L;
+    cp.K = K;
+    cp.n_chunks = n_chunks;
+    cp.scale = scale;
+    {
+        Launch pl("tiled_centroid", st, 2.0 * head_bytes);
+        tiled::tiled_centroid_kernel<<<dim3(n_chunks, (unsigned)NH), tiled::kThreads, clay.total, st>>>(cp);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+    {
+        Launch pl("tiled_combine", st, 0.0);
+        centroid_attn_combine_kernel<<<(unsigned)NH, 256, 0, st>>>(K, n_chunks, cpart, vcent);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
+
+    const tiled::WindowLayout wlay(K, p.W / 2);
+    tiled::WindowParams wp{};
+    wp.q = q;
+    wp.k = k;
+    wp.v = v;
+    wp.vcent = vcent;
+    wp.assign = assign;
+    wp.out = out;
+    wp.L = L;
+    wp.K = K;
+    wp.r = p.W / 2;
+    wp.alpha = p.alpha;
+    wp.scale = scale;
+    {
+        Launch pl("tiled_window", st, 4.0 * head_bytes);
+        tiled::tiled_window_kernel<<<dim3((L + tiled::kWinQ - 1) / tiled::kWinQ, (unsigned)NH), tiled::kThreads, wlay.total, st>>>(wp);
         pl.after();
     }
     CA_CUDA(cudaGetLastError());
@@ -256,6 +402,9 @@ ca_status dispatch(const void *q, const void *k, const void *v, int dtype, const
     cudaStream_t st = (cudaStream_t)stream;
     if (fused_eligible(dtype, p))
         return run_fused((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, p,
+                         (__nv_bfloat16 *)out, assign_out, cent_out, hist, st);
+    if (tiled_eligible(dtype, p))
+        return run_tiled((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, p,
                          (__nv_bfloat16 *)out, assign_out, cent_out, hist, st);
     if (dtype == 0)
         return run_forward<float>((const float *)q, (const float *)k, (const float *)v, p, (float *)out,

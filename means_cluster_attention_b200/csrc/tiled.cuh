@@ -1,0 +1,959 @@
+// Tiled cluster-attention kernels for long sequences (bf16): the same phase
+// code as the fused one-CTA-per-head kernel, cut into launches that split a
+// head over several CTAs.
+//
+//   tiled_mu_kernel        (K, heads)      mu = strided init, or the update
+//                                          mu_k = fp32(sum_k / max(1, count_k))
+//                                          from per-tile exact partial sums;
+//                                          also the bf16 hi/lo split, |mu|^2
+//                                          and a row hash for each centroid.
+//   tiled_assign_kernel    (tiles, heads)  one Lloyd assignment for a tile of
+//                                          512 queries (tensor-core distances,
+//                                          exact argmin) and the tile's exact
+//                                          fp64 member sums.
+//   tiled_centroid_kernel  (chunks, heads) partial softmax state of every
+//                                          centroid over 512 keys; combined by
+//                                          centroid_attn_combine_kernel.
+//   tiled_window_kernel    (blocks, heads) clipped window attention for 128
+//                                          queries, gather V_cent[c_i], blend.
+//
+// Model card "Hooshaai/distilbert-sst2-cluster-attention", Architecture
+// Overview and Mathematical Formulation section 1; "Hooshaai/svd-sst2-
+// roberta-cluster" sections 2.1 and 3.
+#pragma once
+
+#include "fused.cuh"
+
+namespace ca {
+namespace tiled {
+
+using fused::Best;
+using fused::best_merge;
+using fused::best_push;
+using fused::best_quad;
+using fused::bf16_to_f64;
+using fused::bf16hi;
+using fused::bf16lo;
+using fused::bf16x2_has_zero_exp;
+using fused::bf16x2_to_f64_normal;
+using fused::ex2;
+using fused::kEps;
+using fused::kLog2e;
+using fused::load_rows;
+using fused::up;
+
+constexpr int kThreads = 256;
+constexpr int kWarps = 8;
+constexpr int kTileQ = 512;   // queries per assignment tile
+constexpr int kChunk = 512;   // keys per centroid-attention CTA
+constexpr int kTile = 64;
+constexpr int kSlots = 5;
+constexpr int kWinQ = 128;    // queries per window CTA
+constexpr int kMaxR = 128;    // largest window radius floor(W/2)
+constexpr int kNTChunk = 6;   // key n-tiles per online-softmax step in the window
+
+__host__ __device__ inline int kpad(int K) { return K <= 16 ? 16 : (K <= 32 ? 32 : 64); }
+
+// ---------------------------------------------------------------------------
+// Centroid set: mu^(0) or the update from per-tile partial sums.
+struct MuParams {
+    const __nv_bfloat16 *q;
+    const double *part_sum;  // [NH][n_tiles][Kp][64]
+    const int *part_cnt;     // [NH][n_tiles][Kp]
+    float *mu;               // [NH][Kp][64]
+    __nv_bfloat16 *hi, *lo;  // [NH][Kp][64]
+    float *mm;               // [NH][Kp]
+    uint32_t *hash;          // [NH][Kp]
+    float *cent_out;         // [NH][K][64] or null
+    int L, K, Kp, n_tiles, init;
+};
+
+// grid (Kp, NH), 64 threads: thread j owns coordinate j of centroid k.
+__global__ void __launch_bounds__(64) tiled_mu_kernel(MuParams P) {
+    __shared__ float red_sq[2];
+    __shared__ uint32_t red_h[2];
+    const int k = blockIdx.x, j = threadIdx.x, lane = j & 31, wid = j >> 5;
+    const int64_t head = blockIdx.y;
+    float x = 0.f;
+    if (k < P.K) {
+        if (P.init) {
+            const int64_t row = ((int64_t)k * P.L) / P.K;
+            x = __bfloat162float(P.q[(head * P.L + row) * kD + j]);
+        } else {
+            double s = 0.0;
+            int cnt = 0;
+            for (int t = 0; t < P.n_tiles; ++t) {
+                const int64_t base = (head * P.n_tiles + t) * P.Kp + k;
+                s += P.part_sum[base * kD + j];
+                cnt += P.part_cnt[base];
+            }
+            x = __double2float_rn(s / (double)(cnt > 1 ? cnt : 1));
+        }
+    }
+    const int64_t o = (head * P.Kp + k) * kD + j;
+    P.mu[o] = x;
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    P.hi[o] = h;
+    P.lo[o] = __float2bfloat16_rn(x - __bfloat162float(h));
+    if (P.cent_out && k < P.K) P.cent_out[(head * P.K + k) * kD + j] = x;
+    float sq = x * x;
+    uint32_t hv = __float_as_uint(x) * (0x9E3779B1u + 2u * (uint32_t)j) + (uint32_t)j * 0xC2B2AE3Du;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        hv += __shfl_xor_sync(0xffffffffu, hv, off);
+    }
+    if (lane == 0) {
+        red_sq[wid] = sq;
+        red_h[wid] = hv;
+    }
+    __syncthreads();
+    if (j == 0) {
+        P.mm[head * P.Kp + k] = red_sq[0] + red_sq[1];
+        P.hash[head * P.Kp + k] = red_h[0] + red_h[1];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// One Lloyd assignment for a tile of up to 512 queries.
+struct AssignLayout {
+    int Kp, Tp;
+    uint32_t q_off, sums_off, mu_off, hi_off, lo_off, mm_off, hash_off, cnt_off, base_off, dead_off,
+        c_off, sc_off, list_off, perm_off, table_off, misc_off, total;
+    __host__ __device__ AssignLayout(int K) {
+        Kp = kpad(K);
+        Tp = kTileQ;
+        uint32_t o = 0;
+        q_off = o;
+        o += (uint32_t)Tp * 128u;
+        sums_off = o;
+        o += (uint32_t)Kp * 64u * 8u;
+        mu_off = o;
+        o += up((uint32_t)Kp * 65u * 4u, 128);
+        hi_off = o;
+        o += (uint32_t)Kp * 128u;
+        lo_off = o;
+        o += (uint32_t)Kp * 128u;
+        mm_off = o;
+        o += (uint32_t)Kp * 4u;
+        hash_off = o;
+        o += (uint32_t)Kp * 4u;
+        cnt_off = o;
+        o += (uint32_t)Kp * 4u;
+        base_off = o;
+        o += (uint32_t)Kp * 4u;
+        dead_off = o;
+        o += up((uint32_t)Kp, 16);
+        c_off = o;
+        o += (uint32_t)Tp;
+        sc_off = o;
+        o += (uint32_t)Tp;
+        list_off = o;
+        o += (uint32_t)Tp * 2u;
+        perm_off = o;
+        o += (uint32_t)Tp * 2u;
+        table_off = o;
+        o += up((uint32_t)(Tp / 32) * (uint32_t)Kp * 2u, 16);
+        misc_off = o;
+        o += 64;
+        total = up(o, 128);
+    }
+};
+
+struct AssignParams {
+    const __nv_bfloat16 *q;
+    const float *mu;
+    const __nv_bfloat16 *hi, *lo;
+    const float *mm;
+    const uint32_t *hash;
+    int32_t *assign;     // [NH][L]
+    int32_t *hist;       // [NH][iters][L] or null (already offset by the iteration)
+    int64_t hist_stride; // iters * L
+    double *part_sum;    // [NH][n_tiles][Kp][64]
+    int *part_cnt;       // [NH][n_tiles][Kp]
+    int L, K, n_tiles;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) tiled_assign_kernel(AssignParams P) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const AssignLayout lay(P.K);
+    const int K = P.K, Kp = lay.Kp;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int tile = blockIdx.x;
+    const int64_t head = blockIdx.y;
+    const int t0 = tile * kTileQ;
+    const int Lt = min(kTileQ, P.L - t0);  // tokens in this tile
+    const __nv_bfloat16 *qh = P.q + (head * P.L + t0) * kD;
+
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t q_s = sbase + lay.q_off, hi_s = sbase + lay.hi_off, lo_s = sbase + lay.lo_off;
+    unsigned char *qbytes = smem + lay.q_off;
+    double *sums = reinterpret_cast<double *>(smem + lay.sums_off);
+    float *mu = reinterpret_cast<float *>(smem + lay.mu_off);
+    float *mm = reinterpret_cast<float *>(smem + lay.mm_off);
+    uint32_t *hsh = reinterpret_cast<uint32_t *>(smem + lay.hash_off);
+    int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
+    int *base_s = reinterpret_cast<int *>(smem + lay.base_off);
+    uint8_t *dead = smem + lay.dead_off;
+    uint8_t *cs = smem + lay.c_off;
+    uint8_t *sc = smem + lay.sc_off;
+    uint16_t *list = reinterpret_cast<uint16_t *>(smem + lay.list_off);
+    uint16_t *perm = reinterpret_cast<uint16_t *>(smem + lay.perm_off);
+    int16_t *table = reinterpret_cast<int16_t *>(smem + lay.table_off);
+    int *misc = reinterpret_cast<int *>(smem + lay.misc_off);
+
+    load_rows(q_s, qh, 0, kTileQ, Lt);
+    cp_async_commit();
+    const int64_t cb = head * Kp;
+    for (int e = threadIdx.x; e < Kp * kD; e += kThreads) {
+        const int kk = e / kD, j = e % kD;
+        mu[kk * 65 + j] = P.mu[(cb + kk) * kD + j];
+    }
+    for (int e = threadIdx.x; e < Kp * 8; e += kThreads) {
+        const int kk = e >> 3, ch = e & 7;
+        const uint4 vh = *reinterpret_cast<const uint4 *>(P.hi + (cb + kk) * kD + ch * 8);
+        const uint4 vl = *reinterpret_cast<const uint4 *>(P.lo + (cb + kk) * kD + ch * 8);
+        *reinterpret_cast<uint4 *>(smem + lay.hi_off + swz(kk, ch)) = vh;
+        *reinterpret_cast<uint4 *>(smem + lay.lo_off + swz(kk, ch)) = vl;
+    }
+    for (int kk = threadIdx.x; kk < Kp; kk += kThreads) {
+        mm[kk] = P.mm[cb + kk];
+        hsh[kk] = P.hash[cb + kk];
+    }
+    for (int i = threadIdx.x; i < kTileQ; i += kThreads) cs[i] = i < Lt ? 0 : 0xFF;
+    if (threadIdx.x == 0) misc[0] = 0;
+    __syncthreads();
+    // dead centroids: padding and bitwise copies of a lower-index centroid
+    {
+        const int kk = threadIdx.x;
+        bool dd = true;
+        if (kk < Kp) {
+            dd = kk >= K;
+            for (int a = 0; a < kk && !dd; ++a) {
+                if (hsh[a] != hsh[kk]) continue;
+                bool same = true;
+                for (int j = 0; j < kD && same; ++j)
+                    same = __float_as_uint(mu[a * 65 + j]) == __float_as_uint(mu[kk * 65 + j]);
+                dd = same;
+            }
+            dead[kk] = dd ? 1 : 0;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            float mx = 0.f;
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                const int k2 = lane + 32 * s;
+                if (k2 < Kp) {
+                    if (dead[k2]) mm[k2] = INFINITY;
+                    else mx = fmaxf(mx, mm[k2]);
+                }
+            }
+            mx = warp_max(mx);
+            if (lane == 0) {
+                misc[1] = __float_as_int(mx);
+                misc[2] = __float_as_int(sqrtf(mx));
+            }
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    const float mm_max = __int_as_float(misc[1]), mun_max = __int_as_float(misc[2]);
+    constexpr int kMtPerWarp = kTileQ / 16 / kWarps;  // 4
+    const int n_mt = (Lt + 15) / 16;
+
+    // assignment: tensor-core distances + certified argmin
+#pragma unroll
+    for (int jp = 0; jp < kMtPerWarp; jp += 2) {
+        const int mt0 = warp + jp * kWarps, mt1 = mt0 + kWarps;
+        if (mt0 >= n_mt) break;
+        const bool two = mt1 < n_mt;
+        uint32_t a0[4][4], a1[4][4];
+        float qn[2][2];
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const int m = lane >> 3;
+            const int rr = (lane & 7) + ((m & 1) ? 8 : 0);
+            ldmatrix_x4(a0[ks], q_s + swz(mt0 * 16 + rr, 2 * ks + (m >> 1)));
+            if (two) ldmatrix_x4(a1[ks], q_s + swz(mt1 * 16 + rr, 2 * ks + (m >> 1)));
+            else a1[ks][0] = a1[ks][1] = a1[ks][2] = a1[ks][3] = 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int mt = u ? mt1 : mt0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float a = 0.f;
+                const int row = mt * 16 + g + 8 * h;
+                if (u == 0 || two) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(qbytes + swz(row, 2 * t + c));
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float x0 = bf16lo(ws[e]), x1 = bf16hi(ws[e]);
+                            a = fmaf(x0, x0, fmaf(x1, x1, a));
+                        }
+                    }
+                }
+                a += __shfl_xor_sync(0xffffffffu, a, 1);
+                a += __shfl_xor_sync(0xffffffffu, a, 2);
+                qn[u][h] = sqrtf(a);
+            }
+        }
+        Best b[2][2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) b[u][h] = Best{INFINITY, INFINITY, 0};
+        for (int nt = 0; nt < Kp / 8; ++nt) {
+            uint32_t bh[2][4], bl[2][4];
+#pragma unroll
+            for (int kp = 0; kp < 2; ++kp) {
+                const int row = nt * 8 + (lane & 7);
+                const int chunk = 4 * kp + (lane >> 3);
+                ldmatrix_x4(bh[kp], hi_s + swz(row, chunk));
+                ldmatrix_x4(bl[kp], lo_s + swz(row, chunk));
+            }
+            float acc[2][2][4];
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int s = 0; s < 2; ++s)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[u][s][e] = 0.f;
+#pragma unroll
+            for (int kp = 0; kp < 2; ++kp) {
+                mma_16816(acc[0][0], a0[2 * kp], bh[kp][0], bh[kp][1]);
+                mma_16816(acc[0][1], a0[2 * kp], bl[kp][0], bl[kp][1]);
+                mma_16816(acc[1][0], a1[2 * kp], bh[kp][0], bh[kp][1]);
+                mma_16816(acc[1][1], a1[2 * kp], bl[kp][0], bl[kp][1]);
+                mma_16816(acc[0][0], a0[2 * kp + 1], bh[kp][2], bh[kp][3]);
+                mma_16816(acc[0][1], a0[2 * kp + 1], bl[kp][2], bl[kp][3]);
+                mma_16816(acc[1][0], a1[2 * kp + 1], bh[kp][2], bh[kp][3]);
+                mma_16816(acc[1][1], a1[2 * kp + 1], bl[kp][2], bl[kp][3]);
+            }
+            const int c0 = nt * 8 + 2 * t;
+            const float m0 = mm[c0], m1 = mm[c0 + 1];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                best_push(b[u][0], fmaf(-2.f, acc[u][0][0] + acc[u][1][0], m0), c0);
+                best_push(b[u][0], fmaf(-2.f, acc[u][0][1] + acc[u][1][1], m1), c0 + 1);
+                best_push(b[u][1], fmaf(-2.f, acc[u][0][2] + acc[u][1][2], m0), c0);
+                best_push(b[u][1], fmaf(-2.f, acc[u][0][3] + acc[u][1][3], m1), c0 + 1);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int mt = u ? mt1 : mt0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const Best bb = best_quad(b[u][h]);
+                const int row = mt * 16 + g + 8 * h;
+                if (t == 0 && (u == 0 || two) && row < Lt) {
+                    const float E = kEps * fmaf(qn[u][h], mun_max, mm_max);
+                    cs[row] = (uint8_t)bb.k1;
+                    if (bb.m2 <= bb.m1 + 2.f * E) list[atomicAdd(&misc[0], 1)] = (uint16_t)row;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    // exact re-measure of ambiguous tokens, one warp per token
+    const int n_ref = misc[0];
+    for (int e = warp; e < n_ref; e += kWarps) {
+        const int row = list[e];
+        double qq = 0.0, qm0 = 0.0, qm1 = 0.0, m20 = 0.0, m21 = 0.0;
+        const int k0 = lane, k1 = lane + 32;
+        const bool v0 = k0 < Kp, v1 = k1 < Kp;
+#pragma unroll 2
+        for (int jb = 0; jb < kD; jb += 8) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(qbytes + swz(row, jb >> 3));
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+            double qj[8], mj0[8], mj1[8];
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+                qj[2 * e2] = bf16_to_f64(ws[e2] & 0xffffu);
+                qj[2 * e2 + 1] = bf16_to_f64(ws[e2] >> 16);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                mj0[u] = v0 ? (double)mu[k0 * 65 + jb + u] : 0.0;
+                mj1[u] = v1 ? (double)mu[k1 * 65 + jb + u] : 0.0;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                qq = __dadd_rn(qq, __dmul_rn(qj[u], qj[u]));
+                qm0 = __dadd_rn(qm0, __dmul_rn(qj[u], mj0[u]));
+                m20 = __dadd_rn(m20, __dmul_rn(mj0[u], mj0[u]));
+                qm1 = __dadd_rn(qm1, __dmul_rn(qj[u], mj1[u]));
+                m21 = __dadd_rn(m21, __dmul_rn(mj1[u], mj1[u]));
+            }
+        }
+        double bd = INFINITY;
+        int bk = 0x7fffffff;
+        if (v0 && !dead[k0]) {
+            bd = __dsub_rn(__dadd_rn(qq, m20), __dmul_rn(2.0, qm0));
+            bk = k0;
+        }
+        if (v1 && !dead[k1]) {
+            const double D = __dsub_rn(__dadd_rn(qq, m21), __dmul_rn(2.0, qm1));
+            if (D < bd) {
+                bd = D;
+                bk = k1;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const double od = __shfl_xor_sync(0xffffffffu, bd, o);
+            const int ok = __shfl_xor_sync(0xffffffffu, bk, o);
+            if (od < bd || (od == bd && ok < bk)) {
+                bd = od;
+                bk = ok;
+            }
+        }
+        if (lane == 0) {
+            if (bk >= K) {
+                record_error(5, 3);
+                bk = 0;
+            }
+            cs[row] = (uint8_t)bk;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < Lt; i += kThreads) {
+        P.assign[head * P.L + t0 + i] = cs[i];
+        if (P.hist) P.hist[head * P.hist_stride + t0 + i] = cs[i];
+    }
+    // stable counting sort of the tile's tokens by cluster
+    const int nch = kTileQ / 32;
+    for (int i = threadIdx.x; i < nch * Kp; i += kThreads) table[i] = 0;
+    for (int i = threadIdx.x; i < Kp * kD; i += kThreads) sums[i] = 0.0;
+    __syncthreads();
+    int my_c[2], my_rank[2];
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        const int ch = warp + s * kWarps;
+        const int c = cs[ch * 32 + lane];
+        const unsigned peers = __match_any_sync(0xffffffffu, c);
+        my_c[s] = c;
+        my_rank[s] = __popc(peers & ((1u << lane) - 1u));
+        if (c != 0xFF && lane == __ffs(peers) - 1) table[ch * Kp + c] = (int16_t)__popc(peers);
+    }
+    __syncthreads();
+    if (threadIdx.x < Kp) {
+        int run = 0;
+        for (int ch = 0; ch < nch; ++ch) {
+            const int v = table[ch * Kp + threadIdx.x];
+            table[ch * Kp + threadIdx.x] = (int16_t)run;
+            run += v;
+        }
+        cnt_s[threadIdx.x] = run;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int c0 = lane < Kp ? cnt_s[lane] : 0, c1 = lane + 32 < Kp ? cnt_s[lane + 32] : 0;
+        int s0 = c0, s1 = c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x0 = __shfl_up_sync(0xffffffffu, s0, o), x1 = __shfl_up_sync(0xffffffffu, s1, o);
+            if (lane >= o) {
+                s0 += x0;
+                s1 += x1;
+            }
+        }
+        const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
+        if (lane < Kp) base_s[lane] = s0 - c0;
+        if (lane + 32 < Kp) base_s[lane + 32] = tot0 + s1 - c1;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        const int ch = warp + s * kWarps;
+        if (my_c[s] != 0xFF) {
+            const int pos = base_s[my_c[s]] + table[ch * Kp + my_c[s]] + my_rank[s];
+            perm[pos] = (uint16_t)(ch * 32 + lane);
+            sc[pos] = (uint8_t)my_c[s];
+        }
+    }
+    __syncthreads();
+    // exact member sums, run by run over the sorted tokens
+    {
+        const int seg = (Lt + kWarps - 1) / kWarps;
+        const int p1 = min(Lt, (warp + 1) * seg);
+        int p = warp * seg;
+        while (p < p1) {
+            const int c = sc[p];
+            double s0[4] = {0.0, 0.0, 0.0, 0.0}, s1[4] = {0.0, 0.0, 0.0, 0.0};
+            for (;;) {
+                const int qq = p + lane;
+                const unsigned same = __ballot_sync(0xffffffffu, qq < p1 && sc[qq] == c);
+                const int n = __ffs(~same) ? __ffs(~same) - 1 : 32;
+                const int rowl = (lane < n) ? perm[p + lane] : 0;
+                for (int j = 0; j < n; j += 4) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int rr = __shfl_sync(0xffffffffu, rowl, (j + u) & 31);
+                        w[u] = (j + u < n) ? *reinterpret_cast<const uint32_t *>(qbytes + swz(rr, lane >> 2) + (lane & 3) * 4) : 0u;
+                    }
+                    bool slow = false;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) slow |= (j + u < n) && bf16x2_has_zero_exp(w[u]);
+                    if (__any_sync(0xffffffffu, slow)) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            if (j + u < n) {
+                                s0[u] += bf16_to_f64(w[u] & 0xffffu);
+                                s1[u] += bf16_to_f64(w[u] >> 16);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            if (j + u < n) {
+                                double d0, d1;
+                                bf16x2_to_f64_normal(w[u], d0, d1);
+                                s0[u] += d0;
+                                s1[u] += d1;
+                            }
+                        }
+                    }
+                }
+                p += n;
+                if (n < 32) break;
+            }
+            atomicAdd(&sums[c * kD + 2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
+            atomicAdd(&sums[c * kD + 2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
+        }
+    }
+    __syncthreads();
+    const int64_t pb = (head * P.n_tiles + tile) * Kp;
+    for (int e = threadIdx.x; e < Kp * kD; e += kThreads) P.part_sum[pb * kD + e] = sums[e];
+    for (int kk = threadIdx.x; kk < Kp; kk += kThreads) P.part_cnt[pb + kk] = cnt_s[kk];
+}
+
+// ---------------------------------------------------------------------------
+// Centroid attention over a chunk of up to 512 keys: the chunk's softmax
+// state (sum of exp-weighted V rows, running max in natural-log units, and
+// running denominator) for every centroid, in the layout of
+// centroid_attn_combine_kernel: part[head][chunk][K][64 + 2].
+struct CentroidLayout {
+    int Kp;
+    uint32_t slots_off, hi_off, lo_off, ml_off, total;
+    __host__ __device__ CentroidLayout(int K) {
+        Kp = kpad(K);
+        uint32_t o = 0;
+        slots_off = o;
+        const uint32_t slots = (uint32_t)kSlots * 2u * kTile * 128u;
+        const uint32_t comb = (uint32_t)kWarps * 16u * 64u * 4u;
+        o += up(slots > comb ? slots : comb, 1024);
+        hi_off = o;
+        o += (uint32_t)Kp * 128u;
+        lo_off = o;
+        o += (uint32_t)Kp * 128u;
+        ml_off = o;
+        o += (uint32_t)kWarps * 16u * 2u * 4u;
+        total = up(o, 128);
+    }
+};
+
+struct CentroidParams {
+    const __nv_bfloat16 *k, *v;
+    const __nv_bfloat16 *hi, *lo;  // [NH][Kp][64]
+    float *part;                   // [NH][n_chunks][K][66]
+    int L, K, n_chunks;
+    float scale;
+};
+
+__global__ void __launch_bounds__(kThreads, 2) tiled_centroid_kernel(CentroidParams P) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const CentroidLayout lay(P.K);
+    const int K = P.K, Kp = lay.Kp;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int chunk = blockIdx.x;
+    const int64_t head = blockIdx.y;
+    const int k0 = chunk * kChunk;
+    const int Lc = min(kChunk, P.L - k0);
+    const int nT = (Lc + kTile - 1) / kTile;
+    const __nv_bfloat16 *kh = P.k + (head * P.L + k0) * kD;
+    const __nv_bfloat16 *vh = P.v + (head * P.L + k0) * kD;
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t slot_s = sbase + lay.slots_off, hi_s = sbase + lay.hi_off, lo_s = sbase + lay.lo_off;
+    float *ml = reinterpret_cast<float *>(smem + lay.ml_off);
+
+    for (int s = 0; s < kSlots; ++s) {
+        if (s < nT) {
+            const uint32_t slot = slot_s + s * 2 * kTile * 128;
+            load_rows(slot, kh, s * kTile, kTile, Lc);
+            load_rows(slot + kTile * 128, vh, s * kTile, kTile, Lc);
+        }
+        cp_async_commit();
+    }
+    const int64_t cb = head * Kp;
+    for (int e = threadIdx.x; e < Kp * 8; e += kThreads) {
+        const int kk = e >> 3, ch = e & 7;
+        *reinterpret_cast<uint4 *>(smem + lay.hi_off + swz(kk, ch)) = *reinterpret_cast<const uint4 *>(P.hi + (cb + kk) * kD + ch * 8);
+        *reinterpret_cast<uint4 *>(smem + lay.lo_off + swz(kk, ch)) = *reinterpret_cast<const uint4 *>(P.lo + (cb + kk) * kD + ch * 8);
+    }
+    __syncthreads();
+    const int n_cm = Kp / 16, G = kWarps / n_cm, cm = warp / G, kb = warp % G, keys_w = kTile / G;
+    const float csc = P.scale * kLog2e;
+    uint32_t ahi[4][4], alo[4][4];
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+        const int m = lane >> 3;
+        const int row = cm * 16 + (lane & 7) + ((m & 1) ? 8 : 0);
+        ldmatrix_x4(ahi[ks], hi_s + swz(row, 2 * ks + (m >> 1)));
+        ldmatrix_x4(alo[ks], lo_s + swz(row, 2 * ks + (m >> 1)));
+    }
+    float o_acc[8][4];
+#pragma unroll
+    for (int d = 0; d < 8; ++d)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o_acc[d][e] = 0.f;
+    float rm[2] = {-INFINITY, -INFINITY}, rl[2] = {0.f, 0.f};
+    for (int tt = 0; tt < nT; ++tt) {
+        cp_async_wait<kSlots - 1>();
+        __syncthreads();
+        const uint32_t kt = slot_s + (tt % kSlots) * 2 * kTile * 128;
+        const uint32_t vt = kt + kTile * 128;
+        float sacc[4][4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[n][e] = 0.f;
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            if (n * 8 >= keys_w) break;
+            const int key0 = kb * keys_w + n * 8;
+#pragma unroll
+            for (int kp = 0; kp < 2; ++kp) {
+                uint32_t bk[4];
+                ldmatrix_x4(bk, kt + swz(key0 + (lane & 7), 4 * kp + (lane >> 3)));
+                mma_16816(sacc[n], ahi[2 * kp], bk[0], bk[1]);
+                mma_16816(sacc[n], ahi[2 * kp + 1], bk[2], bk[3]);
+                mma_16816(sacc[n], alo[2 * kp], bk[0], bk[1]);
+                mma_16816(sacc[n], alo[2 * kp + 1], bk[2], bk[3]);
+            }
+        }
+        float tmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            if (n * 8 >= keys_w) break;
+            const int key = tt * kTile + kb * keys_w + n * 8 + 2 * t;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (key + (e & 1) >= Lc) sacc[n][e] = -INFINITY;
+            tmax[0] = fmaxf(tmax[0], fmaxf(sacc[n][0], sacc[n][1]));
+            tmax[1] = fmaxf(tmax[1], fmaxf(sacc[n][2], sacc[n][3]));
+        }
+        float corr[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 1));
+            tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 2));
+            const float mn = fmaxf(rm[h], tmax[h]);
+            corr[h] = (mn == -INFINITY) ? 1.f : ex2((rm[h] - mn) * csc);
+            rm[h] = mn;
+            rl[h] *= corr[h];
+        }
+#pragma unroll
+        for (int d = 0; d < 8; ++d) {
+            o_acc[d][0] *= corr[0];
+            o_acc[d][1] *= corr[0];
+            o_acc[d][2] *= corr[1];
+            o_acc[d][3] *= corr[1];
+        }
+        uint32_t pa[4][2];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            pa[n][0] = pa[n][1] = 0u;
+            if (n * 8 >= keys_w) break;
+            float p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float mh = rm[e >> 1];
+                p[e] = (mh == -INFINITY) ? 0.f : ex2((sacc[n][e] - mh) * csc);
+            }
+            rl[0] += p[0] + p[1];
+            rl[1] += p[2] + p[3];
+            pa[n][0] = pack_bf16(p[0], p[1]);
+            pa[n][1] = pack_bf16(p[2], p[3]);
+        }
+        if (keys_w == 8) {
+            const int key0 = kb * keys_w;
+#pragma unroll
+            for (int dq = 0; dq < 2; ++dq) {
+                uint32_t bv[4];
+                ldmatrix_x4_trans(bv, vt + swz(key0 + (lane & 7), 4 * dq + (lane >> 3)));
+#pragma unroll
+                for (int u = 0; u < 4; ++u) mma_1688(o_acc[4 * dq + u], pa[0][0], pa[0][1], bv[u]);
+            }
+        } else {
+#pragma unroll
+            for (int n2 = 0; n2 < 2; ++n2) {
+                if (n2 * 16 >= keys_w) break;
+                const uint32_t a4[4] = {pa[2 * n2][0], pa[2 * n2][1], pa[2 * n2 + 1][0], pa[2 * n2 + 1][1]};
+                const int key0 = kb * keys_w + n2 * 16;
+#pragma unroll
+                for (int dq = 0; dq < 4; ++dq) {
+                    uint32_t bv[4];
+                    const int m = lane >> 3;
+                    ldmatrix_x4_trans(bv, vt + swz(key0 + (lane & 7) + ((m & 1) ? 8 : 0), 2 * dq + (m >> 1)));
+                    mma_16816(o_acc[2 * dq], a4, bv[0], bv[1]);
+                    mma_16816(o_acc[2 * dq + 1], a4, bv[2], bv[3]);
+                }
+            }
+        }
+        __syncthreads();
+        if (tt + kSlots < nT) {
+            load_rows(kt, kh, (tt + kSlots) * kTile, kTile, Lc);
+            load_rows(vt, vh, (tt + kSlots) * kTile, kTile, Lc);
+        }
+        cp_async_commit();
+    }
+    cp_async_wait<0>();
+    float *part = reinterpret_cast<float *>(smem + lay.slots_off);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        rl[h] += __shfl_xor_sync(0xffffffffu, rl[h], 1);
+        rl[h] += __shfl_xor_sync(0xffffffffu, rl[h], 2);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int d = 0; d < 8; ++d) {
+        float *p0 = part + (warp * 16 + g) * 64 + 8 * d + 2 * t;
+        float *p1 = part + (warp * 16 + g + 8) * 64 + 8 * d + 2 * t;
+        p0[0] = o_acc[d][0];
+        p0[1] = o_acc[d][1];
+        p1[0] = o_acc[d][2];
+        p1[1] = o_acc[d][3];
+    }
+    if (t == 0) {
+        ml[(warp * 16 + g) * 2 + 0] = rm[0];
+        ml[(warp * 16 + g) * 2 + 1] = rl[0];
+        ml[(warp * 16 + g + 8) * 2 + 0] = rm[1];
+        ml[(warp * 16 + g + 8) * 2 + 1] = rl[1];
+    }
+    __syncthreads();
+    float *outp = P.part + ((head * P.n_chunks + chunk) * (int64_t)K) * (kD + 2);
+    for (int e = threadIdx.x; e < K * (kD + 2); e += kThreads) {
+        const int row = e / (kD + 2), col = e % (kD + 2);
+        const int mt = row / 16, rr = row % 16;
+        float M = -INFINITY;
+        for (int w = mt * G; w < mt * G + G; ++w) M = fmaxf(M, ml[(w * 16 + rr) * 2]);
+        float val;
+        if (col == kD) {
+            val = M * P.scale;  // running max in natural-log units
+        } else {
+            float acc = 0.f;
+            for (int w = mt * G; w < mt * G + G; ++w) {
+                const float mw = ml[(w * 16 + rr) * 2];
+                const float f = (mw == -INFINITY) ? 0.f : ex2((mw - M) * csc);
+                acc = fmaf(col == kD + 1 ? ml[(w * 16 + rr) * 2 + 1] : part[(w * 16 + rr) * 64 + col], f, acc);
+            }
+            val = acc;
+        }
+        outp[e] = val;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Window attention + gather + blend for 128 queries; any radius <= kMaxR.
+struct WindowLayout {
+    int rows, Kp;
+    uint32_t k_off, v_off, vc_off, c_off, total;
+    __host__ __device__ WindowLayout(int K, int r) {
+        Kp = kpad(K);
+        rows = (int)up((uint32_t)(kWinQ + 2 * r + 8), 8);
+        uint32_t o = 0;
+        k_off = o;
+        o += (uint32_t)rows * 128u;
+        v_off = o;
+        o += (uint32_t)rows * 128u;
+        vc_off = o;
+        o += (uint32_t)K * 64u * 4u;
+        c_off = o;
+        o += (uint32_t)kWinQ * 4u;
+        total = up(o, 128);
+    }
+};
+
+struct WindowParams {
+    const __nv_bfloat16 *q, *k, *v;
+    const float *vcent;     // [NH][K][64]
+    const int32_t *assign;  // [NH][L]
+    __nv_bfloat16 *out;
+    int L, K, r;
+    float alpha, scale;
+};
+
+__global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams P) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const WindowLayout lay(P.K, P.r);
+    const int L = P.L, K = P.K, r = P.r;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int64_t head = blockIdx.y;
+    const int qb = blockIdx.x * kWinQ;
+    const __nv_bfloat16 *qh = P.q + head * (int64_t)L * kD;
+    const __nv_bfloat16 *kh = P.k + head * (int64_t)L * kD;
+    const __nv_bfloat16 *vh = P.v + head * (int64_t)L * kD;
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t kw_s = sbase + lay.k_off, vw_s = sbase + lay.v_off;
+    float *vc = reinterpret_cast<float *>(smem + lay.vc_off);
+    int *cblk = reinterpret_cast<int *>(smem + lay.c_off);
+
+    const int ks0 = max(0, qb - r) & ~7;
+    const int ke = min(L - 1, qb + kWinQ - 1 + r);
+    const int nrows = (ke - ks0 + 1 + 7) & ~7;
+    load_rows(kw_s, kh, ks0, nrows, ke + 1);
+    load_rows(vw_s, vh, ks0, nrows, ke + 1);
+    cp_async_commit();
+    const float *vch = P.vcent + head * (int64_t)K * kD;
+    for (int e = threadIdx.x; e < K * kD / 4; e += kThreads)
+        reinterpret_cast<float4 *>(vc)[e] = reinterpret_cast<const float4 *>(vch)[e];
+    for (int i = threadIdx.x; i < kWinQ; i += kThreads) cblk[i] = (qb + i < L) ? P.assign[head * L + qb + i] : 0;
+    const int i0 = qb + warp * 16;
+    uint32_t a[4][4];
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int row = i0 + g + ((e & 1) ? 8 : 0);
+            const int col = 16 * ks + 2 * t + ((e & 2) ? 8 : 0);
+            a[ks][e] = row < L ? __ldg(reinterpret_cast<const unsigned int *>(qh + (int64_t)row * kD + col)) : 0u;
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    if (i0 >= L) return;
+    const float csc = P.scale * kLog2e;
+    const int kst = max(0, i0 - r) & ~7;
+    const int kend = min(L - 1, i0 + 15 + r);
+    const int nt = (kend - kst) / 8 + 1;
+    const int lr0 = kst - ks0;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    float oacc[8][4];
+#pragma unroll
+    for (int d = 0; d < 8; ++d)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oacc[d][e] = 0.f;
+    for (int c0 = 0; c0 < nt; c0 += kNTChunk) {
+        const int cn = min(kNTChunk, nt - c0);
+        float sacc[kNTChunk][4];
+#pragma unroll
+        for (int n = 0; n < kNTChunk; ++n) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[n][e] = 0.f;
+            if (n < cn) {
+#pragma unroll
+                for (int kp = 0; kp < 2; ++kp) {
+                    uint32_t bk[4];
+                    ldmatrix_x4(bk, kw_s + swz(lr0 + (c0 + n) * 8 + (lane & 7), 4 * kp + (lane >> 3)));
+                    mma_16816(sacc[n], a[2 * kp], bk[0], bk[1]);
+                    mma_16816(sacc[n], a[2 * kp + 1], bk[2], bk[3]);
+                }
+            }
+        }
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int n = 0; n < kNTChunk; ++n) {
+            if (n < cn) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = i0 + g + 8 * (e >> 1);
+                    const int jk = kst + (c0 + n) * 8 + 2 * t + (e & 1);
+                    const bool ok = jk >= i - r && jk <= i + r && jk < L;
+                    if (!ok) sacc[n][e] = -INFINITY;
+                }
+                mx[0] = fmaxf(mx[0], fmaxf(sacc[n][0], sacc[n][1]));
+                mx[1] = fmaxf(mx[1], fmaxf(sacc[n][2], sacc[n][3]));
+            }
+        }
+        float corr[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+            mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+            const float mn = fmaxf(m_run[h], mx[h]);
+            corr[h] = (mn == -INFINITY) ? 1.f : ex2((m_run[h] - mn) * csc);
+            m_run[h] = mn;
+            l_run[h] *= corr[h];
+        }
+#pragma unroll
+        for (int d = 0; d < 8; ++d) {
+            oacc[d][0] *= corr[0];
+            oacc[d][1] *= corr[0];
+            oacc[d][2] *= corr[1];
+            oacc[d][3] *= corr[1];
+        }
+        uint32_t pa[kNTChunk][2];
+#pragma unroll
+        for (int n = 0; n < kNTChunk; ++n) {
+            pa[n][0] = pa[n][1] = 0u;
+            if (n < cn) {
+                float p[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float mh = m_run[e >> 1];
+                    p[e] = (mh == -INFINITY) ? 0.f : ex2((sacc[n][e] - mh) * csc);
+                }
+                l_run[0] += p[0] + p[1];
+                l_run[1] += p[2] + p[3];
+                pa[n][0] = pack_bf16(p[0], p[1]);
+                pa[n][1] = pack_bf16(p[2], p[3]);
+            }
+        }
+#pragma unroll
+        for (int n2 = 0; n2 < kNTChunk / 2; ++n2) {
+            if (2 * n2 + 1 < cn) {
+                const uint32_t a4[4] = {pa[2 * n2][0], pa[2 * n2][1], pa[2 * n2 + 1][0], pa[2 * n2 + 1][1]};
+#pragma unroll
+                for (int dq = 0; dq < 4; ++dq) {
+                    uint32_t bv[4];
+                    const int m = lane >> 3;
+                    ldmatrix_x4_trans(bv, vw_s + swz(lr0 + (c0 + 2 * n2) * 8 + (lane & 7) + ((m & 1) ? 8 : 0), 2 * dq + (m >> 1)));
+                    mma_16816(oacc[2 * dq], a4, bv[0], bv[1]);
+                    mma_16816(oacc[2 * dq + 1], a4, bv[2], bv[3]);
+                }
+            } else if (2 * n2 < cn) {
+#pragma unroll
+                for (int dq = 0; dq < 2; ++dq) {
+                    uint32_t bv[4];
+                    ldmatrix_x4_trans(bv, vw_s + swz(lr0 + (c0 + 2 * n2) * 8 + (lane & 7), 4 * dq + (lane >> 3)));
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) mma_1688(oacc[4 * dq + u], pa[2 * n2][0], pa[2 * n2][1], bv[u]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
+        l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
+    }
+    const float inv0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f, inv1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
+    const int ia = i0 + g, ib = i0 + g + 8;
+    const int ca = ia < L ? cblk[ia - qb] : 0, cb2 = ib < L ? cblk[ib - qb] : 0;
+    const float al = P.alpha, be = 1.f - P.alpha;
+    __nv_bfloat16 *oh = P.out + head * (int64_t)L * kD;
+#pragma unroll
+    for (int d = 0; d < 8; ++d) {
+        const int col = 8 * d + 2 * t;
+        if (ia < L) {
+            const float y0 = be * vc[ca * kD + col] + al * (oacc[d][0] * inv0);
+            const float y1 = be * vc[ca * kD + col + 1] + al * (oacc[d][1] * inv0);
+            *reinterpret_cast<uint32_t *>(oh + (int64_t)ia * kD + col) = pack_bf16(y0, y1);
+        }
+        if (ib < L) {
+            const float y2 = be * vc[cb2 * kD + col] + al * (oacc[d][2] * inv1);
+            const float y3 = be * vc[cb2 * kD + col + 1] + al * (oacc[d][3] * inv1);
+            *reinterpret_cast<uint32_t *>(oh + (int64_t)ib * kD + col) = pack_bf16(y2, y3);
+        }
+    }
+}
+
+}  // namespace tiled
+}  // namespace ca

@@ -148,3 +148,49 @@ def test_fused_gmm_forced_ties():
                                                       iters=w.iters, W=w.W, alpha=w.alpha, hist=True)
     np.testing.assert_array_equal(g["hist"], ref_hist)
     np.testing.assert_array_equal(g["cent"], ref_cent)
+
+
+# Shapes served by the tiled bf16 path (L > 512 or floor(W/2) > 16, K <= 64,
+# floor(W/2) <= 128): tile and chunk tails, K at the padding boundaries,
+# windows wider than a tile.
+TILED_CASES = [
+    # L, K, iters, W, alpha, B, H
+    (513, 1, 2, 32, 0.5, 1, 2),
+    (1000, 17, 3, 0, 0.4, 1, 2),
+    (1537, 33, 1, 65, 0.3, 1, 1),
+    (2048, 64, 4, 129, 0.6, 1, 1),
+    (300, 16, 3, 100, 0.5, 2, 1),
+    (4095, 32, 0, 256, 0.5, 1, 1),
+]
+
+
+@pytest.mark.parametrize("L,K,iters,W,alpha,B,H", TILED_CASES)
+def test_tiled_path_parity(L, K, iters, W, alpha, B, H):
+    from means_cluster_attention_b200 import _lib
+    w = Workload("tiled", B, H, L, 64, K, iters, W, alpha, "bf16", "normal")
+    x = make_inputs(w, seed=L + 3 * K)
+    _lib.profile_start("tiled_window")
+    g = run_gpu(x, "bf16", K, iters, W, alpha, hist=iters > 0)
+    assert _lib.profile_stop().launches == 1, "the tiled path did not run"
+    ref_out, ref_assign, ref_cent, ref_hist = oracle.forward(
+        x["q64"], x["k64"], x["v64"], K=K, iters=iters, W=W, alpha=alpha, hist=True)
+    if iters > 0:
+        np.testing.assert_array_equal(g["hist"], ref_hist)
+    np.testing.assert_array_equal(g["assign"], ref_assign)
+    np.testing.assert_array_equal(g["cent"], ref_cent)
+    err = float(np.abs(g["out"] - ref_out).max())
+    assert err <= TOL["bf16"], err
+
+
+def test_tiled_forced_ties_across_tiles():
+    from means_cluster_attention_b200 import _lib
+    w = Workload("tiled_dup", 1, 2, 2500, 64, 48, 4, 64, 0.5, "bf16", "gmm", gmm_components=10,
+                 gmm_std=0.05, dup_frac=0.1)
+    x = make_inputs(w, seed=21)
+    _lib.profile_start("tiled_assign")
+    g = run_gpu(x, "bf16", w.K, w.iters, w.W, w.alpha, hist=True)
+    assert _lib.profile_stop().launches == w.iters
+    _, ref_assign, ref_cent, ref_hist = oracle.forward(x["q64"], x["k64"], x["v64"], K=w.K,
+                                                      iters=w.iters, W=w.W, alpha=w.alpha, hist=True)
+    np.testing.assert_array_equal(g["hist"], ref_hist)
+    np.testing.assert_array_equal(g["cent"], ref_cent)
