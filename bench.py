@@ -55,6 +55,22 @@ def dist_info():
     return ws, rank, local
 
 
+def reduce_max(values, dist=None, device=None):
+    """Element-wise max of a list of floats over all ranks (identity alone)."""
+    if dist is None:
+        return [float(x) for x in values]
+    import torch
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_rate(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Weak scaling: every rank processes its own full workload; the job's
+    throughput is all ranks' tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms_per_step / 1e3)
+
+
 def measured_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -245,11 +261,8 @@ def run_ours(args, w):
     ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms_step = sum(ms) / len(ms)
     k_ms = kstat.total_ms / max(1, kstat.launches)
-    if pg:
-        t = torch.tensor([ms_step, k_ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_step, k_ms = float(t[0]), float(t[1])
-    value = w.tokens * ws / (ms_step / 1e3)
+    ms_step, k_ms = reduce_max([ms_step, k_ms], pg, dev)
+    value = whole_job_rate(w.tokens, ws, ms_step)
 
     # End to end through the C ABI with host buffers (pinned), copies included.
     e2e = None
@@ -267,13 +280,9 @@ def run_ours(args, w):
             e_ev.record()
             torch.cuda.synchronize()
             e_ms.append(s_ev.elapsed_time(e_ev))
-        e_step = sum(e_ms) / len(e_ms)
-        if pg:
-            t = torch.tensor([e_step], device=dev, dtype=torch.float64)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e_step = float(t[0])
+        e_step = reduce_max([sum(e_ms) / len(e_ms)], pg, dev)[0]
         nbytes = q.numel() * q.element_size()
-        e2e = {"value": w.tokens * ws / (e_step / 1e3), "unit": UNIT, "h2d_bytes_per_step": 3 * nbytes,
+        e2e = {"value": whole_job_rate(w.tokens, ws, e_step), "unit": UNIT, "h2d_bytes_per_step": 3 * nbytes,
                "d2h_bytes_per_step": nbytes, "ms_per_step": e_step}
 
     peak, peak_kind = measured_peak()

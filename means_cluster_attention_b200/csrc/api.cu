@@ -218,7 +218,7 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     mp.cent_out = p.iters == 0 ? cent_out : nullptr;
     {
         Launch pl("tiled_init", st, 0.0);
-        tiled::tiled_mu_kernel<<<dim3(Kp, (unsigned)NH), 64, 0, st>>>(mp);
+        tiled::tiled_mu_kernel<<<dim3(Kp, (unsigned)NH), 256, 0, st>>>(mp);
         pl.after();
     }
     CA_CUDA(cudaGetLastError());
@@ -251,7 +251,7 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         mp.cent_out = t == p.iters - 1 ? cent_out : nullptr;
         {
             Launch pl("tiled_update", st, 0.0);
-            tiled::tiled_mu_kernel<<<dim3(Kp, (unsigned)NH), 64, 0, st>>>(mp);
+            tiled::tiled_mu_kernel<<<dim3(Kp, (unsigned)NH), 256, 0, st>>>(mp);
             pl.after();
         }
         CA_CUDA(cudaGetLastError());
@@ -276,7 +276,7 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     CA_CUDA(cudaGetLastError());
     {
         Launch pl("tiled_combine", st, 0.0);
-        centroid_attn_combine_kernel<<<(unsigned)NH, 256, 0, st>>>(K, n_chunks, cpart, vcent);
+        tiled::tiled_combine_kernel<<<dim3(K, (unsigned)NH), 64, 0, st>>>(K, n_chunks, cpart, vcent);
         pl.after();
     }
     CA_CUDA(cudaGetLastError());

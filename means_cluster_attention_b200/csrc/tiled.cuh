@@ -58,8 +58,8 @@ __host__ __device__ inline int kpad(int K) { return K <= 16 ? 16 : (K <= 32 ? 32
 // Centroid set: mu^(0) or the update from per-tile partial sums.
 struct MuParams {
     const __nv_bfloat16 *q;
-    const double *part_sum;  // [NH][n_tiles][Kp][64]
-    const int *part_cnt;     // [NH][n_tiles][Kp]
+    const double *part_sum;  // [NH][Kp][n_tiles][64]
+    const int *part_cnt;     // [NH][Kp][n_tiles]
     float *mu;               // [NH][Kp][64]
     __nv_bfloat16 *hi, *lo;  // [NH][Kp][64]
     float *mm;               // [NH][Kp]
@@ -68,29 +68,42 @@ struct MuParams {
     int L, K, Kp, n_tiles, init;
 };
 
-// grid (Kp, NH), 64 threads: thread j owns coordinate j of centroid k.
-__global__ void __launch_bounds__(64) tiled_mu_kernel(MuParams P) {
+// grid (Kp, NH), 256 threads: thread (g4, j) adds tiles g4, g4+4, ... of
+// coordinate j of centroid k; the four exact partial sums are then added in
+// fixed order by group 0, which finalises the centroid row.
+__global__ void __launch_bounds__(256) tiled_mu_kernel(MuParams P) {
+    __shared__ double red_s[3][64];
+    __shared__ int red_c[4];
     __shared__ float red_sq[2];
     __shared__ uint32_t red_h[2];
-    const int k = blockIdx.x, j = threadIdx.x, lane = j & 31, wid = j >> 5;
+    const int k = blockIdx.x, j = threadIdx.x & 63, g4 = threadIdx.x >> 6;
+    const int lane = threadIdx.x & 31, wid = (threadIdx.x >> 5) & 1;
     const int64_t head = blockIdx.y;
+    const int64_t kb = head * P.Kp + k;
+    double s = 0.0;
+    int cnt = 0;
+    if (!P.init && k < P.K) {
+        for (int tt = g4; tt < P.n_tiles; tt += 4) {
+            s += P.part_sum[(kb * P.n_tiles + tt) * kD + j];
+            if (j == 0) cnt += P.part_cnt[kb * P.n_tiles + tt];
+        }
+    }
+    if (g4 > 0) red_s[g4 - 1][j] = s;
+    if (j == 0) red_c[g4] = cnt;
+    __syncthreads();
+    if (g4 != 0) return;
     float x = 0.f;
     if (k < P.K) {
         if (P.init) {
             const int64_t row = ((int64_t)k * P.L) / P.K;
             x = __bfloat162float(P.q[(head * P.L + row) * kD + j]);
         } else {
-            double s = 0.0;
-            int cnt = 0;
-            for (int t = 0; t < P.n_tiles; ++t) {
-                const int64_t base = (head * P.n_tiles + t) * P.Kp + k;
-                s += P.part_sum[base * kD + j];
-                cnt += P.part_cnt[base];
-            }
-            x = __double2float_rn(s / (double)(cnt > 1 ? cnt : 1));
+            const double tot = ((s + red_s[0][j]) + red_s[1][j]) + red_s[2][j];
+            const int n = red_c[0] + red_c[1] + red_c[2] + red_c[3];
+            x = __double2float_rn(tot / (double)(n > 1 ? n : 1));
         }
     }
-    const int64_t o = (head * P.Kp + k) * kD + j;
+    const int64_t o = kb * kD + j;
     P.mu[o] = x;
     const __nv_bfloat16 h = __float2bfloat16_rn(x);
     P.hi[o] = h;
@@ -107,11 +120,28 @@ __global__ void __launch_bounds__(64) tiled_mu_kernel(MuParams P) {
         red_sq[wid] = sq;
         red_h[wid] = hv;
     }
-    __syncthreads();
+    asm volatile("bar.sync 1, 64;");
     if (j == 0) {
-        P.mm[head * P.Kp + k] = red_sq[0] + red_sq[1];
-        P.hash[head * P.Kp + k] = red_h[0] + red_h[1];
+        P.mm[kb] = red_sq[0] + red_sq[1];
+        P.hash[kb] = red_h[0] + red_h[1];
     }
+}
+
+// Centroid-attention combine for the tiled path: grid (K, NH), 64 threads.
+__global__ void __launch_bounds__(64) tiled_combine_kernel(int K, int n_chunks, const float *__restrict__ part,
+                                                            float *__restrict__ vcent) {
+    const int k = blockIdx.x, t = threadIdx.x;
+    const int64_t h = blockIdx.y;
+    float M = -INFINITY;
+    for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, part[((h * n_chunks + c) * K + k) * (kD + 2) + kD]);
+    float lsum = 0.f, acc = 0.f;
+    for (int c = 0; c < n_chunks; ++c) {
+        const float *p = part + ((h * n_chunks + c) * K + k) * (kD + 2);
+        const float w = expf(p[kD] - M);
+        lsum = fmaf(p[kD + 1], w, lsum);
+        acc = fmaf(p[t], w, acc);
+    }
+    vcent[(h * K + k) * kD + t] = acc / lsum;
 }
 
 // ---------------------------------------------------------------------------
@@ -126,10 +156,12 @@ struct AssignLayout {
         uint32_t o = 0;
         q_off = o;
         o += (uint32_t)Tp * 128u;
+        // Member sums stay in shared memory when they fit beside two CTAs per
+        // SM (Kp <= 32); for Kp = 64 they go straight to the tile's global slot.
         sums_off = o;
-        o += (uint32_t)Kp * 64u * 8u;
-        mu_off = o;
-        o += up((uint32_t)Kp * 65u * 4u, 128);
+        if (Kp <= 32) o += (uint32_t)Kp * 64u * 8u;
+        mu_off = o;  // fp32 centroid copy (rows padded to 65) for the exact re-measure
+        o += up((uint32_t)Kp * 65u * 4u, 16);
         hi_off = o;
         o += (uint32_t)Kp * 128u;
         lo_off = o;
@@ -169,12 +201,12 @@ struct AssignParams {
     int32_t *assign;     // [NH][L]
     int32_t *hist;       // [NH][iters][L] or null (already offset by the iteration)
     int64_t hist_stride; // iters * L
-    double *part_sum;    // [NH][n_tiles][Kp][64]
-    int *part_cnt;       // [NH][n_tiles][Kp]
+    double *part_sum;    // [NH][Kp][n_tiles][64]
+    int *part_cnt;       // [NH][Kp][n_tiles]
     int L, K, n_tiles;
 };
 
-__global__ void __launch_bounds__(kThreads, 1) tiled_assign_kernel(AssignParams P) {
+__global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams P) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const AssignLayout lay(P.K);
     const int K = P.K, Kp = lay.Kp;
@@ -188,8 +220,6 @@ __global__ void __launch_bounds__(kThreads, 1) tiled_assign_kernel(AssignParams 
     const uint32_t sbase = smem_u32(smem);
     const uint32_t q_s = sbase + lay.q_off, hi_s = sbase + lay.hi_off, lo_s = sbase + lay.lo_off;
     unsigned char *qbytes = smem + lay.q_off;
-    double *sums = reinterpret_cast<double *>(smem + lay.sums_off);
-    float *mu = reinterpret_cast<float *>(smem + lay.mu_off);
     float *mm = reinterpret_cast<float *>(smem + lay.mm_off);
     uint32_t *hsh = reinterpret_cast<uint32_t *>(smem + lay.hash_off);
     int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
@@ -201,13 +231,22 @@ __global__ void __launch_bounds__(kThreads, 1) tiled_assign_kernel(AssignParams 
     uint16_t *perm = reinterpret_cast<uint16_t *>(smem + lay.perm_off);
     int16_t *table = reinterpret_cast<int16_t *>(smem + lay.table_off);
     int *misc = reinterpret_cast<int *>(smem + lay.misc_off);
+    const bool smem_sums = Kp <= 32;
+    double *ssum = reinterpret_cast<double *>(smem + lay.sums_off);  // [Kp][64] when smem_sums
 
     load_rows(q_s, qh, 0, kTileQ, Lt);
     cp_async_commit();
     const int64_t cb = head * Kp;
+    // [Kp][64] centroids: a shared-memory copy when it fits, else global (L2).
+    float *mu = reinterpret_cast<float *>(smem + lay.mu_off);  // [Kp][65]
+    constexpr int mu_ld = 65;
+    for (int e = threadIdx.x; e < Kp * kD; e += kThreads) mu[(e / kD) * 65 + e % kD] = P.mu[cb * kD + e];
+    // This tile's slots of the partial sums, cleared before the run sums add in.
+    double *psum = P.part_sum;
     for (int e = threadIdx.x; e < Kp * kD; e += kThreads) {
         const int kk = e / kD, j = e % kD;
-        mu[kk * 65 + j] = P.mu[(cb + kk) * kD + j];
+        if (smem_sums) ssum[e] = 0.0;
+        else psum[((cb + kk) * P.n_tiles + tile) * kD + j] = 0.0;
     }
     for (int e = threadIdx.x; e < Kp * 8; e += kThreads) {
         const int kk = e >> 3, ch = e & 7;
@@ -233,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) tiled_assign_kernel(AssignParams 
                 if (hsh[a] != hsh[kk]) continue;
                 bool same = true;
                 for (int j = 0; j < kD && same; ++j)
-                    same = __float_as_uint(mu[a * 65 + j]) == __float_as_uint(mu[kk * 65 + j]);
+                    same = __float_as_uint(mu[a * mu_ld + j]) == __float_as_uint(mu[kk * mu_ld + j]);
                 dd = same;
             }
             dead[kk] = dd ? 1 : 0;
@@ -379,8 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1) tiled_assign_kernel(AssignParams 
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                mj0[u] = v0 ? (double)mu[k0 * 65 + jb + u] : 0.0;
-                mj1[u] = v1 ? (double)mu[k1 * 65 + jb + u] : 0.0;
+                mj0[u] = v0 ? (double)mu[k0 * mu_ld + jb + u] : 0.0;
+                mj1[u] = v1 ? (double)mu[k1 * mu_ld + jb + u] : 0.0;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -429,7 +468,6 @@ __global__ void __launch_bounds__(kThreads, 1) tiled_assign_kernel(AssignParams 
     // stable counting sort of the tile's tokens by cluster
     const int nch = kTileQ / 32;
     for (int i = threadIdx.x; i < nch * Kp; i += kThreads) table[i] = 0;
-    for (int i = threadIdx.x; i < Kp * kD; i += kThreads) sums[i] = 0.0;
     __syncthreads();
     int my_c[2], my_rank[2];
 #pragma unroll
@@ -524,14 +562,17 @@ __global__ void __launch_bounds__(kThreads, 1) tiled_assign_kernel(AssignParams 
                 p += n;
                 if (n < 32) break;
             }
-            atomicAdd(&sums[c * kD + 2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
-            atomicAdd(&sums[c * kD + 2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
+            double *dst = smem_sums ? ssum + c * kD : psum + ((cb + c) * P.n_tiles + tile) * kD;
+            atomicAdd(&dst[2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
+            atomicAdd(&dst[2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
         }
     }
-    __syncthreads();
-    const int64_t pb = (head * P.n_tiles + tile) * Kp;
-    for (int e = threadIdx.x; e < Kp * kD; e += kThreads) P.part_sum[pb * kD + e] = sums[e];
-    for (int kk = threadIdx.x; kk < Kp; kk += kThreads) P.part_cnt[pb + kk] = cnt_s[kk];
+    if (smem_sums) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < Kp * kD; e += kThreads)
+            psum[((cb + e / kD) * P.n_tiles + tile) * kD + e % kD] = ssum[e];
+    }
+    for (int kk = threadIdx.x; kk < Kp; kk += kThreads) P.part_cnt[(cb + kk) * P.n_tiles + tile] = cnt_s[kk];
 }
 
 // ---------------------------------------------------------------------------
