@@ -90,7 +90,7 @@ def ncu_traffic(kernel: str, workload: str):
             d = json.load(f)
         e = d[workload][kernel]
         from means_cluster_attention_b200.build import source_hash
-        if e.get("source_hash") != source_hash():
+        if e.get("source_hash") != source_hash(kernel):
             return None
         return float(e["dram_bytes_per_launch"])
     except Exception:

@@ -34,10 +34,21 @@ def sources() -> list:
                   + [os.path.join(INCLUDE, "clusterattn.h")])
 
 
-def source_hash() -> str:
-    """Hash of every kernel and header source (identifies a kernel build)."""
+# Source files each profiled kernel is built from (its own code and the
+# headers it includes), for deciding whether recorded counters still apply.
+KERNEL_SOURCES = {
+    "fused_forward": ["fused.cuh", "mma.cuh", "common.cuh"],
+    "tiled_assign": ["tiled.cuh", "fused.cuh", "mma.cuh", "common.cuh"],
+    "tiled_window": ["tiled.cuh", "fused.cuh", "mma.cuh", "common.cuh"],
+    "tiled_centroid": ["tiled.cuh", "fused.cuh", "mma.cuh", "common.cuh"],
+}
+
+
+def source_hash(kernel: str = None) -> str:
+    """Hash of the sources a kernel is built from (all sources if None)."""
+    files = sources() if kernel is None else [os.path.join(CSRC, f) for f in KERNEL_SOURCES[kernel]]
     h = hashlib.sha256()
-    for s in sources():
+    for s in files:
         h.update(os.path.basename(s).encode())
         with open(s, "rb") as f:
             h.update(f.read())

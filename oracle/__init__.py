@@ -58,12 +58,15 @@ def _load():
             ci, cd = ctypes.c_int, ctypes.c_double
             lib.oracle_forward.argtypes = [dp, dp, dp, ci, ci, ci, ci, ci, ci, ci, cd, ci, dp, ip, dp, ip, ci]
             lib.oracle_forward_at.argtypes = [dp, dp, dp, ci, ci, ci, ci, ci, ci, ci, cd, ci, ip, dp, dp, ci]
+            u8p = ctypes.POINTER(ctypes.c_uint8)
+            lib.oracle_forward_ex.argtypes = [dp, dp, dp, ci, ci, ci, ci, ci, ci, ci, cd, ci, ci, ci, ci, ci,
+                                              u8p, ci, dp, ip, dp, ip, ci]
             lib.oracle_kmeans.argtypes = [dp, ci, ci, ci, ci, ci, ip, dp, ip]
             lib.oracle_update.argtypes = [dp, ip, ci, ci, ci, ci, dp]
             lib.oracle_distances.argtypes = [dp, dp, ci, ci, ci, dp]
             lib.oracle_centroid_attention.argtypes = [dp, dp, dp, ci, ci, ci, dp]
             lib.oracle_window_attention.argtypes = [dp, dp, dp, ci, ci, ci, dp]
-            for f in (lib.oracle_forward, lib.oracle_forward_at, lib.oracle_kmeans, lib.oracle_update,
+            for f in (lib.oracle_forward, lib.oracle_forward_at, lib.oracle_forward_ex, lib.oracle_kmeans, lib.oracle_update,
                       lib.oracle_distances, lib.oracle_centroid_attention, lib.oracle_window_attention):
                 f.restype = ctypes.c_int
             _lib = lib
@@ -113,6 +116,34 @@ def forward(q, k, v, K: int, iters: int, W: int, alpha: float, mu_f32: bool = Tr
                             int(bool(mu_f32)), _dp(out), _ip(assign), _dp(cent), _ip(hh),
                             nthreads or default_threads())
     _check(st, "forward")
+    return out, assign, cent, hh
+
+
+def forward_ex(q, k, v, K: int, iters: int, W: int, alpha: float, mu_f32: bool = True,
+               window_module: bool = False, empty_keep: bool = False, init_stride: bool = False,
+               soft_gather: bool = False, key_valid=None, H_kv: int = 0, hist: bool = False,
+               nthreads: Optional[int] = None):
+    """The forward with the variants of the card's module ([P2] section 5):
+    window_module (band |i-j| <= W; no local branch when W == 0 or W >= L),
+    empty_keep, init_stride (k * max(1, L // K)), soft_gather, key_valid
+    ([B, L] bool/uint8 or None) and grouped key/value heads (k, v of shape
+    [B, H_kv, L, d]).  Returns (out, assign, centroids, hist)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, L, d = q.shape
+    out = np.empty_like(q)
+    assign = np.empty((B, H, L), dtype=np.int32)
+    cent = np.empty((B, H, K, d), dtype=np.float64)
+    hh = np.empty((B, H, iters, L), dtype=np.int32) if hist else None
+    kv = None
+    if key_valid is not None:
+        kv = np.ascontiguousarray(key_valid, dtype=np.uint8).reshape(B, L)
+    kvp = None if kv is None else kv.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+    st = _load().oracle_forward_ex(_dp(q), _dp(k), _dp(v), B, H, L, d, K, iters, W, float(alpha),
+                                   int(bool(mu_f32)), int(bool(window_module)), int(bool(empty_keep)),
+                                   int(bool(init_stride)), int(bool(soft_gather)), kvp, int(H_kv),
+                                   _dp(out), _ip(assign), _dp(cent), _ip(hh),
+                                   nthreads or default_threads())
+    _check(st, "forward_ex")
     return out, assign, cent, hh
 
 

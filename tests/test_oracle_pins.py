@@ -326,3 +326,104 @@ def test_invalid_arguments_rejected():
         oracle.forward(q, q, q, K=5, iters=1, W=2, alpha=0.5)  # K > L
     with pytest.raises(ValueError):
         oracle.forward(q, q, q, K=2, iters=1, W=2, alpha=1.5)
+
+
+# --------------------------------------------------------------------------
+# Variants of the card's module ([P2] section 5).
+
+# With everything off, the extended form is the plain forward.
+def test_ex_defaults_equal_plain():
+    q, k, v = (_f32(_rand((2, 3, 40, 64), s)) for s in (50, 51, 52))
+    a = oracle.forward(q, k, v, K=6, iters=3, W=10, alpha=0.4, hist=True)
+    b = oracle.forward_ex(q, k, v, K=6, iters=3, W=10, alpha=0.4, hist=True)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+# The module's window is the radius W; at alpha = 1 it is band-masked SDPA
+# with |i - j| <= W.  With W == 0 or W >= L it drops the local branch, so
+# the output is the gathered global context at any alpha.
+@pytest.mark.parametrize("W", [1, 5, 17])
+def test_ex_module_window_radius(W):
+    L = 30
+    q, k, v = (_rand((1, 2, L, 64), s) for s in (53, 54, 55))
+    out, *_ = oracle.forward_ex(q, k, v, K=4, iters=2, W=W, alpha=1.0, window_module=True)
+    idx = np.arange(L)
+    ref = _sdpa(q, k, v, mask=np.abs(idx[:, None] - idx[None, :]) <= W)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("W", [0, 30, 64])
+def test_ex_module_window_skipped(W):
+    q, k, v = (_rand((1, 2, 30, 64), s) for s in (56, 57, 58))
+    out, *_ = oracle.forward_ex(q, k, v, K=4, iters=2, W=W, alpha=0.7, window_module=True)
+    g, *_ = oracle.forward_ex(q, k, v, K=4, iters=2, W=3, alpha=0.0, window_module=True)
+    np.testing.assert_allclose(out, g, rtol=0, atol=1e-14)
+
+
+# The module's stride init: rows k * (L // K) (L=10, K=4 -> 0, 2, 4, 6).
+def test_ex_init_stride():
+    q = _f32(_rand((1, 1, 10, 64), 59))
+    _, _, cent, _ = oracle.forward_ex(q, q, q, K=4, iters=0, W=2, alpha=0.5, init_stride=True)
+    np.testing.assert_array_equal(cent[0, 0], q[0, 0][[0, 2, 4, 6]])
+
+
+# Empty cluster keeps its previous centroid (worked example: the tie case of
+# tests/golden, where cluster 1 is empty after one step and keeps (1, 0)).
+def test_ex_empty_keep_golden():
+    g = _golden()["kmeans_tie_and_empty"]
+    q = _pad64(np.asarray(g["Q"], dtype=np.float64))[None, None]
+    _, assign, cent, _ = oracle.forward_ex(q, q, q, K=2, iters=1, W=2, alpha=0.5, empty_keep=True)
+    np.testing.assert_array_equal(assign[0, 0], g["assign"])
+    np.testing.assert_array_equal(cent[0, 0, 0, :2], g["centroids"][0])
+    np.testing.assert_array_equal(cent[0, 0, 1, :2], [1.0, 0.0])
+
+
+# Soft gather: g_i = softmax(Q_i mu^T / sqrt(d)) V_cent and V_cent =
+# softmax(mu K^T / sqrt(d)) V, i.e. two nested SDPA calls on the oracle's
+# own centroids.
+def test_ex_soft_gather_is_nested_sdpa():
+    q, k, v = (_f32(_rand((1, 2, 36, 64), s)) for s in (60, 61, 62))
+    out, assign, cent, _ = oracle.forward_ex(q, k, v, K=5, iters=3, W=6, alpha=0.0, soft_gather=True)
+    vcent = _sdpa(cent, k, v)
+    ref = _sdpa(q, cent, vcent)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+# Key-padding mask: invalid keys take no weight in either branch and rows of
+# invalid queries are zero.  At alpha = 1 the valid rows equal band-masked
+# SDPA restricted to valid keys; at alpha = 0 with K = L they equal dense
+# SDPA restricted to valid keys.
+def test_ex_key_padding_mask():
+    B, H, L = 2, 2, 24
+    q, k, v = (_f32(_rand((B, H, L, 64), s)) for s in (63, 64, 65))
+    valid = np.ones((B, L), dtype=bool)
+    valid[0, 17:] = False
+    valid[1, [0, 5, 6, 23]] = False
+    idx = np.arange(L)
+    band = np.abs(idx[:, None] - idx[None, :]) <= 4
+    out1, *_ = oracle.forward_ex(q, k, v, K=3, iters=2, W=8, alpha=1.0, key_valid=valid)
+    out0, *_ = oracle.forward_ex(q, k, v, K=L, iters=2, W=8, alpha=0.0, key_valid=valid)
+    for b in range(B):
+        m1 = band & valid[b][None, :]
+        m0 = np.broadcast_to(valid[b][None, :], (L, L))
+        r1 = _sdpa(q[b:b + 1], k[b:b + 1], v[b:b + 1], mask=np.ascontiguousarray(m1))
+        r0 = _sdpa(q[b:b + 1], k[b:b + 1], v[b:b + 1], mask=np.ascontiguousarray(m0))
+        rows = valid[b]
+        np.testing.assert_allclose(out1[b][:, rows], r1[0][:, rows], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(out0[b][:, rows], r0[0][:, rows], rtol=0, atol=1e-12)
+        assert (out1[b][:, ~rows] == 0).all() and (out0[b][:, ~rows] == 0).all()
+
+
+# Grouped key/value heads equal the plain forward on K, V repeated per group
+# (torch repeat_interleave along the head axis).
+def test_ex_grouped_kv_heads():
+    B, H, Hkv, L = 2, 6, 2, 20
+    q = _f32(_rand((B, H, L, 64), 66))
+    k, v = (_f32(_rand((B, Hkv, L, 64), s)) for s in (67, 68))
+    out, assign, cent, _ = oracle.forward_ex(q, k, v, K=4, iters=2, W=6, alpha=0.5, H_kv=Hkv)
+    kr = torch.from_numpy(k).repeat_interleave(H // Hkv, dim=1).numpy()
+    vr = torch.from_numpy(v).repeat_interleave(H // Hkv, dim=1).numpy()
+    ref, ref_a, ref_c, _ = oracle.forward(q, kr, vr, K=4, iters=2, W=6, alpha=0.5)
+    np.testing.assert_array_equal(out, ref)
+    np.testing.assert_array_equal(assign, ref_a)
