@@ -84,6 +84,43 @@ ca_status ca_forward_trace(const void *q, const void *k, const void *v, int dtyp
                            int32_t *assign_out, float *centroids_out, int32_t *assign_hist,
                            void *stream);
 
+/* Variants of the card's own module ("Hooshaai/svd-sst2-roberta-cluster",
+ * section 5), selected per call; all zero / NULL gives the forward above:
+ *   window_mode  0: window |i-j| <= floor(W/2) (default);
+ *                1: the module's radius |i-j| <= W, and no local branch at
+ *                   all (O = gathered) when W == 0 or W >= L;
+ *   empty_mode   0: an empty cluster becomes the zero vector (default);
+ *                1: an empty cluster keeps its previous centroid;
+ *   init_mode    0: mu_k = Q[floor(k L / K)] (default);
+ *                1: mu_k = Q[k * max(1, L / K)] (the module's stride);
+ *   gather_mode  0: hard gather V_cent[c_i] (default);
+ *                1: soft assignment softmax(Q_i mu^T / sqrt(d)) V_cent;
+ *   key_valid    [B, L] device bytes (1 = valid) or NULL: invalid keys take
+ *                no weight in either softmax (a row with no valid key weighs
+ *                every key equally, as the module's all -10000 row does) and
+ *                output rows of invalid queries are zero; k-means still
+ *                clusters every query, as the module does;
+ *   H_kv         key/value heads (0 means H); k and v are [B, H_kv, L, d]
+ *                and query head h reads key/value head h / (H / H_kv).
+ * Unknown mode values or an H_kv that does not divide H return
+ * CA_ERR_INVALID_ARG. */
+typedef struct {
+    int window_mode;
+    int empty_mode;
+    int init_mode;
+    int gather_mode;
+    const uint8_t *key_valid;
+    int H_kv;
+} ca_options;
+
+/* ca_forward_trace with the variants of ca_options (opt may be NULL).  Calls
+ * whose options are all defaults take the same kernels as ca_forward_trace;
+ * any other option runs the general multi-kernel path. */
+ca_status ca_forward_ex(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                        int L, int d, int K, int iters, int W, float alpha, const ca_options *opt,
+                        void *out, int32_t *assign_out, float *centroids_out, int32_t *assign_hist,
+                        void *stream);
+
 /* End-to-end form for callers holding HOST buffers (dtype 0 = fp32 with float
  * arrays, 1 = bf16 with uint16 arrays): copies q, k, v to the device, runs the
  * forward on stream, copies out (and assign_out / centroids_out when non-NULL)

@@ -5,6 +5,6 @@ behind the C ABI declared in ``include/clusterattn.h``); this package holds
 the ctypes binding, the in-tree build script and the seeded input generator.
 """
 
-from ._lib import ClusterAttnError, forward, forward_host, load, sync_status  # noqa: F401
+from ._lib import ClusterAttnError, forward, forward_ex, forward_host, load, sync_status  # noqa: F401
 
-__all__ = ["forward", "forward_host", "load", "sync_status", "ClusterAttnError"]
+__all__ = ["forward", "forward_ex", "forward_host", "load", "sync_status", "ClusterAttnError"]

@@ -25,6 +25,7 @@ SIGNATURES = {
     "ca_forward_bf16": ([_vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp], _ci),
     "ca_forward_trace": ([_vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp, _vp], _ci),
     "ca_forward_host": ([_vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp], _ci),
+    "ca_forward_ex": ([_vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp, _vp, _vp], _ci),
     "ca_forward_noalloc": ([_vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp], _ci),
     "ca_sync_status": ([_vp], _ci),
     "ca_status_string": ([_ci], ctypes.c_char_p),
@@ -34,6 +35,12 @@ SIGNATURES = {
     "ca_profile_stop": ([_vp], _ci),
     "ca_launch_count": ([], ctypes.c_longlong),
 }
+
+
+class Options(ctypes.Structure):
+    """Mirror of ca_options (include/clusterattn.h)."""
+    _fields_ = [("window_mode", ctypes.c_int), ("empty_mode", ctypes.c_int), ("init_mode", ctypes.c_int),
+                ("gather_mode", ctypes.c_int), ("key_valid", ctypes.c_void_p), ("H_kv", ctypes.c_int)]
 
 
 class KernelStat(ctypes.Structure):
@@ -117,6 +124,48 @@ def forward(q, k, v, K: int, iters: int, W: int, alpha: float, out=None, assign=
     st = lib.ca_forward_trace(_ptr(q), _ptr(k), _ptr(v), dtype, B, H, L, d, K, int(iters), int(W),
                               float(alpha), _ptr(out), _ptr(assign), _ptr(centroids),
                               _ptr(assign_hist), _stream_handle(stream))
+    check(st)
+    if sync_check:
+        check(lib.ca_sync_status(_stream_handle(stream)))
+    return out, assign, centroids
+
+
+def forward_ex(q, k, v, K: int, iters: int, W: int, alpha: float, window_mode: int = 0,
+               empty_mode: int = 0, init_mode: int = 0, gather_mode: int = 0, key_valid=None,
+               out=None, assign=None, centroids=None, assign_hist=None, stream=None,
+               sync_check: bool = False) -> Tuple:
+    """The forward with the variants of the card's module (see ca_options):
+    q is [B, H, L, d]; k and v are [B, H_kv, L, d] (grouped key/value heads);
+    key_valid is a [B, L] bool/uint8 CUDA tensor or None."""
+    import torch
+    if q.device.type != "cuda":
+        raise ValueError("q, k, v must be CUDA tensors")
+    if not (q.dtype == k.dtype == v.dtype) or q.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("q, k, v must share dtype float32 or bfloat16")
+    if k.shape != v.shape or q.dim() != 4 or k.dim() != 4 or q.shape[0] != k.shape[0] or q.shape[2:] != k.shape[2:]:
+        raise ValueError("q must be [B, H, L, d] and k, v [B, H_kv, L, d]")
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+    B, H, L, d = q.shape
+    K = min(int(K), L)
+    kv = None
+    if key_valid is not None:
+        kv = key_valid.to(device=q.device, dtype=torch.uint8).contiguous()
+        if kv.numel() != B * L:
+            raise ValueError("key_valid must have B * L elements")
+    if out is None:
+        out = torch.empty_like(q)
+    if assign is None:
+        assign = torch.empty((B, H, L), dtype=torch.int32, device=q.device)
+    if centroids is None:
+        centroids = torch.empty((B, H, K, d), dtype=torch.float32, device=q.device)
+    opt = Options(int(window_mode), int(empty_mode), int(init_mode), int(gather_mode), _ptr(kv), int(k.shape[1]))
+    lib = load()
+    dtype = 0 if q.dtype == torch.float32 else 1
+    st = lib.ca_forward_ex(_ptr(q), _ptr(k), _ptr(v), dtype, B, H, L, d, K, int(iters), int(W), float(alpha),
+                           ctypes.byref(opt), _ptr(out), _ptr(assign), _ptr(centroids), _ptr(assign_hist),
+                           _stream_handle(stream))
     check(st)
     if sync_check:
         check(lib.ca_sync_status(_stream_handle(stream)))

@@ -242,6 +242,7 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     mp.init = 0;
     for (int t = 0; t < p.iters; ++t) {
         ap.hist = hist ? hist + (int64_t)t * L : nullptr;
+        ap.first = t == 0;
         {
             Launch pl("tiled_assign", st, head_bytes);
             tiled::tiled_assign_kernel<<<dim3(n_tiles, (unsigned)NH), tiled::kThreads, alay.total, st>>>(ap);
@@ -303,10 +304,19 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     return CA_OK;
 }
 
+// Options of the module's variants for the general path (defaults: none).
+struct ExOpts {
+    int init_stride = 0, empty_keep = 0, r = -1;  // r < 0: floor(W / 2)
+    ca::Variant var;
+};
+
 template <typename T>
 ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *out,
-                      int32_t *assign_out, float *cent_out, int32_t *hist, cudaStream_t st) {
+                      int32_t *assign_out, float *cent_out, int32_t *hist, cudaStream_t st,
+                      const ExOpts *ex = nullptr) {
     using namespace ca;
+    const ExOpts dflt;
+    const ExOpts &xo = ex ? *ex : dflt;
     const int64_t NH = p.heads();
     const int L = p.L, K = p.K;
     const float scale = 1.0f / sqrtf((float)p.d);
@@ -329,7 +339,7 @@ ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *o
     // 1. strided init (and c = 0 for iters == 0)
     {
         Launch pl("kmeans_init", st, 0.0);
-        kmeans_init_kernel<T><<<(unsigned)NH, 256, 0, st>>>(q, L, K, mu);
+        kmeans_init_kernel<T><<<(unsigned)NH, 256, 0, st>>>(q, L, K, mu, xo.init_stride);
         pl.after();
     }
     CA_CUDA(cudaGetLastError());
@@ -357,7 +367,8 @@ ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *o
         {
             Launch pl("kmeans_update", st, 0.0);
             kmeans_update_kernel<<<(unsigned)NH, 256, 0, st>>>(K, sums, counts, mu,
-                                                                t == p.iters - 1 ? cent_out : nullptr);
+                                                                t == p.iters - 1 ? cent_out : nullptr,
+                                                                xo.empty_keep);
             pl.after();
         }
         CA_CUDA(cudaGetLastError());
@@ -369,7 +380,7 @@ ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *o
     {
         Launch pl("centroid_attn", st, 2.0 * head_bytes);
         centroid_attn_partial_kernel<T><<<dim3(n_chunks, (unsigned)NH), kCaThreads, csmem, st>>>(
-            k, v, L, K, scale, mu, n_chunks, part);
+            k, v, L, K, scale, mu, n_chunks, part, xo.var);
         pl.after();
     }
     CA_CUDA(cudaGetLastError());
@@ -385,8 +396,10 @@ ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *o
     CA_CUDA(cudaFuncSetAttribute(window_blend_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem));
     {
         Launch pl("window_blend", st, 4.0 * head_bytes);
+        Variant wv = xo.var;
+        wv.mu = mu;
         window_blend_kernel<T><<<dim3((L + kWinQ - 1) / kWinQ, (unsigned)NH), kWinThreads, wsmem, st>>>(
-            q, k, v, L, K, p.W / 2, scale, p.alpha, vcent, assign, out);
+            q, k, v, L, K, xo.r >= 0 ? xo.r : p.W / 2, scale, p.alpha, vcent, assign, out, wv);
         pl.after();
     }
     CA_CUDA(cudaGetLastError());
@@ -440,6 +453,44 @@ ca_status ca_forward_trace(const void *q, const void *k, const void *v, int dtyp
                            void *stream) {
     Problem p{B, H, L, d, K, iters, W, alpha};
     return dispatch(q, k, v, dtype, p, out, assign_out, centroids_out, assign_hist, stream);
+}
+
+ca_status ca_forward_ex(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                        int L, int d, int K, int iters, int W, float alpha, const ca_options *opt,
+                        void *out, int32_t *assign_out, float *centroids_out, int32_t *assign_hist,
+                        void *stream) {
+    Problem p{B, H, L, d, K, iters, W, alpha};
+    if (!opt) return dispatch(q, k, v, dtype, p, out, assign_out, centroids_out, assign_hist, stream);
+    const ca_options &o = *opt;
+    if ((o.window_mode | o.empty_mode | o.init_mode | o.gather_mode) & ~1)
+        return fail(CA_ERR_INVALID_ARG, "window_mode, empty_mode, init_mode and gather_mode must be 0 or 1");
+    const int H_kv = o.H_kv == 0 ? H : o.H_kv;
+    if (H_kv < 1 || H < 1 || H % H_kv != 0)
+        return fail(CA_ERR_INVALID_ARG, "H_kv must divide H (got H=%d, H_kv=%d)", H, o.H_kv);
+    const bool plain = !o.window_mode && !o.empty_mode && !o.init_mode && !o.gather_mode && !o.key_valid && H_kv == H;
+    if (plain) return dispatch(q, k, v, dtype, p, out, assign_out, centroids_out, assign_hist, stream);
+    ca_status s = validate(q, k, v, out, p);
+    if (s != CA_OK) return s;
+    if (((uintptr_t)centroids_out & 15u) || ((uintptr_t)assign_out & 3u) || ((uintptr_t)assign_hist & 3u))
+        return fail(CA_ERR_INVALID_ARG, "centroids_out must be 16-byte aligned, assign buffers 4-byte aligned");
+    ExOpts ex;
+    ex.init_stride = o.init_mode;
+    ex.empty_keep = o.empty_mode;
+    ex.r = o.window_mode ? W : W / 2;
+    ex.var.H = H;
+    ex.var.H_kv = H_kv;
+    ex.var.key_valid = o.key_valid;
+    ex.var.local = o.window_mode ? (W > 0 && W < L) : 1;
+    ex.var.soft = o.gather_mode;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == 0)
+        return run_forward<float>((const float *)q, (const float *)k, (const float *)v, p, (float *)out,
+                                  assign_out, centroids_out, assign_hist, st, &ex);
+    if (dtype == 1)
+        return run_forward<__nv_bfloat16>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
+                                          (const __nv_bfloat16 *)v, p, (__nv_bfloat16 *)out, assign_out,
+                                          centroids_out, assign_hist, st, &ex);
+    return fail(CA_ERR_INVALID_ARG, "dtype must be 0 (fp32) or 1 (bf16), got %d", dtype);
 }
 
 ca_status ca_forward_host(const void *q, const void *k, const void *v, int dtype, int B, int H,

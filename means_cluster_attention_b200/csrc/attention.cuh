@@ -29,7 +29,7 @@ template <typename T>
 __global__ void __launch_bounds__(kCaThreads)
     centroid_attn_partial_kernel(const T *__restrict__ kmat, const T *__restrict__ vmat, int L,
                                  int K, float scale, const float *__restrict__ mu, int n_chunks,
-                                 float *__restrict__ part) {
+                                 float *__restrict__ part, Variant var = Variant()) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *mu_s = reinterpret_cast<float *>(smem_raw);
     float *ks = mu_s + (size_t)K * kD;            // [kCaTile][kD + 1]
@@ -37,8 +37,18 @@ __global__ void __launch_bounds__(kCaThreads)
 
     const int h = blockIdx.y, chunk = blockIdx.x;
     const int j0 = chunk * kCaChunk, j1 = min(L, j0 + kCaChunk);
-    const T *kh = kmat + (int64_t)h * L * kD;
-    const T *vh = vmat + (int64_t)h * L * kD;
+    const int64_t hkv = var.kv_head(h);
+    const T *kh = kmat + hkv * L * kD;
+    const T *vh = vmat + hkv * L * kD;
+    // Key-padding mask: invalid keys take no weight; a row with no valid key
+    // at all gives every key the same weight (the module's all -10000 row).
+    const uint8_t *kvp = var.key_valid ? var.key_valid + var.batch(h) * L : nullptr;
+    int any_valid = 1;
+    if (kvp) {
+        int mine = 0;
+        for (int j = threadIdx.x; j < L; j += blockDim.x) mine |= kvp[j];
+        any_valid = __syncthreads_or(mine);
+    }
     for (int idx = threadIdx.x; idx < K * kD; idx += blockDim.x) mu_s[idx] = mu[(int64_t)h * K * kD + idx];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -79,6 +89,10 @@ __global__ void __launch_bounds__(kCaThreads)
             }
             z0 = lane < nt ? z0 * scale : -INFINITY;
             z1 = lane + 32 < nt ? z1 * scale : -INFINITY;
+            if (kvp) {
+                if (lane < nt) z0 = any_valid ? (kvp[tb + lane] ? z0 : -INFINITY) : 0.f;
+                if (lane + 32 < nt) z1 = any_valid ? (kvp[tb + lane + 32] ? z1 : -INFINITY) : 0.f;
+            }
             const float tmax = warp_max(fmaxf(z0, z1));
             const float m_new = fmaxf(m_r[c], tmax);
             const float corr = expf(m_r[c] - m_new);
@@ -142,7 +156,7 @@ __global__ void __launch_bounds__(kWinThreads)
     window_blend_kernel(const T *__restrict__ q, const T *__restrict__ kmat,
                         const T *__restrict__ vmat, int L, int K, int r, float scale, float alpha,
                         const float *__restrict__ vcent, const int32_t *__restrict__ assign,
-                        T *__restrict__ out) {
+                        T *__restrict__ out, Variant var = Variant()) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     float *ks = reinterpret_cast<float *>(smem_raw);  // [kCaTile][kD + 1]
     float *vs = ks + (size_t)kCaTile * (kD + 1);      // [kCaTile][kD]
@@ -152,11 +166,18 @@ __global__ void __launch_bounds__(kWinThreads)
     const unsigned gmask = 0xFu << (threadIdx.x & 28);
     const bool valid = qi < L;
     const int64_t hoff = (int64_t)h * L * kD;
+    const int64_t kvoff = var.kv_head(h) * L * kD;
+    const uint8_t *kvp = var.key_valid ? var.key_valid + var.batch(h) * L : nullptr;
 
     float qf[16];
 #pragma unroll
     for (int t = 0; t < 16; ++t) qf[t] = valid ? to_f32(q[hoff + (int64_t)qi * kD + 16 * sub + t]) : 0.f;
     const int lo_q = max(0, qi - r), hi_q = min(L - 1, qi + r);
+    int band_any = 1;  // some valid key in this query's window
+    if (kvp && valid) {
+        band_any = 0;
+        for (int j = lo_q; j <= hi_q && !band_any; ++j) band_any = kvp[j];
+    }
     const int i_last = min(L - 1, i0 + kWinQ - 1);
     const int lo = max(0, i0 - r), hi = min(L - 1, i_last + r);
 
@@ -164,15 +185,15 @@ __global__ void __launch_bounds__(kWinThreads)
 #pragma unroll
     for (int t = 0; t < 16; ++t) acc[t] = 0.f;
 
-    for (int tb = lo; tb <= hi; tb += kCaTile) {
+    for (int tb = lo; tb <= hi && var.local; tb += kCaTile) {
         const int nt = min(kCaTile, hi - tb + 1);
         __syncthreads();
         for (int idx = threadIdx.x; idx < kCaTile * kD; idx += blockDim.x) {
             const int rr = idx / kD, t = idx % kD;
             float kv = 0.f, vv = 0.f;
             if (rr < nt) {
-                kv = to_f32(kmat[hoff + (int64_t)(tb + rr) * kD + t]);
-                vv = to_f32(vmat[hoff + (int64_t)(tb + rr) * kD + t]);
+                kv = to_f32(kmat[kvoff + (int64_t)(tb + rr) * kD + t]);
+                vv = to_f32(vmat[kvoff + (int64_t)(tb + rr) * kD + t]);
             }
             ks[rr * (kD + 1) + t] = kv;
             vs[rr * kD + t] = vv;
@@ -181,13 +202,14 @@ __global__ void __launch_bounds__(kWinThreads)
         if (valid) {
             const int jb = max(lo_q, tb), je = min(hi_q, tb + nt - 1);
             for (int j = jb; j <= je; ++j) {
+                if (kvp && band_any && !kvp[j]) continue;
                 const float *kr = ks + (j - tb) * (kD + 1) + 16 * sub;
                 float part = 0.f;
 #pragma unroll
                 for (int t = 0; t < 16; ++t) part = fmaf(qf[t], kr[t], part);
                 part += __shfl_xor_sync(gmask, part, 1);
                 part += __shfl_xor_sync(gmask, part, 2);
-                const float z = part * scale;
+                const float z = (kvp && !band_any) ? 0.f : part * scale;
                 if (z > m) {
                     const float corr = expf(m - z);
                     l *= corr;
@@ -204,12 +226,50 @@ __global__ void __launch_bounds__(kWinThreads)
         }
     }
     if (!valid) return;
-    const int c = assign[(int64_t)h * L + qi];
-    const float *g = vcent + ((int64_t)h * K + c) * kD + 16 * sub;
-    const float inv_l = 1.f / l;
+    // gathered global context: hard V_cent[c_i], or the soft assignment
+    float gv[16];
+    if (!var.soft) {
+        const int c = assign[(int64_t)h * L + qi];
+        const float *g = vcent + ((int64_t)h * K + c) * kD + 16 * sub;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) gv[t] = g[t];
+    } else {
+        float gm = -INFINITY, gl = 0.f;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) gv[t] = 0.f;
+        for (int k = 0; k < K; ++k) {
+            const float *mk = var.mu + ((int64_t)h * K + k) * kD + 16 * sub;
+            float part = 0.f;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) part = fmaf(qf[t], mk[t], part);
+            part += __shfl_xor_sync(gmask, part, 1);
+            part += __shfl_xor_sync(gmask, part, 2);
+            const float z = part * scale;
+            if (z > gm) {
+                const float corr = expf(gm - z);
+                gl *= corr;
+#pragma unroll
+                for (int t = 0; t < 16; ++t) gv[t] *= corr;
+                gm = z;
+            }
+            const float p = expf(z - gm);
+            gl += p;
+            const float *vk = vcent + ((int64_t)h * K + k) * kD + 16 * sub;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) gv[t] = fmaf(p, vk[t], gv[t]);
+        }
+        const float inv = 1.f / gl;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) gv[t] *= inv;
+    }
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    const bool zero_row = kvp && !kvp[qi];
     T *o = out + hoff + (int64_t)qi * kD + 16 * sub;
 #pragma unroll
-    for (int t = 0; t < 16; ++t) o[t] = from_f32<T>((1.f - alpha) * g[t] + alpha * (acc[t] * inv_l));
+    for (int t = 0; t < 16; ++t) {
+        const float y = var.local ? (1.f - alpha) * gv[t] + alpha * (acc[t] * inv_l) : gv[t];
+        o[t] = from_f32<T>(zero_row ? 0.f : y);
+    }
 }
 
 }  // namespace ca

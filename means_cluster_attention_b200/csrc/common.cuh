@@ -17,6 +17,21 @@ constexpr int kMaxK = 128;
 __device__ int g_dev_error;
 __device__ int g_dev_error_where;
 
+// Options of the general path for the variants of the card's module:
+// grouped key/value heads, key-padding masks, no local branch, soft gather.
+// The defaults leave the forward unchanged.
+struct Variant {
+    int H = 1, H_kv = 1;                  // query / key-value heads per batch row
+    const uint8_t *key_valid = nullptr;   // [B][L], 1 = valid key (and query)
+    int local = 1;                        // 0: no local branch, O = gathered
+    int soft = 0;                         // 1: soft gather softmax(Q mu^T s) V_cent
+    const float *mu = nullptr;            // [NH][K][64] final centroids (soft gather)
+    __host__ __device__ int64_t kv_head(int64_t h) const {
+        return (h / H) * H_kv + (h % H) / (H / H_kv);
+    }
+    __host__ __device__ int64_t batch(int64_t h) const { return h / H; }
+};
+
 __device__ __forceinline__ void record_error(int code, int where) {
     if (atomicCAS(&g_dev_error, 0, code) == 0) g_dev_error_where = where;
 }

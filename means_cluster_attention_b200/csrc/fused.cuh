@@ -26,9 +26,11 @@
 // copies of a lower-index centroid can never win (their distances are equal
 // and the lower index takes the tie) and are excluded up front.
 //
-// Member sums: tokens are ordered by cluster with a stable counting sort;
-// each warp walks a contiguous slice of the sorted tokens, turning bf16
-// values into doubles with integer operations and adding in fp64.  Those sums are exact for any input
+// Member sums: in the first iteration tokens are ordered by cluster with a
+// stable counting sort and each warp walks a contiguous slice of the sorted
+// tokens, turning bf16 values into doubles with integer operations and
+// adding in fp64; later iterations only subtract / add the tokens whose
+// cluster changed.  Those sums are exact for any input
 // whose non-zero magnitudes lie within 2^-27 .. 16, so the centroid
 // mu_k = fp32(sum / max(1, count)) does not depend on the order of the adds.
 #pragma once
@@ -57,7 +59,8 @@ __host__ __device__ inline uint32_t umax(uint32_t a, uint32_t b) { return a > b 
 struct Layout {
     int Lp, Kp, r, nT, win_rows;
     uint32_t big_off, sums_off, mu_off, hi_off, lo_off, vc_off, mm_off, hash_off, dead_off, c_off,
-        list_off, perm_off, sc_off, table_off, cnt_off, base_off, misc_off, ml_off, win_stage, total;
+        list_off, perm_off, sc_off, cprev_off, table_off, cnt_off, base_off, misc_off, ml_off, win_stage,
+        total;
 
     __host__ __device__ Layout(int L, int K, int r_) {
         Lp = (int)up((uint32_t)L, 64);
@@ -98,6 +101,8 @@ struct Layout {
         c_off = o;
         o += up((uint32_t)Lp, 16);
         sc_off = o;
+        o += up((uint32_t)Lp, 16);
+        cprev_off = o;
         o += up((uint32_t)Lp, 16);
         list_off = o;
         o += up((uint32_t)Lp * 2u, 16);
@@ -228,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     uint8_t *dead = smem + lay.dead_off;
     uint8_t *cs = smem + lay.c_off;                                              // [Lp]
     uint8_t *sc = smem + lay.sc_off;                                             // [Lp] sorted cluster ids
+    uint8_t *cprev = smem + lay.cprev_off;                                       // [Lp] previous assignment
     uint16_t *list = reinterpret_cast<uint16_t *>(smem + lay.list_off);
     uint16_t *perm = reinterpret_cast<uint16_t *>(smem + lay.perm_off);
     int16_t *table = reinterpret_cast<int16_t *>(smem + lay.table_off);           // [Lp/32][Kp]
@@ -332,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                 misc[1] = __float_as_int(mx);
                 misc[2] = __float_as_int(sqrtf(mx));
                 misc[0] = 0;
+                misc[3] = 0;
             }
         }
         __syncthreads();
@@ -493,117 +500,145 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
             int32_t *hrow = P.hist + (head * P.iters + it) * (int64_t)L;
             for (int i = threadIdx.x; i < L; i += kThreads) hrow[i] = cs[i];
         }
-        // (3) stable counting sort of the tokens by cluster
-        for (int i = threadIdx.x; i < nch * Kp; i += kThreads) table[i] = 0;
-        __syncthreads();
-        int my_c[2], my_rank[2];
+        if (it == 0) {
+            // (3) stable counting sort of the tokens by cluster
+            for (int i = threadIdx.x; i < nch * Kp; i += kThreads) table[i] = 0;
+            __syncthreads();
+            int my_c[2], my_rank[2];
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-            const int ch = warp + s * kWarps;
-            my_c[s] = 0xFF;
-            my_rank[s] = 0;
-            if (ch < nch) {
-                const int c = cs[ch * 32 + lane];
-                const unsigned peers = __match_any_sync(0xffffffffu, c);
-                my_c[s] = c;
-                my_rank[s] = __popc(peers & ((1u << lane) - 1u));
-                if (c != 0xFF && lane == __ffs(peers) - 1) table[ch * Kp + c] = (int16_t)__popc(peers);
-            }
-        }
-        __syncthreads();
-        if (threadIdx.x < Kp) {
-            int run = 0;
-            for (int ch = 0; ch < nch; ++ch) {
-                const int v = table[ch * Kp + threadIdx.x];
-                table[ch * Kp + threadIdx.x] = (int16_t)run;
-                run += v;
-            }
-            cnt_s[threadIdx.x] = run;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            int c0 = lane < Kp ? cnt_s[lane] : 0, c1 = lane + 32 < Kp ? cnt_s[lane + 32] : 0;
-            int s0 = c0, s1 = c1;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int x0 = __shfl_up_sync(0xffffffffu, s0, o), x1 = __shfl_up_sync(0xffffffffu, s1, o);
-                if (lane >= o) {
-                    s0 += x0;
-                    s1 += x1;
+            for (int s = 0; s < 2; ++s) {
+                const int ch = warp + s * kWarps;
+                my_c[s] = 0xFF;
+                my_rank[s] = 0;
+                if (ch < nch) {
+                    const int c = cs[ch * 32 + lane];
+                    const unsigned peers = __match_any_sync(0xffffffffu, c);
+                    my_c[s] = c;
+                    my_rank[s] = __popc(peers & ((1u << lane) - 1u));
+                    if (c != 0xFF && lane == __ffs(peers) - 1) table[ch * Kp + c] = (int16_t)__popc(peers);
                 }
             }
-            const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
-            if (lane < Kp) base_s[lane] = s0 - c0;
-            if (lane + 32 < Kp) base_s[lane + 32] = tot0 + s1 - c1;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-            const int ch = warp + s * kWarps;
-            if (ch < nch && my_c[s] != 0xFF) {
-                const int pos = base_s[my_c[s]] + table[ch * Kp + my_c[s]] + my_rank[s];
-                perm[pos] = (uint16_t)(ch * 32 + lane);
-                sc[pos] = (uint8_t)my_c[s];
+            __syncthreads();
+            if (threadIdx.x < Kp) {
+                int run = 0;
+                for (int ch = 0; ch < nch; ++ch) {
+                    const int v = table[ch * Kp + threadIdx.x];
+                    table[ch * Kp + threadIdx.x] = (int16_t)run;
+                    run += v;
+                }
+                cnt_s[threadIdx.x] = run;
             }
-        }
-        __syncthreads();
-        // (4) exact member sums: each warp walks a contiguous slice of the
-        // sorted tokens run by run (one cluster per run), lane holding
-        // coordinates 2*lane and 2*lane+1, four independent accumulators; a
-        // run's sum is added into the cluster's row with an (exact) fp64
-        // shared-memory atomic, so runs split between warps combine exactly.
-        for (int i = threadIdx.x; i < Kp * kD; i += kThreads) sums[i] = 0.0;
-        __syncthreads();
-        {
-            const int seg = (L + kWarps - 1) / kWarps;
-            const int p1 = min(L, (warp + 1) * seg);
-            int p = warp * seg;
-            while (p < p1) {
-                const int c = sc[p];
-                double s0[4] = {0.0, 0.0, 0.0, 0.0}, s1[4] = {0.0, 0.0, 0.0, 0.0};
-                for (;;) {
-                    const int q = p + lane;
-                    const unsigned same = __ballot_sync(0xffffffffu, q < p1 && sc[q] == c);
-                    const int n = __ffs(~same) ? __ffs(~same) - 1 : 32;
-                    const int rowl = (lane < n) ? perm[p + lane] : 0;
-                    for (int j = 0; j < n; j += 4) {
-                        uint32_t w[4];
+            __syncthreads();
+            if (warp == 0) {
+                int c0 = lane < Kp ? cnt_s[lane] : 0, c1 = lane + 32 < Kp ? cnt_s[lane + 32] : 0;
+                int s0 = c0, s1 = c1;
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int rr = __shfl_sync(0xffffffffu, rowl, (j + u) & 31);
-                            w[u] = (j + u < n) ? *reinterpret_cast<const uint32_t *>(qbytes + swz(rr, lane >> 2) + (lane & 3) * 4) : 0u;
-                        }
-                        bool slow = false;
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) slow |= (j + u < n) && bf16x2_has_zero_exp(w[u]);
-                        if (__any_sync(0xffffffffu, slow)) {
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                if (j + u < n) {
-                                    s0[u] += bf16_to_f64(w[u] & 0xffffu);
-                                    s1[u] += bf16_to_f64(w[u] >> 16);
-                                }
-                            }
-                        } else {
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                if (j + u < n) {
-                                    double d0, d1;
-                                    bf16x2_to_f64_normal(w[u], d0, d1);
-                                    s0[u] += d0;
-                                    s1[u] += d1;
-                                }
-                            }
-                        }
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int x0 = __shfl_up_sync(0xffffffffu, s0, o), x1 = __shfl_up_sync(0xffffffffu, s1, o);
+                    if (lane >= o) {
+                        s0 += x0;
+                        s1 += x1;
                     }
-                    p += n;
-                    if (n < 32) break;
                 }
-                atomicAdd(&sums[c * kD + 2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
-                atomicAdd(&sums[c * kD + 2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
+                const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
+                if (lane < Kp) base_s[lane] = s0 - c0;
+                if (lane + 32 < Kp) base_s[lane + 32] = tot0 + s1 - c1;
             }
+            __syncthreads();
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                const int ch = warp + s * kWarps;
+                if (ch < nch && my_c[s] != 0xFF) {
+                    const int pos = base_s[my_c[s]] + table[ch * Kp + my_c[s]] + my_rank[s];
+                    perm[pos] = (uint16_t)(ch * 32 + lane);
+                    sc[pos] = (uint8_t)my_c[s];
+                }
+            }
+            __syncthreads();
+            // (4) exact member sums: each warp walks a contiguous slice of the
+            // sorted tokens run by run (one cluster per run), lane holding
+            // coordinates 2*lane and 2*lane+1, four independent accumulators; a
+            // run's sum is added into the cluster's row with an (exact) fp64
+            // shared-memory atomic, so runs split between warps combine exactly.
+            for (int i = threadIdx.x; i < Kp * kD; i += kThreads) sums[i] = 0.0;
+            __syncthreads();
+            {
+                const int seg = (L + kWarps - 1) / kWarps;
+                const int p1 = min(L, (warp + 1) * seg);
+                int p = warp * seg;
+                while (p < p1) {
+                    const int c = sc[p];
+                    double s0[4] = {0.0, 0.0, 0.0, 0.0}, s1[4] = {0.0, 0.0, 0.0, 0.0};
+                    for (;;) {
+                        const int q = p + lane;
+                        const unsigned same = __ballot_sync(0xffffffffu, q < p1 && sc[q] == c);
+                        const int n = __ffs(~same) ? __ffs(~same) - 1 : 32;
+                        const int rowl = (lane < n) ? perm[p + lane] : 0;
+                        for (int j = 0; j < n; j += 4) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int rr = __shfl_sync(0xffffffffu, rowl, (j + u) & 31);
+                                w[u] = (j + u < n) ? *reinterpret_cast<const uint32_t *>(qbytes + swz(rr, lane >> 2) + (lane & 3) * 4) : 0u;
+                            }
+                            bool slow = false;
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) slow |= (j + u < n) && bf16x2_has_zero_exp(w[u]);
+                            if (__any_sync(0xffffffffu, slow)) {
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    if (j + u < n) {
+                                        s0[u] += bf16_to_f64(w[u] & 0xffffu);
+                                        s1[u] += bf16_to_f64(w[u] >> 16);
+                                    }
+                                }
+                            } else {
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    if (j + u < n) {
+                                        double d0, d1;
+                                        bf16x2_to_f64_normal(w[u], d0, d1);
+                                        s0[u] += d0;
+                                        s1[u] += d1;
+                                    }
+                                }
+                            }
+                        }
+                        p += n;
+                        if (n < 32) break;
+                    }
+                    atomicAdd(&sums[c * kD + 2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
+                    atomicAdd(&sums[c * kD + 2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
+                }
+            }
+            __syncthreads();
+            for (int i = threadIdx.x; i < Lp; i += kThreads) cprev[i] = cs[i];
+        } else {
+            // (3') later iterations: only tokens whose cluster changed move
+            // between the member sums (exact fp64 subtract / add) and counts.
+            for (int i = threadIdx.x; i < L; i += kThreads) {
+                const uint8_t cn = cs[i], co = cprev[i];
+                if (cn != co) list[atomicAdd(&misc[3], 1)] = (uint16_t)i;
+            }
+            __syncthreads();
+            const int n_mv = misc[3];
+            for (int e = warp; e < n_mv; e += kWarps) {
+                const int row = list[e];
+                const int co = cprev[row], cn = cs[row];
+                const uint32_t w = *reinterpret_cast<const uint32_t *>(qbytes + swz(row, lane >> 2) + (lane & 3) * 4);
+                const double d0 = bf16_to_f64(w & 0xffffu), d1 = bf16_to_f64(w >> 16);
+                atomicAdd(&sums[co * kD + 2 * lane], -d0);
+                atomicAdd(&sums[co * kD + 2 * lane + 1], -d1);
+                atomicAdd(&sums[cn * kD + 2 * lane], d0);
+                atomicAdd(&sums[cn * kD + 2 * lane + 1], d1);
+                if (lane == 0) {
+                    atomicSub(&cnt_s[co], 1);
+                    atomicAdd(&cnt_s[cn], 1);
+                }
+            }
+            __syncthreads();
+            for (int i = threadIdx.x; i < L; i += kThreads) cprev[i] = cs[i];
         }
-        __syncthreads();
         // (5) mu_k = fp32(sum_k / max(1, count_k)), one warp per centroid
         const bool last = it == P.iters - 1;
         for (int kk = warp; kk < Kp; kk += kWarps) {

@@ -31,15 +31,18 @@ namespace ca {
 constexpr float kFilterEps = 1.52587890625e-05f;  // 2^-16
 constexpr int kAssignThreads = 256;
 
-// mu^(0)_k = Q[floor(k L / K)], one block per head.
+// mu^(0)_k = Q[floor(k L / K)] (or Q[k * max(1, L / K)], the module's
+// stride, when init_stride), one block per head.
 template <typename T>
-__global__ void kmeans_init_kernel(const T *__restrict__ q, int L, int K, float *__restrict__ mu) {
+__global__ void kmeans_init_kernel(const T *__restrict__ q, int L, int K, float *__restrict__ mu,
+                                   int init_stride = 0) {
     const int64_t h = blockIdx.x;
     const T *qh = q + h * (int64_t)L * kD;
     float *muh = mu + h * (int64_t)K * kD;
     for (int idx = threadIdx.x; idx < K * kD; idx += blockDim.x) {
         const int k = idx / kD, j = idx % kD;
-        const int64_t row = ((int64_t)k * L) / K;
+        const int64_t step = L / K > 1 ? L / K : 1;
+        const int64_t row = init_stride ? (int64_t)k * step : ((int64_t)k * L) / K;
         muh[idx] = to_f32(qh[row * kD + j]);
     }
 }
@@ -193,10 +196,12 @@ __global__ void __launch_bounds__(kAssignThreads)
         if (cnt_s[k] > 0) atomicAdd(&counts[(int64_t)h * K + k], cnt_s[k]);
 }
 
-// mu_k = fp32(sum_k / max(1, count_k)); then clears sums / counts for the next
+// mu_k = fp32(sum_k / max(1, count_k)) (an empty cluster keeps its previous
+// centroid when empty_keep); then clears sums / counts for the next
 // iteration.  One block per head.
 __global__ void kmeans_update_kernel(int K, double *__restrict__ sums, int32_t *__restrict__ counts,
-                                     float *__restrict__ mu, float *__restrict__ cent_out) {
+                                     float *__restrict__ mu, float *__restrict__ cent_out,
+                                     int empty_keep = 0) {
     const int64_t h = blockIdx.x;
     double *s = sums + h * K * kD;
     int32_t *cn = counts + h * K;
@@ -204,7 +209,7 @@ __global__ void kmeans_update_kernel(int K, double *__restrict__ sums, int32_t *
     for (int idx = threadIdx.x; idx < K * kD; idx += blockDim.x) {
         const int c = cn[idx / kD];
         const double v = s[idx] / (double)(c > 1 ? c : 1);
-        const float f = __double2float_rn(v);
+        const float f = (empty_keep && c == 0) ? m[idx] : __double2float_rn(v);
         m[idx] = f;
         if (cent_out) cent_out[h * K * kD + idx] = f;
     }

@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(64) tiled_combine_kernel(int K, int n_chunks, 
 struct AssignLayout {
     int Kp, Tp;
     uint32_t q_off, sums_off, mu_off, hi_off, lo_off, mm_off, hash_off, cnt_off, base_off, dead_off,
-        c_off, sc_off, list_off, perm_off, table_off, misc_off, total;
+        c_off, sc_off, cprev_off, list_off, perm_off, table_off, misc_off, total;
     __host__ __device__ AssignLayout(int K) {
         Kp = kpad(K);
         Tp = kTileQ;
@@ -180,6 +180,8 @@ struct AssignLayout {
         o += (uint32_t)Tp;
         sc_off = o;
         o += (uint32_t)Tp;
+        cprev_off = o;
+        o += (uint32_t)Tp;
         list_off = o;
         o += (uint32_t)Tp * 2u;
         perm_off = o;
@@ -204,6 +206,7 @@ struct AssignParams {
     double *part_sum;    // [NH][Kp][n_tiles][64]
     int *part_cnt;       // [NH][Kp][n_tiles]
     int L, K, n_tiles;
+    int first;           // 1: first Lloyd iteration (full sums); 0: only changed tokens move
 };
 
 __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams P) {
@@ -227,11 +230,12 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
     uint8_t *dead = smem + lay.dead_off;
     uint8_t *cs = smem + lay.c_off;
     uint8_t *sc = smem + lay.sc_off;
+    uint8_t *cprev = smem + lay.cprev_off;
     uint16_t *list = reinterpret_cast<uint16_t *>(smem + lay.list_off);
     uint16_t *perm = reinterpret_cast<uint16_t *>(smem + lay.perm_off);
     int16_t *table = reinterpret_cast<int16_t *>(smem + lay.table_off);
     int *misc = reinterpret_cast<int *>(smem + lay.misc_off);
-    const bool smem_sums = Kp <= 32;
+    const bool smem_sums = Kp <= 32 && P.first;
     double *ssum = reinterpret_cast<double *>(smem + lay.sums_off);  // [Kp][64] when smem_sums
 
     load_rows(q_s, qh, 0, kTileQ, Lt);
@@ -243,10 +247,14 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
     for (int e = threadIdx.x; e < Kp * kD; e += kThreads) mu[(e / kD) * 65 + e % kD] = P.mu[cb * kD + e];
     // This tile's slots of the partial sums, cleared before the run sums add in.
     double *psum = P.part_sum;
-    for (int e = threadIdx.x; e < Kp * kD; e += kThreads) {
-        const int kk = e / kD, j = e % kD;
-        if (smem_sums) ssum[e] = 0.0;
-        else psum[((cb + kk) * P.n_tiles + tile) * kD + j] = 0.0;
+    if (P.first) {
+        for (int e = threadIdx.x; e < Kp * kD; e += kThreads) {
+            const int kk = e / kD, j = e % kD;
+            if (smem_sums) ssum[e] = 0.0;
+            else psum[((cb + kk) * P.n_tiles + tile) * kD + j] = 0.0;
+        }
+    } else {
+        for (int i = threadIdx.x; i < Lt; i += kThreads) cprev[i] = (uint8_t)P.assign[head * P.L + t0 + i];
     }
     for (int e = threadIdx.x; e < Kp * 8; e += kThreads) {
         const int kk = e >> 3, ch = e & 7;
@@ -260,7 +268,10 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
         hsh[kk] = P.hash[cb + kk];
     }
     for (int i = threadIdx.x; i < kTileQ; i += kThreads) cs[i] = i < Lt ? 0 : 0xFF;
-    if (threadIdx.x == 0) misc[0] = 0;
+    if (threadIdx.x == 0) {
+        misc[0] = 0;
+        misc[3] = 0;
+    }
     __syncthreads();
     // dead centroids: padding and bitwise copies of a lower-index centroid
     {
@@ -464,6 +475,31 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
     for (int i = threadIdx.x; i < Lt; i += kThreads) {
         P.assign[head * P.L + t0 + i] = cs[i];
         if (P.hist) P.hist[head * P.hist_stride + t0 + i] = cs[i];
+    }
+    if (!P.first) {
+        // Later iterations: only tokens whose cluster changed move between the
+        // tile's member sums (exact fp64 subtract / add) and counts.
+        for (int i = threadIdx.x; i < Lt; i += kThreads)
+            if (cs[i] != cprev[i]) list[atomicAdd(&misc[3], 1)] = (uint16_t)i;
+        __syncthreads();
+        const int n_mv = misc[3];
+        for (int e = warp; e < n_mv; e += kWarps) {
+            const int row = list[e];
+            const int co = cprev[row], cn = cs[row];
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(qbytes + swz(row, lane >> 2) + (lane & 3) * 4);
+            const double d0 = bf16_to_f64(w & 0xffffu), d1 = bf16_to_f64(w >> 16);
+            double *so = psum + ((cb + co) * P.n_tiles + tile) * kD;
+            double *sn = psum + ((cb + cn) * P.n_tiles + tile) * kD;
+            atomicAdd(&so[2 * lane], -d0);
+            atomicAdd(&so[2 * lane + 1], -d1);
+            atomicAdd(&sn[2 * lane], d0);
+            atomicAdd(&sn[2 * lane + 1], d1);
+            if (lane == 0) {
+                atomicSub(&P.part_cnt[(cb + co) * P.n_tiles + tile], 1);
+                atomicAdd(&P.part_cnt[(cb + cn) * P.n_tiles + tile], 1);
+            }
+        }
+        return;
     }
     // stable counting sort of the tile's tokens by cluster
     const int nch = kTileQ / 32;
