@@ -50,6 +50,7 @@ constexpr int kTile = 64;       // keys per centroid-attention tile
 constexpr int kSlots = 5;       // centroid-attention tiles in flight
 constexpr int kWinBlock = 128;  // queries per window block (8 warps x 16)
 constexpr int kMaxNT = (16 + 2 * kMaxR + 14) / 8;  // key n-tiles per window m-tile
+constexpr int kVcStride = 72;   // floats per V_cent row (conflict-free float2 gathers)
 constexpr float kEps = 1.220703125e-04f;           // 2^-13
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -87,7 +88,7 @@ struct Layout {
         lo_off = o;
         o += (uint32_t)Kp * 128u;
         vc_off = o;
-        o += (uint32_t)Kp * 64u * 4u;
+        o += (uint32_t)Kp * (uint32_t)kVcStride * 4u;
         mm_off = o;
         o += (uint32_t)Kp * 4u;
         hash_off = o;
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     const uint32_t hi_s = sbase + lay.hi_off, lo_s = sbase + lay.lo_off;
     unsigned char *qbytes = smem + lay.big_off;
     float *mu = reinterpret_cast<float *>(smem + lay.mu_off);                     // [Kp][65]
-    float *vc = reinterpret_cast<float *>(smem + lay.vc_off);                     // [Kp][64]
+    float *vc = reinterpret_cast<float *>(smem + lay.vc_off);  // [Kp][kVcStride], (1 - alpha) V_cent
     float *mm = reinterpret_cast<float *>(smem + lay.mm_off);                     // [Kp]
     uint32_t *hsh = reinterpret_cast<uint32_t *>(smem + lay.hash_off);
     int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
@@ -829,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                 den = fmaf(ml[(w * 16 + rr) * 2 + 1], f, den);
                 num = fmaf(part[(w * 16 + rr) * 64 + col], f, num);
             }
-            vc[row * kD + col] = num / den;
+            vc[row * kVcStride + col] = (1.f - P.alpha) * (num / den);
         }
         __syncthreads();
     }
@@ -853,6 +854,26 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     issue_block(0);
     issue_block(1);
     __nv_bfloat16 *oh = P.out + head * (int64_t)L * kD;
+    // Band mask of a warp's 16 x (8 kMaxNT) score tile as bits 4n+e: key
+    // kst + 8n + 2t + (e&1) against query i0 + g + 8(e>>1).  A warp whose
+    // whole band lies inside [0, L) sees the same pattern everywhere.
+    auto band_bits = [&](int kst, int i0, bool check_L) {
+        uint32_t m = 0u;
+#pragma unroll
+        for (int n = 0; n < kMaxNT; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = i0 + g + 8 * (e >> 1);
+                const int jk = kst + n * 8 + 2 * t + (e & 1);
+                const bool ok = jk >= i - r && jk <= i + r && (!check_L || jk < L);
+                m |= (ok ? 1u : 0u) << (4 * n + e);
+            }
+        return m;
+    };
+    const uint32_t inner_bits = band_bits(-((r + 7) & ~7), 0, false);
+    // Per-warp output staging (8 rows x 128 bytes, swizzled) in the centroid
+    // region, which is dead once V_cent is formed.
+    const uint32_t ost = sbase + lay.mu_off + warp * 1024;
     // Q fragments of this warp's 16 rows of a block, read from global memory
     // (L2); fetched one block ahead.
     uint32_t a[4][4];
@@ -882,6 +903,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
             const int kend = min(L - 1, i0 + 15 + r);
             const int nt = (kend - kst) / 8 + 1;
             const int lr0 = kst - ks0;
+            const uint32_t mbits = (i0 >= r && i0 + 15 + r <= L - 1) ? inner_bits : band_bits(kst, i0, true);
             float sacc[kMaxNT][4];
 #pragma unroll
             for (int n = 0; n < kMaxNT; ++n) {
@@ -902,21 +924,19 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
             for (int n = 0; n < kMaxNT; ++n) {
                 if (n < nt) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = i0 + g + 8 * (e >> 1);
-                        const int jk = kst + n * 8 + 2 * t + (e & 1);
-                        const bool ok = jk >= i - r && jk <= i + r && jk < L;
-                        if (!ok) sacc[n][e] = -INFINITY;
-                    }
+                    for (int e = 0; e < 4; ++e)
+                        if (!((mbits >> (4 * n + e)) & 1u)) sacc[n][e] = -INFINITY;
                     mx[0] = fmaxf(mx[0], fmaxf(sacc[n][0], sacc[n][1]));
                     mx[1] = fmaxf(mx[1], fmaxf(sacc[n][2], sacc[n][3]));
                 }
             }
-            float sum[2] = {0.f, 0.f};
+            float sum[2] = {0.f, 0.f}, mxc[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
                 mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+                // rows past L have no key: every score is -inf and p = 0
+                mxc[h] = (mx[h] == -INFINITY) ? 0.f : mx[h] * csc;
             }
             uint32_t pa[kMaxNT][2];
 #pragma unroll
@@ -925,10 +945,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                 if (n < nt) {
                     float p[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float mh = mx[e >> 1];
-                        p[e] = (mh == -INFINITY) ? 0.f : ex2((sacc[n][e] - mh) * csc);
-                    }
+                    for (int e = 0; e < 4; ++e) p[e] = ex2(fmaf(sacc[n][e], csc, -mxc[e >> 1]));
                     sum[0] += p[0] + p[1];
                     sum[1] += p[2] + p[3];
                     pa[n][0] = pack_bf16(p[0], p[1]);
@@ -967,24 +984,37 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                     }
                 }
             }
-            // gather + blend, stored straight to global memory
-            const float inv0 = sum[0] > 0.f ? 1.f / sum[0] : 0.f, inv1 = sum[1] > 0.f ? 1.f / sum[1] : 0.f;
-            const int ia = i0 + g, ib = i0 + g + 8;
-            const int ca = ia < L ? cs[ia] : 0, cb = ib < L ? cs[ib] : 0;
-            const float al = P.alpha, be = 1.f - P.alpha;
+            // gather + blend: O = (1 - alpha) V_cent[c_i] + alpha o_i, staged
+            // eight rows at a time through shared memory (stmatrix) and
+            // stored as whole 128-byte rows
+            const float f0 = sum[0] > 0.f ? P.alpha / sum[0] : 0.f, f1 = sum[1] > 0.f ? P.alpha / sum[1] : 0.f;
 #pragma unroll
-            for (int d = 0; d < 8; ++d) {
-                const int col = 8 * d + 2 * t;
-                if (ia < L) {
-                    const float y0 = be * vc[ca * kD + col] + al * (oacc[d][0] * inv0);
-                    const float y1 = be * vc[ca * kD + col + 1] + al * (oacc[d][1] * inv0);
-                    *reinterpret_cast<uint32_t *>(oh + (int64_t)ia * kD + col) = pack_bf16(y0, y1);
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i = i0 + g + 8 * hh;
+                const float f = hh ? f1 : f0;
+                const float *vrow = vc + (i < L ? cs[i] : 0) * kVcStride + 2 * t;
+                uint32_t wv[8];
+#pragma unroll
+                for (int d = 0; d < 8; ++d) {
+                    const float2 c2 = *reinterpret_cast<const float2 *>(vrow + 8 * d);
+                    wv[d] = pack_bf16(fmaf(f, oacc[d][2 * hh], c2.x), fmaf(f, oacc[d][2 * hh + 1], c2.y));
                 }
-                if (ib < L) {
-                    const float y2 = be * vc[cb * kD + col] + al * (oacc[d][2] * inv1);
-                    const float y3 = be * vc[cb * kD + col + 1] + al * (oacc[d][3] * inv1);
-                    *reinterpret_cast<uint32_t *>(oh + (int64_t)ib * kD + col) = pack_bf16(y2, y3);
+                const int sr = lane & 7, sd = lane >> 3;
+                stmatrix_x4(ost + sr * 128 + ((sd ^ sr) << 4), wv[0], wv[1], wv[2], wv[3]);
+                stmatrix_x4(ost + sr * 128 + (((sd + 4) ^ sr) << 4), wv[4], wv[5], wv[6], wv[7]);
+                __syncwarp();
+#pragma unroll
+                for (int it2 = 0; it2 < 2; ++it2) {
+                    const int rr = it2 * 4 + (lane >> 3), ch = lane & 7;
+                    const int row = i0 + 8 * hh + rr;
+                    uint4 val;
+                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                                 : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                                 : "r"(ost + rr * 128 + ((ch ^ rr) << 4))
+                                 : "memory");
+                    if (row < L) *reinterpret_cast<uint4 *>(oh + (int64_t)row * kD + ch * 8) = val;
                 }
+                __syncwarp();
             }
         }
         fetch_q(b + 1);

@@ -1,5 +1,6 @@
 // Warp-level tensor-core and async-copy primitives (inline PTX) used by the
-// fused kernels: ldmatrix, bf16 mma.sync with fp32 accumulation, cp.async.
+// fused kernels: ldmatrix / stmatrix, bf16 mma.sync with fp32 accumulation,
+// cp.async.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -33,6 +34,15 @@ __device__ __forceinline__ void ldmatrix_x2_trans(uint32_t (&r)[2], uint32_t add
     asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n"
                  : "=r"(r[0]), "=r"(r[1])
                  : "r"(addr));
+}
+
+// Stores four 8x8 b16 matrices held in the mma accumulator layout (lane
+// holds row lane/4, columns 2*(lane%4) and +1 of each); lane i gives the
+// address of row i%8 of matrix i/8.
+__device__ __forceinline__ void stmatrix_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(r0), "r"(r1),
+                 "r"(r2), "r"(r3)
+                 : "memory");
 }
 
 // D = A(16x16, bf16, row) * B(16x8, bf16, col) + D, fp32 accumulation.
