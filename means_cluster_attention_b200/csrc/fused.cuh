@@ -26,13 +26,13 @@
 // copies of a lower-index centroid can never win (their distances are equal
 // and the lower index takes the tie) and are excluded up front.
 //
-// Member sums: in the first iteration tokens are ordered by cluster with a
-// stable counting sort and each warp walks a contiguous slice of the sorted
-// tokens, turning bf16 values into doubles with integer operations and
-// adding in fp64; later iterations only subtract / add the tokens whose
-// cluster changed.  Those sums are exact for any input
-// whose non-zero magnitudes lie within 2^-27 .. 16, so the centroid
-// mu_k = fp32(sum / max(1, count)) does not depend on the order of the adds.
+// Member sums: tokens are grouped by cluster with a counting sort and each
+// warp walks a contiguous slice of the sorted tokens, turning bf16 values
+// into doubles with integer operations and adding in fp64; a later iteration
+// in which few tokens change cluster only subtracts / adds those.  The sums
+// are exact for any input whose non-zero magnitudes lie within 2^-27 .. 16,
+// so the centroid mu_k = fp32(sum / max(1, count)) does not depend on the
+// order of the adds.
 #pragma once
 
 #include "common.cuh"
@@ -60,7 +60,7 @@ __host__ __device__ inline uint32_t umax(uint32_t a, uint32_t b) { return a > b 
 struct Layout {
     int Lp, Kp, r, nT, win_rows;
     uint32_t big_off, sums_off, mu_off, hi_off, lo_off, vc_off, mm_off, hash_off, dead_off, c_off,
-        list_off, perm_off, sc_off, cprev_off, table_off, cnt_off, base_off, misc_off, ml_off, win_stage,
+        list_off, perm_off, sc_off, cprev_off, cnt_off, misc_off, ml_off, win_stage,
         total;
 
     __host__ __device__ Layout(int L, int K, int r_) {
@@ -95,8 +95,6 @@ struct Layout {
         o += (uint32_t)Kp * 4u;
         cnt_off = o;
         o += (uint32_t)Kp * 4u;
-        base_off = o;
-        o += (uint32_t)Kp * 4u;
         dead_off = o;
         o += up((uint32_t)Kp, 16);
         c_off = o;
@@ -109,8 +107,6 @@ struct Layout {
         o += up((uint32_t)Lp * 2u, 16);
         perm_off = o;
         o += up((uint32_t)Lp * 2u, 16);
-        table_off = o;
-        o += up((uint32_t)(Lp / 32) * (uint32_t)Kp * 2u, 16);
         misc_off = o;
         o += 64;
         ml_off = o;
@@ -229,23 +225,21 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     float *mm = reinterpret_cast<float *>(smem + lay.mm_off);                     // [Kp]
     uint32_t *hsh = reinterpret_cast<uint32_t *>(smem + lay.hash_off);
     int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
-    int *base_s = reinterpret_cast<int *>(smem + lay.base_off);
     double *sums = reinterpret_cast<double *>(smem + lay.big_off + lay.sums_off);  // [Kp][64]
     uint8_t *dead = smem + lay.dead_off;
     uint8_t *cs = smem + lay.c_off;                                              // [Lp]
-    uint8_t *sc = smem + lay.sc_off;                                             // [Lp] sorted cluster ids
-    uint8_t *cprev = smem + lay.cprev_off;                                       // [Lp] previous assignment
+    uint8_t *sc = smem + lay.sc_off;        // [Lp] cluster ids in sorted order
+    uint8_t *cprev = smem + lay.cprev_off;  // [Lp] previous iteration's assignment
     uint16_t *list = reinterpret_cast<uint16_t *>(smem + lay.list_off);
-    uint16_t *perm = reinterpret_cast<uint16_t *>(smem + lay.perm_off);
-    int16_t *table = reinterpret_cast<int16_t *>(smem + lay.table_off);           // [Lp/32][Kp]
-    int *misc = reinterpret_cast<int *>(smem + lay.misc_off);  // 0 refine count, 1 mm_max, 2 mun_max
+    uint16_t *perm = reinterpret_cast<uint16_t *>(smem + lay.perm_off);  // [Lp] tokens in sorted order
+    int *misc = reinterpret_cast<int *>(smem + lay.misc_off);  // 0 refine count, 1 max |mu|^2 bits, 3 movers
     float *ml = reinterpret_cast<float *>(smem + lay.ml_off);
 
     // ---- prologue: Q ------------------------------------------------------
     load_rows(big_s, qh, 0, Lp, L);
     cp_async_commit();
     for (int i = threadIdx.x; i < Lp; i += kThreads) cs[i] = i < L ? 0 : 0xFF;
-    if (threadIdx.x == 0) misc[0] = 0;
+    if (threadIdx.x == 0) misc[0] = misc[1] = 0;
     cp_async_wait<0>();
     __syncthreads();
 
@@ -301,45 +295,33 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
             hv32 += __shfl_xor_sync(0xffffffffu, hv32, o);
         }
         if (lane == 0) {
-            mm[kk] = sq;
+            // padding rows can never win; live rows feed max |mu|^2 (a
+            // duplicate has its original's norm, so it cannot raise the max)
+            mm[kk] = kk < K ? sq : INFINITY;
             hsh[kk] = hv32;
+            dead[kk] = kk < K ? 0 : 1;
+            if (kk < K) atomicMax(&misc[1], __float_as_int(sq));
         }
     };
 
-    // After every centroid row is final: mark padding and bitwise duplicates
-    // of a lower-index centroid dead (+inf), and take max |mu|^2, max |mu|
-    // over the live centroids.
-    auto finalize_set = [&]() {
+    // After every centroid row is final: mark bitwise duplicates of a
+    // lower-index centroid dead (|mu|^2 = +inf), one thread per pair; write
+    // the iteration's assignments to hrow when given.
+    auto finalize_set = [&](int32_t *hrow) {
         __syncthreads();
-        const int kk = threadIdx.x;
-        if (kk < Kp) {
-            bool dd = kk >= K;
-            for (int a = 0; a < kk && !dd; ++a) {
-                if (hsh[a] != hsh[kk]) continue;
+        if (threadIdx.x == 0) misc[0] = misc[3] = 0;
+        if (hrow)
+            for (int i = threadIdx.x; i < L; i += kThreads) hrow[i] = cs[i];
+        for (int pr = threadIdx.x; pr < K * K; pr += kThreads) {
+            const int kk = pr / K, a = pr - kk * K;
+            if (a < kk && hsh[a] == hsh[kk]) {
                 bool same = true;
                 for (int j = 0; j < kD && same; ++j)
                     same = __float_as_uint(mu[a * 65 + j]) == __float_as_uint(mu[kk * 65 + j]);
-                dd = same;
-            }
-            dead[kk] = dd ? 1 : 0;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            float mx = 0.f;
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                const int k2 = lane + 32 * s;
-                if (k2 < Kp) {
-                    if (dead[k2]) mm[k2] = INFINITY;
-                    else mx = fmaxf(mx, mm[k2]);
+                if (same) {
+                    dead[kk] = 1;
+                    mm[kk] = INFINITY;
                 }
-            }
-            mx = warp_max(mx);
-            if (lane == 0) {
-                misc[1] = __float_as_int(mx);
-                misc[2] = __float_as_int(sqrtf(mx));
-                misc[0] = 0;
-                misc[3] = 0;
             }
         }
         __syncthreads();
@@ -356,12 +338,16 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         }
         finalize_row(kk, x0, x1);
     }
-    finalize_set();
+    finalize_set(nullptr);
 
     const int nch = Lp / 32;
     // ---- Lloyd iterations -----------------------------------------------------
     for (int it = 0; it < P.iters; ++it) {
-        const float mm_max = __int_as_float(misc[1]), mun_max = __int_as_float(misc[2]);
+        const float mm_max = __int_as_float(misc[1]), mun_max = sqrtf(mm_max);
+        if (it == 0) {
+            for (int i = threadIdx.x; i < Kp * kD; i += kThreads) sums[i] = 0.0;
+            if (threadIdx.x < Kp) cnt_s[threadIdx.x] = 0;
+        }
         // (1) assignment: tensor-core distances + certified argmin, two m-tiles at a time
 #pragma unroll
         for (int jp = 0; jp < kMtPerWarp; jp += 2) {
@@ -437,6 +423,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         __syncthreads();
         // (2) exact re-measure of ambiguous tokens, one warp per token
         const int n_ref = misc[0];
+        if (threadIdx.x == 0) misc[1] = 0;
         for (int e = warp; e < n_ref; e += kWarps) {
             const int row = list[e];
             double qq = 0.0, qm0 = 0.0, qm1 = 0.0, m20 = 0.0, m21 = 0.0;
@@ -457,13 +444,16 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                     mj0[u] = v0 ? (double)mu[k0 * 65 + jb + u] : 0.0;
                     mj1[u] = v1 ? (double)mu[k1 * 65 + jb + u] : 0.0;
                 }
+                // Every product (bf16 x bf16, bf16 x fp32, fp32 x fp32) is
+                // exact in fp64, so one fused multiply-add rounds exactly as
+                // a separately rounded product followed by a rounded sum.
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    qq = __dadd_rn(qq, __dmul_rn(qj[u], qj[u]));
-                    qm0 = __dadd_rn(qm0, __dmul_rn(qj[u], mj0[u]));
-                    m20 = __dadd_rn(m20, __dmul_rn(mj0[u], mj0[u]));
-                    qm1 = __dadd_rn(qm1, __dmul_rn(qj[u], mj1[u]));
-                    m21 = __dadd_rn(m21, __dmul_rn(mj1[u], mj1[u]));
+                    qq = __fma_rn(qj[u], qj[u], qq);
+                    qm0 = __fma_rn(qj[u], mj0[u], qm0);
+                    m20 = __fma_rn(mj0[u], mj0[u], m20);
+                    qm1 = __fma_rn(qj[u], mj1[u], qm1);
+                    m21 = __fma_rn(mj1[u], mj1[u], m21);
                 }
             }
             double bd = INFINITY;
@@ -488,141 +478,31 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                     bk = ok;
                 }
             }
-            if (lane == 0) {
-                if (bk >= K) {
-                    record_error(5, 2);
-                    bk = 0;
-                }
-                cs[row] = (uint8_t)bk;
+            if (bk >= K) {
+                if (lane == 0) record_error(5, 2);
+                bk = 0;
             }
+            if (lane == 0) cs[row] = (uint8_t)bk;
         }
         __syncthreads();
-        if (P.hist) {
-            int32_t *hrow = P.hist + (head * P.iters + it) * (int64_t)L;
-            for (int i = threadIdx.x; i < L; i += kThreads) hrow[i] = cs[i];
+        // (3) member sums.  Later iterations first list the tokens whose
+        // cluster changed; when they are few, only they move between the
+        // sums (exact fp64 subtract / add) and the counts.
+        int n_mv = L;
+        if (it > 0) {
+            for (int ch = warp; ch < nch; ch += kWarps) {
+                const int i = ch * 32 + lane;
+                const bool mv = i < L && cs[i] != cprev[i];
+                const unsigned bal = __ballot_sync(0xffffffffu, mv);
+                int base = 0;
+                if (lane == 0 && bal) base = atomicAdd(&misc[3], __popc(bal));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                if (mv) list[base + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)i;
+            }
+            __syncthreads();
+            n_mv = misc[3];
         }
-        if (it == 0) {
-            // (3) stable counting sort of the tokens by cluster
-            for (int i = threadIdx.x; i < nch * Kp; i += kThreads) table[i] = 0;
-            __syncthreads();
-            int my_c[2], my_rank[2];
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                const int ch = warp + s * kWarps;
-                my_c[s] = 0xFF;
-                my_rank[s] = 0;
-                if (ch < nch) {
-                    const int c = cs[ch * 32 + lane];
-                    const unsigned peers = __match_any_sync(0xffffffffu, c);
-                    my_c[s] = c;
-                    my_rank[s] = __popc(peers & ((1u << lane) - 1u));
-                    if (c != 0xFF && lane == __ffs(peers) - 1) table[ch * Kp + c] = (int16_t)__popc(peers);
-                }
-            }
-            __syncthreads();
-            if (threadIdx.x < Kp) {
-                int run = 0;
-                for (int ch = 0; ch < nch; ++ch) {
-                    const int v = table[ch * Kp + threadIdx.x];
-                    table[ch * Kp + threadIdx.x] = (int16_t)run;
-                    run += v;
-                }
-                cnt_s[threadIdx.x] = run;
-            }
-            __syncthreads();
-            if (warp == 0) {
-                int c0 = lane < Kp ? cnt_s[lane] : 0, c1 = lane + 32 < Kp ? cnt_s[lane + 32] : 0;
-                int s0 = c0, s1 = c1;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int x0 = __shfl_up_sync(0xffffffffu, s0, o), x1 = __shfl_up_sync(0xffffffffu, s1, o);
-                    if (lane >= o) {
-                        s0 += x0;
-                        s1 += x1;
-                    }
-                }
-                const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
-                if (lane < Kp) base_s[lane] = s0 - c0;
-                if (lane + 32 < Kp) base_s[lane + 32] = tot0 + s1 - c1;
-            }
-            __syncthreads();
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                const int ch = warp + s * kWarps;
-                if (ch < nch && my_c[s] != 0xFF) {
-                    const int pos = base_s[my_c[s]] + table[ch * Kp + my_c[s]] + my_rank[s];
-                    perm[pos] = (uint16_t)(ch * 32 + lane);
-                    sc[pos] = (uint8_t)my_c[s];
-                }
-            }
-            __syncthreads();
-            // (4) exact member sums: each warp walks a contiguous slice of the
-            // sorted tokens run by run (one cluster per run), lane holding
-            // coordinates 2*lane and 2*lane+1, four independent accumulators; a
-            // run's sum is added into the cluster's row with an (exact) fp64
-            // shared-memory atomic, so runs split between warps combine exactly.
-            for (int i = threadIdx.x; i < Kp * kD; i += kThreads) sums[i] = 0.0;
-            __syncthreads();
-            {
-                const int seg = (L + kWarps - 1) / kWarps;
-                const int p1 = min(L, (warp + 1) * seg);
-                int p = warp * seg;
-                while (p < p1) {
-                    const int c = sc[p];
-                    double s0[4] = {0.0, 0.0, 0.0, 0.0}, s1[4] = {0.0, 0.0, 0.0, 0.0};
-                    for (;;) {
-                        const int q = p + lane;
-                        const unsigned same = __ballot_sync(0xffffffffu, q < p1 && sc[q] == c);
-                        const int n = __ffs(~same) ? __ffs(~same) - 1 : 32;
-                        const int rowl = (lane < n) ? perm[p + lane] : 0;
-                        for (int j = 0; j < n; j += 4) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const int rr = __shfl_sync(0xffffffffu, rowl, (j + u) & 31);
-                                w[u] = (j + u < n) ? *reinterpret_cast<const uint32_t *>(qbytes + swz(rr, lane >> 2) + (lane & 3) * 4) : 0u;
-                            }
-                            bool slow = false;
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) slow |= (j + u < n) && bf16x2_has_zero_exp(w[u]);
-                            if (__any_sync(0xffffffffu, slow)) {
-#pragma unroll
-                                for (int u = 0; u < 4; ++u) {
-                                    if (j + u < n) {
-                                        s0[u] += bf16_to_f64(w[u] & 0xffffu);
-                                        s1[u] += bf16_to_f64(w[u] >> 16);
-                                    }
-                                }
-                            } else {
-#pragma unroll
-                                for (int u = 0; u < 4; ++u) {
-                                    if (j + u < n) {
-                                        double d0, d1;
-                                        bf16x2_to_f64_normal(w[u], d0, d1);
-                                        s0[u] += d0;
-                                        s1[u] += d1;
-                                    }
-                                }
-                            }
-                        }
-                        p += n;
-                        if (n < 32) break;
-                    }
-                    atomicAdd(&sums[c * kD + 2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
-                    atomicAdd(&sums[c * kD + 2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
-                }
-            }
-            __syncthreads();
-            for (int i = threadIdx.x; i < Lp; i += kThreads) cprev[i] = cs[i];
-        } else {
-            // (3') later iterations: only tokens whose cluster changed move
-            // between the member sums (exact fp64 subtract / add) and counts.
-            for (int i = threadIdx.x; i < L; i += kThreads) {
-                const uint8_t cn = cs[i], co = cprev[i];
-                if (cn != co) list[atomicAdd(&misc[3], 1)] = (uint16_t)i;
-            }
-            __syncthreads();
-            const int n_mv = misc[3];
+        if (n_mv <= (L >> 2)) {
             for (int e = warp; e < n_mv; e += kWarps) {
                 const int row = list[e];
                 const int co = cprev[row], cn = cs[row];
@@ -637,9 +517,112 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                     atomicAdd(&cnt_s[cn], 1);
                 }
             }
+        } else {
+            if (it > 0) {
+                for (int i = threadIdx.x; i < Kp * kD; i += kThreads) sums[i] = 0.0;
+                if (threadIdx.x < Kp) cnt_s[threadIdx.x] = 0;
+                __syncthreads();
+            }
+            // Counting sort by cluster (order inside a cluster is free: the
+            // sums are exact).  Peers of one cluster in a 32-token chunk take
+            // their offsets with one atomic on the count; every warp then
+            // scans the counts itself.
+            int my_c[2], my_off[2];
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) {
+                const int ch = warp + s2 * kWarps;
+                my_c[s2] = 0xFF;
+                my_off[s2] = 0;
+                if (ch < nch) {
+                    const int c = cs[ch * 32 + lane];
+                    const unsigned peers = __match_any_sync(0xffffffffu, c);
+                    const int leader = __ffs(peers) - 1;
+                    int off = 0;
+                    if (c != 0xFF && lane == leader) off = atomicAdd(&cnt_s[c], __popc(peers));
+                    off = __shfl_sync(0xffffffffu, off, leader);
+                    my_c[s2] = c;
+                    my_off[s2] = off + __popc(peers & ((1u << lane) - 1u));
+                }
+            }
             __syncthreads();
-            for (int i = threadIdx.x; i < L; i += kThreads) cprev[i] = cs[i];
+            {
+                const int c0 = lane < Kp ? cnt_s[lane] : 0, c1 = lane + 32 < Kp ? cnt_s[lane + 32] : 0;
+                int s0 = c0, s1 = c1;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int x0 = __shfl_up_sync(0xffffffffu, s0, o), x1 = __shfl_up_sync(0xffffffffu, s1, o);
+                    if (lane >= o) {
+                        s0 += x0;
+                        s1 += x1;
+                    }
+                }
+                const int b0 = s0 - c0, b1 = __shfl_sync(0xffffffffu, s0, 31) + s1 - c1;
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2) {
+                    const int c = my_c[s2];
+                    const int x0 = __shfl_sync(0xffffffffu, b0, c & 31), x1 = __shfl_sync(0xffffffffu, b1, c & 31);
+                    if (c != 0xFF) {
+                        const int pos = (c < 32 ? x0 : x1) + my_off[s2];
+                        perm[pos] = (uint16_t)((warp + s2 * kWarps) * 32 + lane);
+                        sc[pos] = (uint8_t)c;
+                    }
+                }
+            }
+            __syncthreads();
+            // Each warp walks a contiguous slice of the sorted tokens run by
+            // run (one cluster per run), lane holding coordinates 2*lane and
+            // 2*lane+1, four independent accumulators; a run's sum is added
+            // into the cluster's row with an fp64 shared-memory atomic.
+            const int seg = (L + kWarps - 1) / kWarps;
+            const int p1 = min(L, (warp + 1) * seg);
+            int p = warp * seg;
+            while (p < p1) {
+                const int c = sc[p];
+                double s0[4] = {0.0, 0.0, 0.0, 0.0}, s1[4] = {0.0, 0.0, 0.0, 0.0};
+                for (;;) {
+                    const int q = p + lane;
+                    const unsigned same = __ballot_sync(0xffffffffu, q < p1 && sc[q] == c);
+                    const int n = __ffs(~same) ? __ffs(~same) - 1 : 32;
+                    const int rowl = (lane < n) ? perm[p + lane] : 0;
+                    for (int j = 0; j < n; j += 4) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int rr = __shfl_sync(0xffffffffu, rowl, (j + u) & 31);
+                            w[u] = (j + u < n) ? *reinterpret_cast<const uint32_t *>(qbytes + swz(rr, lane >> 2) + (lane & 3) * 4) : 0u;
+                        }
+                        bool slow = false;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) slow |= (j + u < n) && bf16x2_has_zero_exp(w[u]);
+                        if (__any_sync(0xffffffffu, slow)) {
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                if (j + u < n) {
+                                    s0[u] += bf16_to_f64(w[u] & 0xffffu);
+                                    s1[u] += bf16_to_f64(w[u] >> 16);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                if (j + u < n) {
+                                    double d0, d1;
+                                    bf16x2_to_f64_normal(w[u], d0, d1);
+                                    s0[u] += d0;
+                                    s1[u] += d1;
+                                }
+                            }
+                        }
+                    }
+                    p += n;
+                    if (n < 32) break;
+                }
+                atomicAdd(&sums[c * kD + 2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
+                atomicAdd(&sums[c * kD + 2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
+            }
         }
+        __syncthreads();
+        for (int i = threadIdx.x; i < Lp; i += kThreads) cprev[i] = cs[i];
         // (5) mu_k = fp32(sum_k / max(1, count_k)), one warp per centroid
         const bool last = it == P.iters - 1;
         for (int kk = warp; kk < Kp; kk += kWarps) {
@@ -653,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                 dst[lane] = make_float2(x0, x1);
             }
         }
-        finalize_set();
+        finalize_set(P.hist ? P.hist + (head * P.iters + it) * (int64_t)L : nullptr);
     }
     if (P.iters == 0 && P.cent) {
         for (int e = threadIdx.x; e < K * kD; e += kThreads) P.cent[head * K * kD + e] = mu[(e / kD) * 65 + e % kD];
