@@ -81,6 +81,37 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// Marks every centroid kk < K that is a bitwise copy of a lower-index
+// centroid dead (dead[kk] = 1, mm[kk] = +inf): such a centroid can never win
+// an argmin whose ties go to the lowest index.  One warp per centroid: the
+// lanes compare the hashes of 32 lower indices at once, then each hash match,
+// lowest first, row against row (two coordinates per lane) until one is equal.
+// mu rows are mu_ld floats apart; the caller initialises dead and mm.
+__device__ inline void mark_copies(int K, const uint32_t *hsh, const float *mu, int mu_ld, uint8_t *dead, float *mm,
+                                   int warp, int nwarps, int lane) {
+    for (int kk = warp; kk < K; kk += nwarps) {
+        const uint32_t hk = hsh[kk];
+        const uint32_t x0 = __float_as_uint(mu[kk * mu_ld + 2 * lane]);
+        const uint32_t x1 = __float_as_uint(mu[kk * mu_ld + 2 * lane + 1]);
+        bool found = false;
+        for (int a0 = 0; a0 < kk && !found; a0 += 32) {
+            const int a = a0 + lane;
+            unsigned cand = __ballot_sync(0xffffffffu, a < kk && hsh[a] == hk);
+            while (cand && !found) {
+                const int b = a0 + __ffs(cand) - 1;
+                cand &= cand - 1u;
+                const bool eq = __float_as_uint(mu[b * mu_ld + 2 * lane]) == x0 &&
+                                __float_as_uint(mu[b * mu_ld + 2 * lane + 1]) == x1;
+                found = __all_sync(0xffffffffu, eq);
+            }
+        }
+        if (found && lane == 0) {
+            dead[kk] = 1;
+            mm[kk] = INFINITY;
+        }
+    }
+}
+
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));

@@ -305,25 +305,14 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     };
 
     // After every centroid row is final: mark bitwise duplicates of a
-    // lower-index centroid dead (|mu|^2 = +inf), one thread per pair; write
-    // the iteration's assignments to hrow when given.
+    // lower-index centroid dead (|mu|^2 = +inf); write the iteration's
+    // assignments to hrow when given.
     auto finalize_set = [&](int32_t *hrow) {
         __syncthreads();
         if (threadIdx.x == 0) misc[0] = misc[3] = 0;
         if (hrow)
             for (int i = threadIdx.x; i < L; i += kThreads) hrow[i] = cs[i];
-        for (int pr = threadIdx.x; pr < K * K; pr += kThreads) {
-            const int kk = pr / K, a = pr - kk * K;
-            if (a < kk && hsh[a] == hsh[kk]) {
-                bool same = true;
-                for (int j = 0; j < kD && same; ++j)
-                    same = __float_as_uint(mu[a * 65 + j]) == __float_as_uint(mu[kk * 65 + j]);
-                if (same) {
-                    dead[kk] = 1;
-                    mm[kk] = INFINITY;
-                }
-            }
-        }
+        mark_copies(K, hsh, mu, 65, dead, mm, warp, kWarps, lane);
         __syncthreads();
     };
 

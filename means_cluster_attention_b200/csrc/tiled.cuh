@@ -148,8 +148,8 @@ __global__ void __launch_bounds__(64) tiled_combine_kernel(int K, int n_chunks, 
 // One Lloyd assignment for a tile of up to 512 queries.
 struct AssignLayout {
     int Kp, Tp;
-    uint32_t q_off, sums_off, mu_off, hi_off, lo_off, mm_off, hash_off, cnt_off, base_off, dead_off,
-        c_off, sc_off, cprev_off, list_off, perm_off, table_off, misc_off, total;
+    uint32_t q_off, sums_off, mu_off, hi_off, lo_off, mm_off, hash_off, cnt_off, dead_off,
+        c_off, sc_off, cprev_off, list_off, perm_off, misc_off, total;
     __host__ __device__ AssignLayout(int K) {
         Kp = kpad(K);
         Tp = kTileQ;
@@ -172,8 +172,6 @@ struct AssignLayout {
         o += (uint32_t)Kp * 4u;
         cnt_off = o;
         o += (uint32_t)Kp * 4u;
-        base_off = o;
-        o += (uint32_t)Kp * 4u;
         dead_off = o;
         o += up((uint32_t)Kp, 16);
         c_off = o;
@@ -186,8 +184,6 @@ struct AssignLayout {
         o += (uint32_t)Tp * 2u;
         perm_off = o;
         o += (uint32_t)Tp * 2u;
-        table_off = o;
-        o += up((uint32_t)(Tp / 32) * (uint32_t)Kp * 2u, 16);
         misc_off = o;
         o += 64;
         total = up(o, 128);
@@ -226,14 +222,12 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
     float *mm = reinterpret_cast<float *>(smem + lay.mm_off);
     uint32_t *hsh = reinterpret_cast<uint32_t *>(smem + lay.hash_off);
     int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
-    int *base_s = reinterpret_cast<int *>(smem + lay.base_off);
     uint8_t *dead = smem + lay.dead_off;
     uint8_t *cs = smem + lay.c_off;
     uint8_t *sc = smem + lay.sc_off;
     uint8_t *cprev = smem + lay.cprev_off;
     uint16_t *list = reinterpret_cast<uint16_t *>(smem + lay.list_off);
     uint16_t *perm = reinterpret_cast<uint16_t *>(smem + lay.perm_off);
-    int16_t *table = reinterpret_cast<int16_t *>(smem + lay.table_off);
     int *misc = reinterpret_cast<int *>(smem + lay.misc_off);
     const bool smem_sums = Kp <= 32 && P.first;
     double *ssum = reinterpret_cast<double *>(smem + lay.sums_off);  // [Kp][64] when smem_sums
@@ -264,8 +258,10 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
         *reinterpret_cast<uint4 *>(smem + lay.lo_off + swz(kk, ch)) = vl;
     }
     for (int kk = threadIdx.x; kk < Kp; kk += kThreads) {
-        mm[kk] = P.mm[cb + kk];
+        mm[kk] = kk < K ? P.mm[cb + kk] : INFINITY;
         hsh[kk] = P.hash[cb + kk];
+        dead[kk] = kk < K ? 0 : 1;
+        cnt_s[kk] = 0;
     }
     for (int i = threadIdx.x; i < kTileQ; i += kThreads) cs[i] = i < Lt ? 0 : 0xFF;
     if (threadIdx.x == 0) {
@@ -273,37 +269,17 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
         misc[3] = 0;
     }
     __syncthreads();
-    // dead centroids: padding and bitwise copies of a lower-index centroid
-    {
-        const int kk = threadIdx.x;
-        bool dd = true;
-        if (kk < Kp) {
-            dd = kk >= K;
-            for (int a = 0; a < kk && !dd; ++a) {
-                if (hsh[a] != hsh[kk]) continue;
-                bool same = true;
-                for (int j = 0; j < kD && same; ++j)
-                    same = __float_as_uint(mu[a * mu_ld + j]) == __float_as_uint(mu[kk * mu_ld + j]);
-                dd = same;
-            }
-            dead[kk] = dd ? 1 : 0;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            float mx = 0.f;
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-                const int k2 = lane + 32 * s;
-                if (k2 < Kp) {
-                    if (dead[k2]) mm[k2] = INFINITY;
-                    else mx = fmaxf(mx, mm[k2]);
-                }
-            }
-            mx = warp_max(mx);
-            if (lane == 0) {
-                misc[1] = __float_as_int(mx);
-                misc[2] = __float_as_int(sqrtf(mx));
-            }
+    // dead centroids: bitwise copies of a lower-index centroid (|mu|^2 = +inf);
+    // max |mu|^2 over the live ones (a copy has its original's norm, so the
+    // max over all k < K is the same) from L2.
+    mark_copies(K, hsh, mu, mu_ld, dead, mm, warp, kWarps, lane);
+    if (warp == 0) {
+        float mx = 0.f;
+        for (int k2 = lane; k2 < K; k2 += 32) mx = fmaxf(mx, P.mm[cb + k2]);
+        mx = warp_max(mx);
+        if (lane == 0) {
+            misc[1] = __float_as_int(mx);
+            misc[2] = __float_as_int(sqrtf(mx));
         }
     }
     cp_async_wait<0>();
@@ -432,13 +408,15 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
                 mj0[u] = v0 ? (double)mu[k0 * mu_ld + jb + u] : 0.0;
                 mj1[u] = v1 ? (double)mu[k1 * mu_ld + jb + u] : 0.0;
             }
+            // every product is exact in fp64: one fused multiply-add rounds
+            // exactly as a rounded product followed by a rounded sum
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                qq = __dadd_rn(qq, __dmul_rn(qj[u], qj[u]));
-                qm0 = __dadd_rn(qm0, __dmul_rn(qj[u], mj0[u]));
-                m20 = __dadd_rn(m20, __dmul_rn(mj0[u], mj0[u]));
-                qm1 = __dadd_rn(qm1, __dmul_rn(qj[u], mj1[u]));
-                m21 = __dadd_rn(m21, __dmul_rn(mj1[u], mj1[u]));
+                qq = __fma_rn(qj[u], qj[u], qq);
+                qm0 = __fma_rn(qj[u], mj0[u], qm0);
+                m20 = __fma_rn(mj0[u], mj0[u], m20);
+                qm1 = __fma_rn(qj[u], mj1[u], qm1);
+                m21 = __fma_rn(mj1[u], mj1[u], m21);
             }
         }
         double bd = INFINITY;
@@ -479,8 +457,15 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
     if (!P.first) {
         // Later iterations: only tokens whose cluster changed move between the
         // tile's member sums (exact fp64 subtract / add) and counts.
-        for (int i = threadIdx.x; i < Lt; i += kThreads)
-            if (cs[i] != cprev[i]) list[atomicAdd(&misc[3], 1)] = (uint16_t)i;
+        for (int ch = warp; ch < kTileQ / 32; ch += kWarps) {
+            const int i = ch * 32 + lane;
+            const bool mv = i < Lt && cs[i] != cprev[i];
+            const unsigned bal = __ballot_sync(0xffffffffu, mv);
+            int base = 0;
+            if (lane == 0 && bal) base = atomicAdd(&misc[3], __popc(bal));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (mv) list[base + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)i;
+        }
         __syncthreads();
         const int n_mv = misc[3];
         for (int e = warp; e < n_mv; e += kWarps) {
@@ -501,33 +486,26 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
         }
         return;
     }
-    // stable counting sort of the tile's tokens by cluster
-    const int nch = kTileQ / 32;
-    for (int i = threadIdx.x; i < nch * Kp; i += kThreads) table[i] = 0;
-    __syncthreads();
-    int my_c[2], my_rank[2];
+    // counting sort of the tile's tokens by cluster (order inside a cluster
+    // is free: the sums are exact).  Peers of one cluster in a 32-token chunk
+    // take their offsets with one atomic on the count; every warp then scans
+    // the counts itself.
+    {
+        int my_c[2], my_off[2];
 #pragma unroll
-    for (int s = 0; s < 2; ++s) {
-        const int ch = warp + s * kWarps;
-        const int c = cs[ch * 32 + lane];
-        const unsigned peers = __match_any_sync(0xffffffffu, c);
-        my_c[s] = c;
-        my_rank[s] = __popc(peers & ((1u << lane) - 1u));
-        if (c != 0xFF && lane == __ffs(peers) - 1) table[ch * Kp + c] = (int16_t)__popc(peers);
-    }
-    __syncthreads();
-    if (threadIdx.x < Kp) {
-        int run = 0;
-        for (int ch = 0; ch < nch; ++ch) {
-            const int v = table[ch * Kp + threadIdx.x];
-            table[ch * Kp + threadIdx.x] = (int16_t)run;
-            run += v;
+        for (int s2 = 0; s2 < 2; ++s2) {
+            const int ch = warp + s2 * kWarps;
+            const int c = cs[ch * 32 + lane];
+            const unsigned peers = __match_any_sync(0xffffffffu, c);
+            const int leader = __ffs(peers) - 1;
+            int off = 0;
+            if (c != 0xFF && lane == leader) off = atomicAdd(&cnt_s[c], __popc(peers));
+            off = __shfl_sync(0xffffffffu, off, leader);
+            my_c[s2] = c;
+            my_off[s2] = off + __popc(peers & ((1u << lane) - 1u));
         }
-        cnt_s[threadIdx.x] = run;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        int c0 = lane < Kp ? cnt_s[lane] : 0, c1 = lane + 32 < Kp ? cnt_s[lane + 32] : 0;
+        __syncthreads();
+        const int c0 = lane < Kp ? cnt_s[lane] : 0, c1 = lane + 32 < Kp ? cnt_s[lane + 32] : 0;
         int s0 = c0, s1 = c1;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -537,18 +515,16 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
                 s1 += x1;
             }
         }
-        const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
-        if (lane < Kp) base_s[lane] = s0 - c0;
-        if (lane + 32 < Kp) base_s[lane + 32] = tot0 + s1 - c1;
-    }
-    __syncthreads();
+        const int b0 = s0 - c0, b1 = __shfl_sync(0xffffffffu, s0, 31) + s1 - c1;
 #pragma unroll
-    for (int s = 0; s < 2; ++s) {
-        const int ch = warp + s * kWarps;
-        if (my_c[s] != 0xFF) {
-            const int pos = base_s[my_c[s]] + table[ch * Kp + my_c[s]] + my_rank[s];
-            perm[pos] = (uint16_t)(ch * 32 + lane);
-            sc[pos] = (uint8_t)my_c[s];
+        for (int s2 = 0; s2 < 2; ++s2) {
+            const int c = my_c[s2];
+            const int x0 = __shfl_sync(0xffffffffu, b0, c & 31), x1 = __shfl_sync(0xffffffffu, b1, c & 31);
+            if (c != 0xFF) {
+                const int pos = (c < 32 ? x0 : x1) + my_off[s2];
+                perm[pos] = (uint16_t)((warp + s2 * kWarps) * 32 + lane);
+                sc[pos] = (uint8_t)c;
+            }
         }
     }
     __syncthreads();
