@@ -55,6 +55,28 @@ def test_gmm_with_tiny_clusters_and_exact_ties():
     np.testing.assert_array_equal(g["cent"], ref_cent)
 
 
+@pytest.mark.parametrize("L,K,profile_kernel", [(512, 64, "fused_forward"), (1500, 64, "tiled_assign")])
+def test_three_distinct_queries(L, K, profile_kernel):
+    # Every query is one of three rows: all but three strided starting centroids
+    # are bitwise copies of a lower one, most clusters end empty (zero
+    # centroids, themselves copies of each other) and all distances tie.
+    from means_cluster_attention_b200 import _lib
+    w = Workload("three_rows", 1, 2, L, 64, K, 3, 32, 0.5, "bf16", "normal")
+    x = make_inputs(w, seed=L + K)
+    src = np.random.default_rng(L).integers(0, 3, size=L)
+    for key in ("q", "q64"):
+        x[key] = np.ascontiguousarray(x[key][:, :, src, :])
+    _lib.profile_start(profile_kernel)
+    g = run_gpu(x, "bf16", K, w.iters, w.W, w.alpha, hist=True)
+    stat = _lib.profile_stop()
+    assert stat.launches > 0, f"{profile_kernel} did not run"
+    ref_out, ref_assign, ref_cent, ref_hist = oracle.forward(x["q64"], x["k64"], x["v64"], K=K, iters=w.iters,
+                                                             W=w.W, alpha=w.alpha, hist=True)
+    np.testing.assert_array_equal(g["hist"], ref_hist)
+    np.testing.assert_array_equal(g["cent"], ref_cent)
+    assert float(np.abs(g["out"] - ref_out).max()) <= TOL["bf16"]
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_deterministic(dtype):
     import torch
