@@ -817,7 +817,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_centroid_kernel(CentroidPar
 // Window attention + gather + blend for 128 queries; any radius <= kMaxR.
 struct WindowLayout {
     int rows, Kp;
-    uint32_t k_off, v_off, vc_off, c_off, total;
+    uint32_t k_off, v_off, vc_off, c_off, st_off, total;
     __host__ __device__ WindowLayout(int K, int r) {
         Kp = kpad(K);
         rows = (int)up((uint32_t)(kWinQ + 2 * r + 8), 8);
@@ -826,10 +826,12 @@ struct WindowLayout {
         o += (uint32_t)rows * 128u;
         v_off = o;
         o += (uint32_t)rows * 128u;
-        vc_off = o;
-        o += (uint32_t)K * 64u * 4u;
+        vc_off = o;  // (1 - alpha) V_cent, rows of fused::kVcStride floats
+        o += (uint32_t)K * (uint32_t)fused::kVcStride * 4u;
         c_off = o;
         o += (uint32_t)kWinQ * 4u;
+        st_off = o;  // per-warp output staging, 8 rows x 128 bytes
+        o += (uint32_t)kWarps * 1024u;
         total = up(o, 128);
     }
 };
@@ -865,8 +867,15 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
     load_rows(vw_s, vh, ks0, nrows, ke + 1);
     cp_async_commit();
     const float *vch = P.vcent + head * (int64_t)K * kD;
-    for (int e = threadIdx.x; e < K * kD / 4; e += kThreads)
-        reinterpret_cast<float4 *>(vc)[e] = reinterpret_cast<const float4 *>(vch)[e];
+    const float be = 1.f - P.alpha;
+    for (int e = threadIdx.x; e < K * kD / 4; e += kThreads) {
+        float4 x = reinterpret_cast<const float4 *>(vch)[e];
+        x.x *= be;
+        x.y *= be;
+        x.z *= be;
+        x.w *= be;
+        *reinterpret_cast<float4 *>(vc + (e >> 4) * fused::kVcStride + (e & 15) * 4) = x;
+    }
     for (int i = threadIdx.x; i < kWinQ; i += kThreads) cblk[i] = (qb + i < L) ? P.assign[head * L + qb + i] : 0;
     const int i0 = qb + warp * 16;
     uint32_t a[4][4];
@@ -914,18 +923,23 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
 #pragma unroll
         for (int n = 0; n < kNTChunk; ++n) {
             if (n < cn) {
+                // keys j0..j0+7 against rows i0..i0+15: only a tile that is not
+                // inside every row's band (and inside [0, L)) needs the mask
+                const int j0 = kst + (c0 + n) * 8;
+                if (!(j0 >= i0 + 15 - r && j0 + 7 <= i0 + r && j0 + 7 < L)) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i = i0 + g + 8 * (e >> 1);
-                    const int jk = kst + (c0 + n) * 8 + 2 * t + (e & 1);
-                    const bool ok = jk >= i - r && jk <= i + r && jk < L;
-                    if (!ok) sacc[n][e] = -INFINITY;
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = i0 + g + 8 * (e >> 1);
+                        const int jk = j0 + 2 * t + (e & 1);
+                        const bool ok = jk >= i - r && jk <= i + r && jk < L;
+                        if (!ok) sacc[n][e] = -INFINITY;
+                    }
                 }
                 mx[0] = fmaxf(mx[0], fmaxf(sacc[n][0], sacc[n][1]));
                 mx[1] = fmaxf(mx[1], fmaxf(sacc[n][2], sacc[n][3]));
             }
         }
-        float corr[2];
+        float corr[2], mhc[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
@@ -934,6 +948,8 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
             corr[h] = (mn == -INFINITY) ? 1.f : ex2((m_run[h] - mn) * csc);
             m_run[h] = mn;
             l_run[h] *= corr[h];
+            // a row with no key yet: every score is -inf and p = 0
+            mhc[h] = (mn == -INFINITY) ? 0.f : mn * csc;
         }
 #pragma unroll
         for (int d = 0; d < 8; ++d) {
@@ -949,10 +965,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
             if (n < cn) {
                 float p[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float mh = m_run[e >> 1];
-                    p[e] = (mh == -INFINITY) ? 0.f : ex2((sacc[n][e] - mh) * csc);
-                }
+                for (int e = 0; e < 4; ++e) p[e] = ex2(fmaf(sacc[n][e], csc, -mhc[e >> 1]));
                 l_run[0] += p[0] + p[1];
                 l_run[1] += p[2] + p[3];
                 pa[n][0] = pack_bf16(p[0], p[1]);
@@ -987,24 +1000,39 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
         l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
         l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
     }
-    const float inv0 = l_run[0] > 0.f ? 1.f / l_run[0] : 0.f, inv1 = l_run[1] > 0.f ? 1.f / l_run[1] : 0.f;
-    const int ia = i0 + g, ib = i0 + g + 8;
-    const int ca = ia < L ? cblk[ia - qb] : 0, cb2 = ib < L ? cblk[ib - qb] : 0;
-    const float al = P.alpha, be = 1.f - P.alpha;
+    // gather + blend: O = (1 - alpha) V_cent[c_i] + alpha o_i, staged eight
+    // rows at a time through shared memory (stmatrix) and stored as whole
+    // 128-byte rows
+    const float f0 = l_run[0] > 0.f ? P.alpha / l_run[0] : 0.f, f1 = l_run[1] > 0.f ? P.alpha / l_run[1] : 0.f;
     __nv_bfloat16 *oh = P.out + head * (int64_t)L * kD;
+    const uint32_t ost = sbase + lay.st_off + warp * 1024;
 #pragma unroll
-    for (int d = 0; d < 8; ++d) {
-        const int col = 8 * d + 2 * t;
-        if (ia < L) {
-            const float y0 = be * vc[ca * kD + col] + al * (oacc[d][0] * inv0);
-            const float y1 = be * vc[ca * kD + col + 1] + al * (oacc[d][1] * inv0);
-            *reinterpret_cast<uint32_t *>(oh + (int64_t)ia * kD + col) = pack_bf16(y0, y1);
+    for (int hh = 0; hh < 2; ++hh) {
+        const int i = i0 + g + 8 * hh;
+        const float f = hh ? f1 : f0;
+        const float *vrow = vc + (i < L ? cblk[i - qb] : 0) * fused::kVcStride + 2 * t;
+        uint32_t wv[8];
+#pragma unroll
+        for (int d = 0; d < 8; ++d) {
+            const float2 c2 = *reinterpret_cast<const float2 *>(vrow + 8 * d);
+            wv[d] = pack_bf16(fmaf(f, oacc[d][2 * hh], c2.x), fmaf(f, oacc[d][2 * hh + 1], c2.y));
         }
-        if (ib < L) {
-            const float y2 = be * vc[cb2 * kD + col] + al * (oacc[d][2] * inv1);
-            const float y3 = be * vc[cb2 * kD + col + 1] + al * (oacc[d][3] * inv1);
-            *reinterpret_cast<uint32_t *>(oh + (int64_t)ib * kD + col) = pack_bf16(y2, y3);
+        const int sr = lane & 7, sd = lane >> 3;
+        stmatrix_x4(ost + sr * 128 + ((sd ^ sr) << 4), wv[0], wv[1], wv[2], wv[3]);
+        stmatrix_x4(ost + sr * 128 + (((sd + 4) ^ sr) << 4), wv[4], wv[5], wv[6], wv[7]);
+        __syncwarp();
+#pragma unroll
+        for (int it2 = 0; it2 < 2; ++it2) {
+            const int rr = it2 * 4 + (lane >> 3), ch = lane & 7;
+            const int row = i0 + 8 * hh + rr;
+            uint4 val;
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                         : "r"(ost + rr * 128 + ((ch ^ rr) << 4))
+                         : "memory");
+            if (row < L) *reinterpret_cast<uint4 *>(oh + (int64_t)row * kD + ch * 8) = val;
         }
+        __syncwarp();
     }
 }
 
