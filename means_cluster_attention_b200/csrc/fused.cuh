@@ -664,16 +664,26 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         for (int e = 0; e < 4; ++e) o_acc[d][e] = 0.f;
     float rm[2] = {-INFINITY, -INFINITY}, rl[2] = {0.f, 0.f};
 
+    // One group is committed per iteration (empty when there is nothing to
+    // load), so tile tt's group is always the fifth newest at the wait.  The
+    // slot of tile tt-1 is refilled right after the barrier that shows every
+    // warp is done with it.
     for (int tt = 0; tt < nT; ++tt) {
         cp_async_wait<kSlots - 1>();
         __syncthreads();
+        if (tt >= 1 && tt - 1 + kSlots < nT) {
+            const uint32_t ks = big_s + ((tt - 1) % kSlots) * 2 * kTile * 128;
+            load_rows(ks, kh, (tt - 1 + kSlots) * kTile, kTile, L);
+            load_rows(ks + kTile * 128, vh, (tt - 1 + kSlots) * kTile, kTile, L);
+        }
+        cp_async_commit();
         const uint32_t kt = big_s + (tt % kSlots) * 2 * kTile * 128;
         const uint32_t vt = kt + kTile * 128;
-        float sacc[4][4];
+        float sacc[4][4], slo[4][4];
 #pragma unroll
         for (int n = 0; n < 4; ++n)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) sacc[n][e] = 0.f;
+            for (int e = 0; e < 4; ++e) sacc[n][e] = slo[n][e] = 0.f;
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
             if (n * 8 >= keys_w) break;
@@ -683,10 +693,12 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                 uint32_t bk[4];
                 ldmatrix_x4(bk, kt + swz(key0 + (lane & 7), 4 * kp + (lane >> 3)));
                 mma_16816(sacc[n], ahi[2 * kp], bk[0], bk[1]);
+                mma_16816(slo[n], alo[2 * kp], bk[0], bk[1]);
                 mma_16816(sacc[n], ahi[2 * kp + 1], bk[2], bk[3]);
-                mma_16816(sacc[n], alo[2 * kp], bk[0], bk[1]);
-                mma_16816(sacc[n], alo[2 * kp + 1], bk[2], bk[3]);
+                mma_16816(slo[n], alo[2 * kp + 1], bk[2], bk[3]);
             }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[n][e] += slo[n][e];
         }
         float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
@@ -700,21 +712,25 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
             tmax[1] = fmaxf(tmax[1], fmaxf(sacc[n][2], sacc[n][3]));
         }
         float corr[2];
+        bool grew = false;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 1));
             tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 2));
             const float mn = fmaxf(rm[h], tmax[h]);
+            grew |= mn != rm[h];
             corr[h] = (mn == -INFINITY) ? 1.f : ex2((rm[h] - mn) * csc);
             rm[h] = mn;
             rl[h] *= corr[h];
         }
+        if (__any_sync(0xffffffffu, grew)) {
 #pragma unroll
-        for (int d = 0; d < 8; ++d) {
-            o_acc[d][0] *= corr[0];
-            o_acc[d][1] *= corr[0];
-            o_acc[d][2] *= corr[1];
-            o_acc[d][3] *= corr[1];
+            for (int d = 0; d < 8; ++d) {
+                o_acc[d][0] *= corr[0];
+                o_acc[d][1] *= corr[0];
+                o_acc[d][2] *= corr[1];
+                o_acc[d][3] *= corr[1];
+            }
         }
         uint32_t pa[4][2];
 #pragma unroll
@@ -757,12 +773,6 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                 }
             }
         }
-        __syncthreads();
-        if (tt + kSlots < nT) {
-            load_rows(kt, kh, (tt + kSlots) * kTile, kTile, L);
-            load_rows(vt, vh, (tt + kSlots) * kTile, kTile, L);
-        }
-        cp_async_commit();
     }
     cp_async_wait<0>();
     // combine the G partial states of each centroid m-tile (big region reused)
@@ -824,7 +834,6 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         cp_async_commit();
     };
     issue_block(0);
-    issue_block(1);
     __nv_bfloat16 *oh = P.out + head * (int64_t)L * kD;
     // Band mask of a warp's 16 x (8 kMaxNT) score tile as bits 4n+e: key
     // kst + 8n + 2t + (e&1) against query i0 + g + 8(e>>1).  A warp whose
@@ -862,12 +871,15 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         }
     };
     fetch_q(0);
+    // Block b's stage is waited for, then the other stage (last read by
+    // block b-1, which every warp has left at this barrier) takes block b+1.
     for (int b = 0; b < nblk; ++b) {
         const int qb = b * kWinBlock;
         const int ks0 = max(0, qb - r) & ~7;
         const int i0 = qb + warp * 16;
-        cp_async_wait<1>();
+        cp_async_wait<0>();
         __syncthreads();
+        issue_block(b + 1);
         const uint32_t kw_s = big_s + (b & 1) * lay.win_stage;
         const uint32_t vw_s = kw_s + lay.win_rows * 128;
         if (i0 < L) {
@@ -990,8 +1002,6 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
             }
         }
         fetch_q(b + 1);
-        __syncthreads();
-        issue_block(b + 2);
     }
     cp_async_wait<0>();
 }
