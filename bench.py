@@ -18,6 +18,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -169,9 +170,18 @@ def cpu_oracle_rate(w, target_s: float, max_heads=None):
     t0 = time.perf_counter()
     oracle.forward(x["q64"], x["k64"], x["v64"], K=w.K, iters=w.iters, W=w.W, alpha=w.alpha, nthreads=used)
     dt = time.perf_counter() - t0
-    toks = heads * w.L
-    sample = (f"{heads} of {w.heads} heads (L={w.L}) of {w.name}, same recipe and sizes, "
-              f"{toks} tokens in {dt:.2f} s on {used} threads")
+    passes = 1
+    if heads == w.heads and dt < target_s:
+        # the whole workload is shorter than the target: time repeated passes
+        passes = int(min(1000, math.ceil(target_s / max(dt, 1e-3))))
+        t0 = time.perf_counter()
+        for _ in range(passes):
+            oracle.forward(x["q64"], x["k64"], x["v64"], K=w.K, iters=w.iters, W=w.W, alpha=w.alpha,
+                           nthreads=used)
+        dt = time.perf_counter() - t0
+    toks = heads * w.L * passes
+    sample = (f"{passes} pass(es) over {heads} of {w.heads} heads (L={w.L}) of {w.name}, same recipe "
+              f"and sizes, {toks} tokens in {dt:.2f} s on {used} threads")
     return toks / dt, used, sample, dt
 
 
