@@ -190,7 +190,7 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     # Each step: a bounded head sample sized so warmup + steps end within ~3 min.
-    per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = max(0.5, min(10.0, args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
     rates = []
     cores = sample = None
     for i in range(args.warmup + args.steps):

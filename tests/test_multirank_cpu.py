@@ -46,7 +46,7 @@ def test_max_over_ranks_and_weak_scaling_rate():
 def test_reference_arm_nonzero_rank_exits_quietly():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--workload", "small_f32", "--steps", "1", "--warmup", "3"],
+                        "--workload", "small_f32", "--steps", "1", "--warmup", "3", "--cpu-seconds", "0.5"],
                        env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
@@ -56,7 +56,7 @@ def test_reference_arm_rank0_prints_one_line():
     import json
     env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--workload", "small_f32", "--steps", "1", "--warmup", "3"],
+                        "--workload", "small_f32", "--steps", "1", "--warmup", "3", "--cpu-seconds", "0.5"],
                        env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr
     lines = [l for l in r.stdout.splitlines() if l.strip()]
