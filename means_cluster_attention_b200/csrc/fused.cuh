@@ -59,7 +59,7 @@ __host__ __device__ inline uint32_t umax(uint32_t a, uint32_t b) { return a > b 
 
 struct Layout {
     int Lp, Kp, r, nT, win_rows;
-    uint32_t big_off, sums_off, mu_off, hi_off, lo_off, vc_off, mm_off, hash_off, dead_off, c_off,
+    uint32_t big_off, sums_off, mu64_off, mu_off, hi_off, lo_off, vc_off, mm_off, hash_off, dead_off, c_off,
         list_off, perm_off, sc_off, cprev_off, cnt_off, misc_off, ml_off, win_stage,
         total;
 
@@ -73,13 +73,15 @@ struct Layout {
         win_stage = 2u * (uint32_t)win_rows * 128u;
         const uint32_t q_bytes = (uint32_t)Lp * 128u;
         const uint32_t sums_bytes = (uint32_t)Kp * 64u * 8u;
+        const uint32_t mu64_bytes = (uint32_t)Kp * 65u * 8u;  // fp64 centroid copy for the re-measure
         const uint32_t slots = (uint32_t)(nT < kSlots ? nT : kSlots);
-        uint32_t big = umax(q_bytes + sums_bytes, slots * 2u * kTile * 128u);
+        uint32_t big = umax(q_bytes + sums_bytes + mu64_bytes, slots * 2u * kTile * 128u);
         big = umax(big, 2u * win_stage);
         big = umax(big, (uint32_t)kWarps * 16u * 64u * 4u);  // centroid-phase combine scratch
         uint32_t o = 0;
         big_off = o;
         sums_off = q_bytes;
+        mu64_off = q_bytes + sums_bytes;
         o += up(big, 1024);
         mu_off = o;
         o += up((uint32_t)Kp * 65u * 4u, 128);
@@ -226,6 +228,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     uint32_t *hsh = reinterpret_cast<uint32_t *>(smem + lay.hash_off);
     int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
     double *sums = reinterpret_cast<double *>(smem + lay.big_off + lay.sums_off);  // [Kp][64]
+    double *mu64 = reinterpret_cast<double *>(smem + lay.big_off + lay.mu64_off);  // [Kp][65], exact copy of mu
     uint8_t *dead = smem + lay.dead_off;
     uint8_t *cs = smem + lay.c_off;                                              // [Lp]
     uint8_t *sc = smem + lay.sc_off;        // [Lp] cluster ids in sorted order
@@ -276,6 +279,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     auto finalize_row = [&](int kk, float x0, float x1) {
         mu[kk * 65 + 2 * lane] = x0;
         mu[kk * 65 + 2 * lane + 1] = x1;
+        mu64[kk * 65 + 2 * lane] = (double)x0;
+        mu64[kk * 65 + 2 * lane + 1] = (double)x1;
         const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
         const __nv_bfloat16 l0 = __float2bfloat16_rn(x0 - __bfloat162float(h0));
         const __nv_bfloat16 l1 = __float2bfloat16_rn(x1 - __bfloat162float(h1));
@@ -430,8 +435,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                 }
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    mj0[u] = v0 ? (double)mu[k0 * 65 + jb + u] : 0.0;
-                    mj1[u] = v1 ? (double)mu[k1 * 65 + jb + u] : 0.0;
+                    mj0[u] = v0 ? mu64[k0 * 65 + jb + u] : 0.0;
+                    mj1[u] = v1 ? mu64[k1 * 65 + jb + u] : 0.0;
                 }
                 // Every product (bf16 x bf16, bf16 x fp32, fp32 x fp32) is
                 // exact in fp64, so one fused multiply-add rounds exactly as
