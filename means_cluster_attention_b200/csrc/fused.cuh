@@ -35,6 +35,8 @@
 // order of the adds.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "mma.cuh"
 
@@ -418,11 +420,13 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         // (2) exact re-measure of ambiguous tokens, one warp per token
         const int n_ref = misc[0];
         if (threadIdx.x == 0) misc[1] = 0;
-        for (int e = warp; e < n_ref; e += kWarps) {
-            const int row = list[e];
+        // Lane k holds centroid k (and k + 32 when Kp = 64); the chains of
+        // the second set are only run when that set exists.
+        auto remeasure = [&](int row, auto two_c, double &bd, int &bk) {
+            constexpr bool two = decltype(two_c)::value;
             double qq = 0.0, qm0 = 0.0, qm1 = 0.0, m20 = 0.0, m21 = 0.0;
             const int k0 = lane, k1 = lane + 32;
-            const bool v0 = k0 < Kp, v1 = k1 < Kp;
+            const bool v0 = k0 < Kp, v1 = two && k1 < Kp;
 #pragma unroll 2
             for (int jb = 0; jb < kD; jb += 8) {
                 const uint4 w = *reinterpret_cast<const uint4 *>(qbytes + swz(row, jb >> 3));
@@ -436,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     mj0[u] = v0 ? mu64[k0 * 65 + jb + u] : 0.0;
-                    mj1[u] = v1 ? mu64[k1 * 65 + jb + u] : 0.0;
+                    if constexpr (two) mj1[u] = v1 ? mu64[k1 * 65 + jb + u] : 0.0;
                 }
                 // Every product (bf16 x bf16, bf16 x fp32, fp32 x fp32) is
                 // exact in fp64, so one fused multiply-add rounds exactly as
@@ -446,12 +450,14 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                     qq = __fma_rn(qj[u], qj[u], qq);
                     qm0 = __fma_rn(qj[u], mj0[u], qm0);
                     m20 = __fma_rn(mj0[u], mj0[u], m20);
-                    qm1 = __fma_rn(qj[u], mj1[u], qm1);
-                    m21 = __fma_rn(mj1[u], mj1[u], m21);
+                    if constexpr (two) {
+                        qm1 = __fma_rn(qj[u], mj1[u], qm1);
+                        m21 = __fma_rn(mj1[u], mj1[u], m21);
+                    }
                 }
             }
-            double bd = INFINITY;
-            int bk = 0x7fffffff;
+            bd = INFINITY;
+            bk = 0x7fffffff;
             if (v0 && !dead[k0]) {
                 bd = __dsub_rn(__dadd_rn(qq, m20), __dmul_rn(2.0, qm0));
                 bk = k0;
@@ -463,6 +469,13 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                     bk = k1;
                 }
             }
+        };
+        for (int e = warp; e < n_ref; e += kWarps) {
+            const int row = list[e];
+            double bd;
+            int bk;
+            if (Kp > 32) remeasure(row, std::true_type{}, bd, bk);
+            else remeasure(row, std::false_type{}, bd, bk);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 const double od = __shfl_xor_sync(0xffffffffu, bd, o);
@@ -618,16 +631,28 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         __syncthreads();
         for (int i = threadIdx.x; i < Lp; i += kThreads) cprev[i] = cs[i];
         // (5) mu_k = fp32(sum_k / max(1, count_k)), one warp per centroid
+        // (two rows per warp at a time, so their fp64 divisions overlap)
         const bool last = it == P.iters - 1;
-        for (int kk = warp; kk < Kp; kk += kWarps) {
-            const int cnt = kk < K ? cnt_s[kk] : 0;
-            const double den = (double)(cnt > 1 ? cnt : 1);
-            const float x0 = kk < K ? __double2float_rn(sums[kk * kD + 2 * lane] / den) : 0.f;
-            const float x1 = kk < K ? __double2float_rn(sums[kk * kD + 2 * lane + 1] / den) : 0.f;
-            finalize_row(kk, x0, x1);
-            if (last && P.cent && kk < K) {
-                float2 *dst = reinterpret_cast<float2 *>(P.cent + (head * K + kk) * kD);
-                dst[lane] = make_float2(x0, x1);
+        for (int kb2 = warp; kb2 < Kp; kb2 += 2 * kWarps) {
+            float x[2][2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int kk = kb2 + h * kWarps;
+                const int cnt = kk < K ? cnt_s[kk] : 0;
+                const double den = (double)(cnt > 1 ? cnt : 1);
+                x[h][0] = kk < K ? __double2float_rn(sums[kk * kD + 2 * lane] / den) : 0.f;
+                x[h][1] = kk < K ? __double2float_rn(sums[kk * kD + 2 * lane + 1] / den) : 0.f;
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int kk = kb2 + h * kWarps;
+                if (kk < Kp) {
+                    finalize_row(kk, x[h][0], x[h][1]);
+                    if (last && P.cent && kk < K) {
+                        float2 *dst = reinterpret_cast<float2 *>(P.cent + (head * K + kk) * kD);
+                        dst[lane] = make_float2(x[h][0], x[h][1]);
+                    }
+                }
             }
         }
         finalize_set(P.hist ? P.hist + (head * P.iters + it) * (int64_t)L : nullptr);
