@@ -12,8 +12,9 @@
 //                                          exact argmin) and the tile's exact
 //                                          fp64 member sums.
 //   tiled_centroid_kernel  (chunks, heads) partial softmax state of every
-//                                          centroid over 512 keys; combined by
-//                                          centroid_attn_combine_kernel.
+//                                          centroid over 512 keys;
+//   tiled_combine_kernel   (K, heads)      combines the chunk states into
+//                                          V_cent.
 //   tiled_window_kernel    (blocks, heads) clipped window attention for 128
 //                                          queries, gather V_cent[c_i], blend.
 //
