@@ -8,6 +8,7 @@ from __future__ import annotations
 
 import glob
 import hashlib
+import re
 import os
 import shutil
 import subprocess
@@ -44,14 +45,23 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text: bytes) -> bytes:
+    """Source text without comments and blank lines: edits to comments do not
+    change the kernel a measurement was taken on."""
+    t = re.sub(rb"/\*.*?\*/", b"", text, flags=re.S)
+    t = re.sub(rb"//[^\n]*", b"", t)
+    return b"\n".join(line.rstrip() for line in t.splitlines() if line.strip())
+
+
 def source_hash(kernel: str = None) -> str:
-    """Hash of the sources a kernel is built from (all sources if None)."""
+    """Hash of the code (comments excluded) a kernel is built from (all
+    sources if None)."""
     files = sources() if kernel is None else [os.path.join(CSRC, f) for f in KERNEL_SOURCES[kernel]]
     h = hashlib.sha256()
     for s in files:
         h.update(os.path.basename(s).encode())
         with open(s, "rb") as f:
-            h.update(f.read())
+            h.update(_code_only(f.read()))
     return h.hexdigest()[:16]
 
 
