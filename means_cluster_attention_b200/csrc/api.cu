@@ -493,6 +493,28 @@ ca_status ca_forward_ex(const void *q, const void *k, const void *v, int dtype, 
     return fail(CA_ERR_INVALID_ARG, "dtype must be 0 (fp32) or 1 (bf16), got %d", dtype);
 }
 
+// Two library-owned streams per device for the host-buffer entry point: one
+// runs the kernels, one copies results back, so that with several chunks the
+// copies in, the kernels and the copies out of different chunks overlap.
+cudaError_t host_streams(cudaStream_t *comp, cudaStream_t *back) {
+    static std::mutex mu;
+    static cudaStream_t streams[64][2] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> g(mu);
+    for (int i = 0; i < 2; ++i) {
+        if (!streams[dev][i]) {
+            e = cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking);
+            if (e != cudaSuccess) return e;
+        }
+    }
+    *comp = streams[dev][0];
+    *back = streams[dev][1];
+    return cudaSuccess;
+}
+
 ca_status ca_forward_host(const void *q, const void *k, const void *v, int dtype, int B, int H,
                           int L, int d, int K, int iters, int W, float alpha, void *out,
                           int32_t *assign_out, float *centroids_out, void *stream) {
@@ -503,27 +525,76 @@ ca_status ca_forward_host(const void *q, const void *k, const void *v, int dtype
     if (s != CA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
     const size_t esz = dtype == 0 ? 4 : 2;
-    const size_t n = (size_t)p.heads() * p.L * p.d;
+    const int64_t NH = p.heads();
+    const size_t head_elems = (size_t)p.L * p.d;
+    const size_t n = (size_t)NH * head_elems;
+    // Heads are independent: a large problem runs as up to eight chunks of
+    // whole heads, each copied in, computed and copied back in turn.
+    const int n_chunks = (NH >= 2 && n * esz * 4 >= (size_t(32) << 20)) ? (int)(NH < 8 ? NH : 8) : 1;
+    cudaStream_t s_comp = st, s_back = st;
+    if (n_chunks > 1) CA_CUDA(host_streams(&s_comp, &s_back));
+    cudaEvent_t ev[2 * 8 + 2] = {};
+    const int n_ev = n_chunks > 1 ? 2 * n_chunks + 2 : 0;
+    for (int i = 0; i < n_ev; ++i) CA_CUDA(cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming));
+    struct Events {
+        cudaEvent_t *ev;
+        int n;
+        ~Events() {
+            for (int i = 0; i < n; ++i) cudaEventDestroy(ev[i]);
+        }
+    } ev_guard{ev, n_ev};
     void *dq = nullptr, *dk = nullptr, *dv = nullptr, *dout = nullptr, *dcent = nullptr;
     int32_t *dassign = nullptr;
     {
         Scratch sc(st);
+        // Before the scratch is released on st (or on any early return),
+        // st waits for everything queued on the other two streams.
+        struct Join {
+            cudaStream_t st, a, b;
+            cudaEvent_t ea, eb;
+            bool on;
+            ~Join() {
+                if (!on) return;
+                cudaEventRecord(ea, a);
+                cudaEventRecord(eb, b);
+                cudaStreamWaitEvent(st, ea, 0);
+                cudaStreamWaitEvent(st, eb, 0);
+            }
+        } join{st, s_comp, s_back, n_ev ? ev[n_ev - 2] : nullptr, n_ev ? ev[n_ev - 1] : nullptr, n_chunks > 1};
         CA_CUDA(sc.get(&dq, n * esz));
         CA_CUDA(sc.get(&dk, n * esz));
         CA_CUDA(sc.get(&dv, n * esz));
         CA_CUDA(sc.get(&dout, n * esz));
-        if (assign_out) CA_CUDA(sc.get((void **)&dassign, sizeof(int32_t) * p.heads() * p.L));
-        if (centroids_out) CA_CUDA(sc.get(&dcent, sizeof(float) * p.heads() * p.K * p.d));
-        CA_CUDA(cudaMemcpyAsync(dq, q, n * esz, cudaMemcpyHostToDevice, st));
-        CA_CUDA(cudaMemcpyAsync(dk, k, n * esz, cudaMemcpyHostToDevice, st));
-        CA_CUDA(cudaMemcpyAsync(dv, v, n * esz, cudaMemcpyHostToDevice, st));
-        s = dispatch(dq, dk, dv, dtype, p, dout, dassign, (float *)dcent, nullptr, stream);
-        if (s != CA_OK) return s;
-        CA_CUDA(cudaMemcpyAsync(out, dout, n * esz, cudaMemcpyDeviceToHost, st));
-        if (assign_out)
-            CA_CUDA(cudaMemcpyAsync(assign_out, dassign, sizeof(int32_t) * p.heads() * p.L, cudaMemcpyDeviceToHost, st));
-        if (centroids_out)
-            CA_CUDA(cudaMemcpyAsync(centroids_out, dcent, sizeof(float) * p.heads() * p.K * p.d, cudaMemcpyDeviceToHost, st));
+        if (assign_out) CA_CUDA(sc.get((void **)&dassign, sizeof(int32_t) * NH * p.L));
+        if (centroids_out) CA_CUDA(sc.get(&dcent, sizeof(float) * NH * p.K * p.d));
+        for (int c = 0; c < n_chunks; ++c) {
+            const int64_t h0 = c * NH / n_chunks, h1 = (c + 1) * NH / n_chunks;
+            const size_t off = (size_t)h0 * head_elems * esz, bytes = (size_t)(h1 - h0) * head_elems * esz;
+            CA_CUDA(cudaMemcpyAsync((char *)dq + off, (const char *)q + off, bytes, cudaMemcpyHostToDevice, st));
+            CA_CUDA(cudaMemcpyAsync((char *)dk + off, (const char *)k + off, bytes, cudaMemcpyHostToDevice, st));
+            CA_CUDA(cudaMemcpyAsync((char *)dv + off, (const char *)v + off, bytes, cudaMemcpyHostToDevice, st));
+            if (n_chunks > 1) {
+                CA_CUDA(cudaEventRecord(ev[2 * c], st));
+                CA_CUDA(cudaStreamWaitEvent(s_comp, ev[2 * c], 0));
+            }
+            const Problem pc{1, (int)(h1 - h0), p.L, p.d, p.K, p.iters, p.W, p.alpha};
+            int32_t *da = dassign ? dassign + h0 * p.L : nullptr;
+            float *dc = dcent ? (float *)dcent + h0 * p.K * p.d : nullptr;
+            s = dispatch((char *)dq + off, (char *)dk + off, (char *)dv + off, dtype, pc, (char *)dout + off, da, dc,
+                         nullptr, s_comp);
+            if (s != CA_OK) return s;
+            if (n_chunks > 1) {
+                CA_CUDA(cudaEventRecord(ev[2 * c + 1], s_comp));
+                CA_CUDA(cudaStreamWaitEvent(s_back, ev[2 * c + 1], 0));
+            }
+            CA_CUDA(cudaMemcpyAsync((char *)out + off, (char *)dout + off, bytes, cudaMemcpyDeviceToHost, s_back));
+            if (assign_out)
+                CA_CUDA(cudaMemcpyAsync(assign_out + h0 * p.L, da, sizeof(int32_t) * (h1 - h0) * p.L,
+                                        cudaMemcpyDeviceToHost, s_back));
+            if (centroids_out)
+                CA_CUDA(cudaMemcpyAsync(centroids_out + h0 * p.K * p.d, dc, sizeof(float) * (h1 - h0) * p.K * p.d,
+                                        cudaMemcpyDeviceToHost, s_back));
+        }
     }
     CA_CUDA(cudaStreamSynchronize(st));
     return CA_OK;

@@ -111,6 +111,32 @@ def test_host_entry_point_matches_device_path(dtype):
     assert torch.equal(c_h, c_dev.cpu())
 
 
+@pytest.mark.parametrize("dtype,B,H,L,K,W", [
+    ("bf16", 10, 13, 512, 16, 32),   # fused kernel, 130 heads in uneven chunks
+    ("bf16", 2, 8, 4096, 32, 64),    # tiled path, two heads per chunk
+    ("f32", 8, 8, 512, 16, 32),      # general path
+])
+def test_host_entry_point_in_chunks_matches_device_path(dtype, B, H, L, K, W):
+    # Large enough (>= 32 MB of q, k, v, out) for the host entry point to copy
+    # in, compute and copy back in chunks of whole heads on three streams.
+    import torch
+    import means_cluster_attention_b200 as ca
+    from helpers import to_device
+    w = Workload("host_chunks", B, H, L, 64, K, 3, W, 0.5, dtype, "normal")
+    x = make_inputs(w, seed=11)
+    q, k, v = to_device(x, dtype)
+    o_dev, a_dev, c_dev = ca.forward(q, k, v, w.K, w.iters, w.W, w.alpha, sync_check=True)
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    o_h = torch.empty_like(qh).pin_memory()
+    a_h = torch.empty((B, H, L), dtype=torch.int32).pin_memory()
+    c_h = torch.empty((B, H, K, 64), dtype=torch.float32).pin_memory()
+    ca.forward_host(qh, kh, vh, w.K, w.iters, w.W, w.alpha, out=o_h, assign=a_h, centroids=c_h)
+    ca.sync_status()
+    assert torch.equal(o_h, o_dev.cpu())
+    assert torch.equal(a_h, a_dev.cpu())
+    assert torch.equal(c_h, c_dev.cpu())
+
+
 def test_invalid_call_launches_nothing_and_status_stays_clean():
     import torch
     import means_cluster_attention_b200 as ca
