@@ -123,10 +123,15 @@ ca_status ca_forward_ex(const void *q, const void *k, const void *v, int dtype, 
 
 /* End-to-end form for callers holding HOST buffers (dtype 0 = fp32 with float
  * arrays, 1 = bf16 with uint16 arrays): copies q, k, v to the device, runs the
- * forward on stream, copies out (and assign_out / centroids_out when non-NULL)
- * back and synchronizes the stream before returning.  Host buffers should be
- * pinned for full copy bandwidth; pageable buffers work but copy slower.
- * Device buffers are stream-ordered allocations released before return. */
+ * forward, copies out (and assign_out / centroids_out when non-NULL) back and
+ * returns once everything has completed.  Problems of at least 32 MB (q, k, v
+ * and out together) run as up to eight chunks of whole heads: copies in on
+ * stream, kernels and copies back on two library-owned streams of the current
+ * device, ordered with events, so that the chunks' transfers and kernels
+ * overlap; results are identical to a single pass because heads are
+ * independent.  Host buffers should be pinned for full copy bandwidth and for
+ * the overlap; pageable buffers work but copy slower.  Device buffers are
+ * stream-ordered allocations released before return. */
 ca_status ca_forward_host(const void *q, const void *k, const void *v, int dtype, int B, int H,
                           int L, int d, int K, int iters, int W, float alpha, void *out,
                           int32_t *assign_out, float *centroids_out, void *stream);
