@@ -122,3 +122,14 @@ def test_product_package_never_imports_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
                 assert "liboracle" not in text, f
+
+
+def test_source_hash_ignores_comments_but_not_code():
+    # The bench reports a kernel's DRAM traffic only while the code the
+    # counters were taken on is unchanged; comment edits must not count.
+    base = b"__global__ void f(int *p) {\n    p[0] = 1;  // store\n}\n"
+    commented = b"// header note\n/* block\n   comment */\n__global__ void f(int *p) {\n\n    p[0] = 1;\n}\n"
+    changed = b"__global__ void f(int *p) {\n    p[0] = 2;\n}\n"
+    assert build._code_only(base) == build._code_only(commented)
+    assert build._code_only(base) != build._code_only(changed)
+    assert re.fullmatch(r"[0-9a-f]{16}", build.source_hash("fused_forward"))
