@@ -31,8 +31,20 @@ sys.path.insert(0, ROOT)
 
 METRIC = "cluster-attention fwd tokens/s (B·H·L/s) and achieved HBM GB/s vs ~8 TB/s"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "l512_bf16"
+DEFAULT_WORKLOAD = "l32k_dup_bf16"
+# Timed beside the headline: the other workloads the roofline target is stated on.
+DEFAULT_ALSO = "l4k_gmm_bf16,l512_bf16"
 FALLBACK_HBM_GBS = 6650.0
+# Heads of each workload the parity block re-checks against the fp64 oracle.
+PARITY_HEADS = {"small_f32": 24, "card_gmm_f32": 48, "l512_bf16": 64, "l4k_gmm_bf16": 12,
+                "l32k_dup_bf16": 8}
+PRECISION = {
+    "bf16": ("bf16 Q/K/V and O in HBM; bf16 tensor-core operands with fp32 accumulation; "
+             "k-means decisions exact on fp32 centroids (certified filter + fp64 re-measure, exact fp64 "
+             "member sums); one rounding of O to bf16"),
+    "f32": ("fp32 Q/K/V and O; fp32 FMA with fp64 re-measure for the k-means decisions, exact fp64 "
+            "member sums; fp32 attention arithmetic"),
+}
 # Kernel whose launches the roofline object reports, per workload.
 DOMINANT = {"small_f32": "window_blend", "card_gmm_f32": "window_blend", "l512_bf16": "fused_forward",
             "l4k_gmm_bf16": "tiled_assign", "l32k_dup_bf16": "tiled_assign"}
@@ -150,17 +162,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+_CALIBRATION = {}
+
+
 def cpu_oracle_rate(w, target_s: float, max_heads=None):
     """Time the fp64 oracle (as it stands) on a bounded head sample of the
     workload on this host's cores.  Returns (tokens/s, cores, sample text)."""
     import oracle
     from means_cluster_attention_b200.inputs import make_inputs
     cores = oracle.default_threads()
-    # calibrate on one head, then size the sample to about target_s
-    x1 = make_inputs(w, heads=1)
-    t0 = time.perf_counter()
-    oracle.forward(x1["q64"], x1["k64"], x1["v64"], K=w.K, iters=w.iters, W=w.W, alpha=w.alpha, nthreads=1)
-    t1 = max(time.perf_counter() - t0, 1e-4)
+    # calibrate on one head (once per workload), then size the sample to
+    # about target_s
+    if w.name not in _CALIBRATION:
+        x1 = make_inputs(w, heads=1)
+        t0 = time.perf_counter()
+        oracle.forward(x1["q64"], x1["k64"], x1["v64"], K=w.K, iters=w.iters, W=w.W, alpha=w.alpha, nthreads=1)
+        _CALIBRATION[w.name] = max(time.perf_counter() - t0, 1e-4)
+    t1 = _CALIBRATION[w.name]
     heads = int(max(1, min(w.heads, (target_s / t1) * cores)))
     if max_heads:
         heads = min(heads, max_heads)
@@ -210,33 +228,30 @@ def run_reference(args, w):
     return 0
 
 
-def run_ours(args, w):
+def _to_device(x, w, dev):
     import numpy as np
+    import torch
+    if w.dtype == "f32":
+        conv = lambda a: torch.from_numpy(a).to(dev)
+    else:
+        conv = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    return conv(x["q"]), conv(x["k"]), conv(x["v"])
+
+
+def time_workload(args, w, dev, pg, flush, clocks=None):
+    """Warm up, then time exactly args.steps forwards of workload w (inputs
+    resident in HBM, L2 flushed before every step outside the event pair).
+    Returns the timing record and the device tensors."""
     import torch
     import means_cluster_attention_b200 as ca
     from means_cluster_attention_b200 import _lib
     from means_cluster_attention_b200.inputs import make_inputs
 
-    ws, rank, local = dist_info()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    pg = None
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-        pg = dist
-
     x = make_inputs(w, seed=0)
-    if w.dtype == "f32":
-        conv = lambda a: torch.from_numpy(a).to(dev)
-    else:
-        conv = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
-    q, k, v = conv(x["q"]), conv(x["k"]), conv(x["v"])
+    q, k, v = _to_device(x, w, dev)
     out = torch.empty_like(q)
     assign = torch.empty((w.B, w.H, w.L), dtype=torch.int32, device=dev)
     cent = torch.empty((w.B, w.H, w.K, w.d), dtype=torch.float32, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def step():
         ca.forward(q, k, v, w.K, w.iters, w.W, w.alpha, out=out, assign=assign, centroids=cent)
@@ -248,8 +263,8 @@ def run_ours(args, w):
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    clocks = ClockSampler(local)
-    clocks.start()
+    if clocks:
+        clocks.start()
     dom = args.profile_kernel or DOMINANT.get(w.name, "kmeans_assign")
     if pg:
         pg.barrier()
@@ -266,18 +281,104 @@ def run_ours(args, w):
     kstat = _lib.profile_stop()
     if pg:
         pg.barrier()
-    clk = clocks.stop()
+    clk = clocks.stop() if clocks else None
     ca.sync_status()
     ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms_step = sum(ms) / len(ms)
     k_ms = kstat.total_ms / max(1, kstat.launches)
     ms_step, k_ms = reduce_max([ms_step, k_ms], pg, dev)
+    ws = dist_info()[0]
     value = whole_job_rate(w.tokens, ws, ms_step)
+
+    peak, peak_kind = measured_peak()
+    achieved = (kstat.algorithmic_bytes / max(1, kstat.launches)) / (k_ms / 1e3) / 1e9 if k_ms > 0 else 0.0
+    step_bytes = 4.0 * w.tokens * w.d * w.elem_bytes
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_kind": peak_kind,
+                "traffic": ncu_traffic(dom, w.name),
+                "kernel_ms_per_launch": k_ms, "launches_timed": int(kstat.launches),
+                "alg_bytes_per_launch": kstat.algorithmic_bytes / max(1, kstat.launches),
+                "step_alg_bytes": step_bytes, "step_achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+                "step_frac": step_bytes / (ms_step / 1e3) / 1e9 / peak,
+                "step_frac_of_8tbs": step_bytes / (ms_step / 1e3) / 8e12}
+    rec = {"value": value, "unit": UNIT, "ms_per_step": ms_step, "step_ms_min": min(ms),
+           "step_ms_median": statistics.median(ms), "roofline": roofline, "gpu_launches": int(n_launch),
+           "config": workload_desc(w)}
+    if clk is not None:
+        rec["clocks"] = clk
+    return rec, x, (q, k, v)
+
+
+def parity_check(w, x, dev_inputs, n_heads):
+    """Outside the timed region: one more forward with the per-iteration
+    assignment history, then the fp64 oracle on the first n_heads heads.
+    Reports the flip rate (final assignments that differ from the oracle's),
+    per-iteration mismatches, centroid and output errors; the output error is
+    taken against the oracle evaluated at the GPU's own assignments."""
+    import numpy as np
+    import torch
+    import oracle
+    import means_cluster_attention_b200 as ca
+    from means_cluster_attention_b200.inputs import bf16_bits_to_f64
+
+    q, k, v = dev_inputs
+    B, H, L, d = q.shape
+    hist = torch.full((B, H, max(w.iters, 1), L), -1, dtype=torch.int32, device=q.device)
+    out, assign, cent = ca.forward(q, k, v, w.K, w.iters, w.W, w.alpha, assign_hist=hist, sync_check=True)
+    torch.cuda.synchronize()
+    heads = list(range(min(n_heads, B * H)))
+    flat = lambda a: a.reshape((B * H,) + a.shape[2:])[heads][None]
+    if out.dtype == torch.bfloat16:
+        g_out = bf16_bits_to_f64(out.view(torch.int16).cpu().numpy().view(np.uint16))
+    else:
+        g_out = out.cpu().numpy().astype(np.float64)
+    g_out, g_assign = flat(g_out), flat(assign.cpu().numpy())
+    g_cent = flat(cent.cpu().numpy().astype(np.float64))
+    g_hist = flat(hist.cpu().numpy()[:, :, :w.iters])
+    xs = {n: np.ascontiguousarray(flat(x[n])) for n in ("q64", "k64", "v64")}
+    t0 = time.perf_counter()
+    r_out, r_assign, r_cent, r_hist = oracle.forward(xs["q64"], xs["k64"], xs["v64"], K=w.K, iters=w.iters,
+                                                     W=w.W, alpha=w.alpha, hist=True)
+    at_out, at_cent = oracle.forward_at(xs["q64"], xs["k64"], xs["v64"], g_assign, K=w.K, iters=w.iters,
+                                        W=w.W, alpha=w.alpha)
+    dt = time.perf_counter() - t0
+    tokens = len(heads) * L
+    flips = int((g_assign != r_assign).sum())
+    denom = np.maximum(np.abs(at_cent), 1e-30)
+    return {"heads_checked": len(heads), "of_heads": B * H, "tokens_checked": tokens,
+            "flip_rate": flips / tokens, "final_assignment_flips": flips,
+            "per_iteration_mismatches": int((g_hist != r_hist).sum()) if w.iters else 0,
+            "centroids_bit_exact": bool(np.array_equal(g_cent, at_cent)),
+            "centroid_max_rel_err": float((np.abs(g_cent - at_cent) / denom).max()),
+            "max_abs_err_at_gpu_assign": float(np.abs(g_out - at_out).max()),
+            "max_abs_err_vs_oracle": float(np.abs(g_out - r_out).max()),
+            "tolerance": 2e-3 if w.dtype == "f32" else 2e-2, "oracle_seconds": round(dt, 2)}
+
+
+def run_ours(args, w):
+    import torch
+    import means_cluster_attention_b200 as ca
+    from means_cluster_attention_b200.inputs import WORKLOADS
+
+    ws, rank, local = dist_info()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    clocks = ClockSampler(local)
+    rec, x, dev_inputs = time_workload(args, w, dev, pg, flush, clocks)
+    q = dev_inputs[0]
 
     # End to end through the C ABI with host buffers (pinned), copies included.
     e2e = None
     if not args.no_e2e:
-        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        qh, kh, vh = (t.cpu().pin_memory() for t in dev_inputs)
         oh = torch.empty_like(qh).pin_memory()
         n_e2e = max(3, min(args.steps, 10))
         for _ in range(2):
@@ -295,26 +396,34 @@ def run_ours(args, w):
         e2e = {"value": whole_job_rate(w.tokens, ws, e_step), "unit": UNIT, "h2d_bytes_per_step": 3 * nbytes,
                "d2h_bytes_per_step": nbytes, "ms_per_step": e_step}
 
-    peak, peak_kind = measured_peak()
-    achieved = (kstat.algorithmic_bytes / max(1, kstat.launches)) / (k_ms / 1e3) / 1e9 if k_ms > 0 else 0.0
-    step_bytes = 4.0 * w.tokens * w.d * w.elem_bytes
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "peak_kind": peak_kind,
-                "traffic": ncu_traffic(dom, w.name),
-                "kernel_ms_per_launch": k_ms, "launches_timed": int(kstat.launches),
-                "alg_bytes_per_launch": kstat.algorithmic_bytes / max(1, kstat.launches),
-                "step_alg_bytes": step_bytes, "step_achieved_gbs": step_bytes / (ms_step / 1e3) / 1e9,
-                "step_frac": step_bytes / (ms_step / 1e3) / 1e9 / peak, "step_frac_of_8tbs": step_bytes / (ms_step / 1e3) / 8e12}
+    # The other bf16 workloads the HBM-roofline target is stated on: their own
+    # timed lines (same steps / warm-up), context for the headline.
+    others = {}
+    extra = [n for n in (args.also.split(",") if args.also else []) if n and n != w.name]
+    extra_inputs = {}
+    for name in extra:
+        ow = WORKLOADS[name]
+        orec, ox, odev = time_workload(args, ow, dev, pg, flush)
+        others[name] = orec
+        extra_inputs[name] = (ow, ox, odev)
 
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_desc(w),
-        "roofline": roofline, "e2e": e2e, "gpu_launches": int(n_launch), "clocks": clk,
-        "step_ms_min": min(ms), "step_ms_median": statistics.median(ms),
+        "metric": METRIC, "value": rec["value"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "precision": PRECISION[w.dtype], "data": "synthetic", "config": rec["config"],
+        "roofline": rec["roofline"], "e2e": e2e, "gpu_launches": rec["gpu_launches"], "clocks": rec["clocks"],
+        "step_ms_min": rec["step_ms_min"], "step_ms_median": rec["step_ms_median"],
     }
+    if others:
+        line["other_workloads"] = others
     if pg:
         line["config"]["parallelism"] = f"replicas x{ws} (independent heads, no collective)"
+    if rank == 0 and ws == 1 and not args.no_parity:
+        par = {w.name: parity_check(w, x, dev_inputs, PARITY_HEADS.get(w.name, 8))}
+        for name, (ow, ox, odev) in extra_inputs.items():
+            par[name] = parity_check(ow, ox, odev, PARITY_HEADS.get(name, 8))
+        line["parity"] = par
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rate, cores, sample, _ = cpu_oracle_rate(w, args.cpu_seconds)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
@@ -338,6 +447,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-parity", action="store_true")
+    ap.add_argument("--also", default=DEFAULT_ALSO,
+                    help="comma-separated workloads timed beside the headline ('' for none)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -46,7 +46,16 @@
  *     0 <= alpha <= 1 (finite); B, H, L >= 1; B*H <= 65535; B*H*L*d < 2^31.
  *     Inputs must be finite.
  *   - Results are deterministic: the same inputs give bitwise-identical
- *     outputs on the same GPU.
+ *     outputs on the same GPU, within this envelope.  The general path
+ *     (every fp32 call; bf16 calls with K > 64 or floor(W/2) > 128) runs
+ *     every floating-point reduction in a fixed order (the member sums of
+ *     the centroid update in index order within each 1024-token block, the
+ *     blocks in order), so any finite input is reproducible.  The bf16
+ *     fused and tiled kernels add the member sums with fp64 atomics whose
+ *     order varies, but the sums are
+ *     exact (hence order-free) whenever the non-zero magnitudes of Q lie
+ *     within 2^-27 .. 16; outside that range the last bit of a centroid may
+ *     vary between runs.
  */
 #ifndef CLUSTERATTN_H_
 #define CLUSTERATTN_H_
@@ -158,8 +167,19 @@ ca_status ca_forward_noalloc(const void *q, const void *k, const void *v, int dt
 
 /* Synchronizes stream, then reports (and clears) the first device-side error
  * recorded by a kernel of this library on the current device, or a pending
- * CUDA error.  CA_OK when nothing went wrong. */
+ * CUDA error.  CA_OK when nothing went wrong.  The device-side error word is
+ * one per device, shared by every stream and thread using the library there:
+ * a kernel on another stream can set it, and a caller that reads it clears
+ * it for everyone; callers that need per-stream attribution must serialize
+ * their work and their status checks. */
 ca_status ca_sync_status(void *stream);
+
+/* Test hook: launches one single-thread kernel on stream that records code
+ * (CA_ERR_TIMEOUT or CA_ERR_DEVICE) in the device-side error word exactly as
+ * a kernel that detected a problem would, without faulting; the next
+ * ca_sync_status then returns that code once.  Any other code returns
+ * CA_ERR_INVALID_ARG and launches nothing.  Not part of the forward pass. */
+ca_status ca_debug_record_error(int code, void *stream);
 
 /* Static description of a status code. */
 const char *ca_status_string(ca_status s);

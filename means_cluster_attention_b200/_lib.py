@@ -28,6 +28,7 @@ SIGNATURES = {
     "ca_forward_ex": ([_vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp, _vp, _vp], _ci),
     "ca_forward_noalloc": ([_vp, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp], _ci),
     "ca_sync_status": ([_vp], _ci),
+    "ca_debug_record_error": ([_ci, _vp], _ci),
     "ca_status_string": ([_ci], ctypes.c_char_p),
     "ca_last_error": ([], ctypes.c_char_p),
     "ca_version": ([], ctypes.c_char_p),

@@ -117,6 +117,33 @@ struct Scratch {
     }
 };
 
+// Every kernel that takes dynamic shared memory may use up to 227 KB of it.
+// The attribute is per device and per function; it is set once per device,
+// under a lock, before the first launch there.
+ca_status ensure_kernel_attributes() {
+    using namespace ca;
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    CA_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(CA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> g(mu);
+    if (done[dev]) return CA_OK;
+    const int big = 227 * 1024;
+    CA_CUDA(cudaFuncSetAttribute(fused::fused_forward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(centroid_attn_partial_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(centroid_attn_partial_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(window_blend_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(window_blend_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    done[dev] = true;
+    return CA_OK;
+}
+
 // The fused one-CTA-per-head kernel handles bf16 heads with L <= 512,
 // K <= 64 and a window radius floor(W/2) <= 16.
 bool fused_eligible(int dtype, const Problem &p) {
@@ -127,13 +154,6 @@ ca_status run_fused(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
                     __nv_bfloat16 *out, int32_t *assign_out, float *cent_out, int32_t *hist, cudaStream_t st) {
     using namespace ca;
     const fused::Layout lay(p.L, p.K, p.W / 2);
-    static bool attr_set[64] = {};
-    int dev = 0;
-    CA_CUDA(cudaGetDevice(&dev));
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        CA_CUDA(cudaFuncSetAttribute(fused::fused_forward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-        attr_set[dev] = true;
-    }
     fused::Params P;
     P.q = q;
     P.k = k;
@@ -190,15 +210,6 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     CA_CUDA(s.get((void **)&vcent, sizeof(float) * NH * K * kD));
     if (!assign) CA_CUDA(s.get((void **)&assign, sizeof(int32_t) * NH * L));
 
-    static bool attr_set[64] = {};
-    int dev = 0;
-    CA_CUDA(cudaGetDevice(&dev));
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-        CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-        CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-        attr_set[dev] = true;
-    }
     const double head_bytes = (double)NH * L * kD * sizeof(__nv_bfloat16);
 
     tiled::MuParams mp{};
@@ -326,11 +337,13 @@ ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *o
     double *sums = nullptr;
     int32_t *counts = nullptr, *assign = assign_out;
     const int n_chunks = (L + kCaChunk - 1) / kCaChunk;
+    const int tokens_per_cta = 1024;
+    const int n_cta = (L + tokens_per_cta - 1) / tokens_per_cta;
     CA_CUDA(s.get((void **)&mu, sizeof(float) * NH * K * kD));
     CA_CUDA(s.get((void **)&vcent, sizeof(float) * NH * K * kD));
     CA_CUDA(s.get((void **)&part, sizeof(float) * NH * n_chunks * K * (kD + 2)));
-    CA_CUDA(s.get((void **)&sums, sizeof(double) * NH * K * kD));
-    CA_CUDA(s.get((void **)&counts, sizeof(int32_t) * NH * K));
+    CA_CUDA(s.get((void **)&sums, sizeof(double) * NH * n_cta * K * kD));
+    CA_CUDA(s.get((void **)&counts, sizeof(int32_t) * NH * n_cta * K));
     if (!assign) CA_CUDA(s.get((void **)&assign, sizeof(int32_t) * NH * L));
 
     const double esz = (double)sizeof(T);
@@ -347,14 +360,10 @@ ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *o
         CA_CUDA(cudaMemsetAsync(assign, 0, sizeof(int32_t) * NH * L, st));
         if (cent_out) CA_CUDA(cudaMemcpyAsync(cent_out, mu, sizeof(float) * NH * K * kD, cudaMemcpyDeviceToDevice, st));
     }
-    CA_CUDA(cudaMemsetAsync(sums, 0, sizeof(double) * NH * K * kD, st));
-    CA_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * NH * K, st));
 
-    // 2. Lloyd iterations
-    const int tokens_per_cta = 1024;
-    const size_t asmem = AssignSmem::bytes(K);
-    CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asmem));
-    const dim3 agrid((L + tokens_per_cta - 1) / tokens_per_cta, (unsigned)NH);
+    // 2. Lloyd iterations (every CTA writes all K rows of its partial-sum slot)
+    const size_t asmem = AssignSmem::bytes(K, tokens_per_cta);
+    const dim3 agrid(n_cta, (unsigned)NH);
     for (int t = 0; t < p.iters; ++t) {
         int32_t *hist_t = hist ? hist + (int64_t)t * L : nullptr;
         {
@@ -366,7 +375,7 @@ ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *o
         CA_CUDA(cudaGetLastError());
         {
             Launch pl("kmeans_update", st, 0.0);
-            kmeans_update_kernel<<<(unsigned)NH, 256, 0, st>>>(K, sums, counts, mu,
+            kmeans_update_kernel<<<(unsigned)NH, 256, 0, st>>>(K, n_cta, sums, counts, mu,
                                                                 t == p.iters - 1 ? cent_out : nullptr,
                                                                 xo.empty_keep);
             pl.after();
@@ -376,7 +385,6 @@ ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *o
 
     // 3. centroid attention
     const size_t csmem = centroid_attn_smem_bytes(K);
-    CA_CUDA(cudaFuncSetAttribute(centroid_attn_partial_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem));
     {
         Launch pl("centroid_attn", st, 2.0 * head_bytes);
         centroid_attn_partial_kernel<T><<<dim3(n_chunks, (unsigned)NH), kCaThreads, csmem, st>>>(
@@ -393,7 +401,6 @@ ca_status run_forward(const T *q, const T *k, const T *v, const Problem &p, T *o
 
     // 4-6. gather + window attention + blend
     const size_t wsmem = window_smem_bytes();
-    CA_CUDA(cudaFuncSetAttribute(window_blend_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem));
     {
         Launch pl("window_blend", st, 4.0 * head_bytes);
         Variant wv = xo.var;
@@ -410,8 +417,11 @@ ca_status dispatch(const void *q, const void *k, const void *v, int dtype, const
                    void *out, int32_t *assign_out, float *cent_out, int32_t *hist, void *stream) {
     ca_status s = validate(q, k, v, out, p);
     if (s != CA_OK) return s;
+    if (dtype != 0 && dtype != 1) return fail(CA_ERR_INVALID_ARG, "dtype must be 0 (fp32) or 1 (bf16), got %d", dtype);
     if (((uintptr_t)cent_out & 15u) || ((uintptr_t)assign_out & 3u) || ((uintptr_t)hist & 3u))
         return fail(CA_ERR_INVALID_ARG, "centroids_out must be 16-byte aligned, assign buffers 4-byte aligned");
+    s = ensure_kernel_attributes();
+    if (s != CA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
     if (fused_eligible(dtype, p))
         return run_fused((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, p,
@@ -482,6 +492,9 @@ ca_status ca_forward_ex(const void *q, const void *k, const void *v, int dtype, 
     ex.var.key_valid = o.key_valid;
     ex.var.local = o.window_mode ? (W > 0 && W < L) : 1;
     ex.var.soft = o.gather_mode;
+    if (dtype != 0 && dtype != 1) return fail(CA_ERR_INVALID_ARG, "dtype must be 0 (fp32) or 1 (bf16), got %d", dtype);
+    s = ensure_kernel_attributes();
+    if (s != CA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
     if (dtype == 0)
         return run_forward<float>((const float *)q, (const float *)k, (const float *)v, p, (float *)out,
@@ -545,10 +558,22 @@ ca_status ca_forward_host(const void *q, const void *k, const void *v, int dtype
     } ev_guard{ev, n_ev};
     void *dq = nullptr, *dk = nullptr, *dv = nullptr, *dout = nullptr, *dcent = nullptr;
     int32_t *dassign = nullptr;
+    // A failure part-way stops queueing work but still lets the streams
+    // drain: copies already queued into or out of the caller's host buffers
+    // must be finished before this call returns, error or not.
+    ca_status status = CA_OK;
+#define CA_STEP(call)                                                          \
+    {                                                                          \
+        cudaError_t e_ = (call);                                               \
+        if (e_ != cudaSuccess) {                                               \
+            status = cuda_fail(e_, #call);                                     \
+            break;                                                             \
+        }                                                                      \
+    }
     {
         Scratch sc(st);
-        // Before the scratch is released on st (or on any early return),
-        // st waits for everything queued on the other two streams.
+        // Before the scratch is released on st (or on an early exit), st
+        // waits for everything queued on the other two streams.
         struct Join {
             cudaStream_t st, a, b;
             cudaEvent_t ea, eb;
@@ -561,42 +586,66 @@ ca_status ca_forward_host(const void *q, const void *k, const void *v, int dtype
                 cudaStreamWaitEvent(st, eb, 0);
             }
         } join{st, s_comp, s_back, n_ev ? ev[n_ev - 2] : nullptr, n_ev ? ev[n_ev - 1] : nullptr, n_chunks > 1};
-        CA_CUDA(sc.get(&dq, n * esz));
-        CA_CUDA(sc.get(&dk, n * esz));
-        CA_CUDA(sc.get(&dv, n * esz));
-        CA_CUDA(sc.get(&dout, n * esz));
-        if (assign_out) CA_CUDA(sc.get((void **)&dassign, sizeof(int32_t) * NH * p.L));
-        if (centroids_out) CA_CUDA(sc.get(&dcent, sizeof(float) * NH * p.K * p.d));
-        for (int c = 0; c < n_chunks; ++c) {
+        do {
+            CA_STEP(sc.get(&dq, n * esz));
+            CA_STEP(sc.get(&dk, n * esz));
+            CA_STEP(sc.get(&dv, n * esz));
+            CA_STEP(sc.get(&dout, n * esz));
+            if (assign_out) CA_STEP(sc.get((void **)&dassign, sizeof(int32_t) * NH * p.L));
+            if (centroids_out) CA_STEP(sc.get(&dcent, sizeof(float) * NH * p.K * p.d));
+        } while (0);
+        for (int c = 0; status == CA_OK && c < n_chunks; ++c) {
             const int64_t h0 = c * NH / n_chunks, h1 = (c + 1) * NH / n_chunks;
             const size_t off = (size_t)h0 * head_elems * esz, bytes = (size_t)(h1 - h0) * head_elems * esz;
-            CA_CUDA(cudaMemcpyAsync((char *)dq + off, (const char *)q + off, bytes, cudaMemcpyHostToDevice, st));
-            CA_CUDA(cudaMemcpyAsync((char *)dk + off, (const char *)k + off, bytes, cudaMemcpyHostToDevice, st));
-            CA_CUDA(cudaMemcpyAsync((char *)dv + off, (const char *)v + off, bytes, cudaMemcpyHostToDevice, st));
+            CA_STEP(cudaMemcpyAsync((char *)dq + off, (const char *)q + off, bytes, cudaMemcpyHostToDevice, st));
+            CA_STEP(cudaMemcpyAsync((char *)dk + off, (const char *)k + off, bytes, cudaMemcpyHostToDevice, st));
+            CA_STEP(cudaMemcpyAsync((char *)dv + off, (const char *)v + off, bytes, cudaMemcpyHostToDevice, st));
             if (n_chunks > 1) {
-                CA_CUDA(cudaEventRecord(ev[2 * c], st));
-                CA_CUDA(cudaStreamWaitEvent(s_comp, ev[2 * c], 0));
+                CA_STEP(cudaEventRecord(ev[2 * c], st));
+                CA_STEP(cudaStreamWaitEvent(s_comp, ev[2 * c], 0));
             }
             const Problem pc{1, (int)(h1 - h0), p.L, p.d, p.K, p.iters, p.W, p.alpha};
             int32_t *da = dassign ? dassign + h0 * p.L : nullptr;
             float *dc = dcent ? (float *)dcent + h0 * p.K * p.d : nullptr;
             s = dispatch((char *)dq + off, (char *)dk + off, (char *)dv + off, dtype, pc, (char *)dout + off, da, dc,
                          nullptr, s_comp);
-            if (s != CA_OK) return s;
-            if (n_chunks > 1) {
-                CA_CUDA(cudaEventRecord(ev[2 * c + 1], s_comp));
-                CA_CUDA(cudaStreamWaitEvent(s_back, ev[2 * c + 1], 0));
+            if (s != CA_OK) {
+                status = s;
+                break;
             }
-            CA_CUDA(cudaMemcpyAsync((char *)out + off, (char *)dout + off, bytes, cudaMemcpyDeviceToHost, s_back));
+            if (n_chunks > 1) {
+                CA_STEP(cudaEventRecord(ev[2 * c + 1], s_comp));
+                CA_STEP(cudaStreamWaitEvent(s_back, ev[2 * c + 1], 0));
+            }
+            CA_STEP(cudaMemcpyAsync((char *)out + off, (char *)dout + off, bytes, cudaMemcpyDeviceToHost, s_back));
             if (assign_out)
-                CA_CUDA(cudaMemcpyAsync(assign_out + h0 * p.L, da, sizeof(int32_t) * (h1 - h0) * p.L,
+                CA_STEP(cudaMemcpyAsync(assign_out + h0 * p.L, da, sizeof(int32_t) * (h1 - h0) * p.L,
                                         cudaMemcpyDeviceToHost, s_back));
             if (centroids_out)
-                CA_CUDA(cudaMemcpyAsync(centroids_out + h0 * p.K * p.d, dc, sizeof(float) * (h1 - h0) * p.K * p.d,
+                CA_STEP(cudaMemcpyAsync(centroids_out + h0 * p.K * p.d, dc, sizeof(float) * (h1 - h0) * p.K * p.d,
                                         cudaMemcpyDeviceToHost, s_back));
         }
     }
-    CA_CUDA(cudaStreamSynchronize(st));
+#undef CA_STEP
+    const std::string detail = status == CA_OK ? std::string() : g_last_error;
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (status != CA_OK) {
+        g_last_error = detail;
+        return status;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    return CA_OK;
+}
+
+ca_status ca_debug_record_error(int code, void *stream) {
+    if (code != CA_ERR_TIMEOUT && code != CA_ERR_DEVICE)
+        return fail(CA_ERR_INVALID_ARG, "code must be CA_ERR_TIMEOUT or CA_ERR_DEVICE (got %d)", code);
+    {
+        ca::Launch pl("debug_record_error", (cudaStream_t)stream, 0.0);
+        ca::debug_record_error_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(code);
+        pl.after();
+    }
+    CA_CUDA(cudaGetLastError());
     return CA_OK;
 }
 
@@ -722,13 +771,15 @@ ca_status run_forward_noalloc(const T *q, const T *k, const T *v, const Problem 
     const int L = p.L, K = p.K;
     const float scale = 1.0f / sqrtf((float)p.d);
     const int n_chunks = (L + kCaChunk - 1) / kCaChunk;
+    const int tokens_per_cta = 1024;
+    const int n_cta = (L + tokens_per_cta - 1) / tokens_per_cta;
 
     // Carve the working buffers out of the fixed array.
     const size_t b_mu = align256(sizeof(float) * NH * K * kD);
     const size_t b_vc = b_mu;
     const size_t b_part = align256(sizeof(float) * NH * n_chunks * K * (kD + 2));
-    const size_t b_sums = align256(sizeof(double) * NH * K * kD);
-    const size_t b_cnt = align256(sizeof(int32_t) * NH * K);
+    const size_t b_sums = align256(sizeof(double) * NH * n_cta * K * kD);
+    const size_t b_cnt = align256(sizeof(int32_t) * NH * n_cta * K);
     const size_t b_asg = assign_out ? 0 : align256(sizeof(int32_t) * NH * L);
     const size_t need = b_mu + b_vc + b_part + b_sums + b_cnt + b_asg;
     if (need > kNoAllocScratchBytes)
@@ -757,14 +808,11 @@ ca_status run_forward_noalloc(const T *q, const T *k, const T *v, const Problem 
         CA_CUDA(cudaMemsetAsync(assign, 0, sizeof(int32_t) * NH * L, st));
         if (cent_out) CA_CUDA(cudaMemcpyAsync(cent_out, mu, sizeof(float) * NH * K * kD, cudaMemcpyDeviceToDevice, st));
     }
-    // The array keeps the last call's contents: clear the running sums.
-    CA_CUDA(cudaMemsetAsync(sums, 0, sizeof(double) * NH * K * kD, st));
-    CA_CUDA(cudaMemsetAsync(counts, 0, sizeof(int32_t) * NH * K, st));
-
-    const int tokens_per_cta = 1024;
-    const size_t asmem = AssignSmem::bytes(K);
-    CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asmem));
-    const dim3 agrid((L + tokens_per_cta - 1) / tokens_per_cta, (unsigned)NH);
+    // The array keeps the last call's contents; nothing in it needs clearing:
+    // every assignment launch writes all K rows of every partial-sum slot
+    // before the update reads them.
+    const size_t asmem = AssignSmem::bytes(K, tokens_per_cta);
+    const dim3 agrid(n_cta, (unsigned)NH);
     for (int t = 0; t < p.iters; ++t) {
         {
             Launch pl("kmeans_assign", st, head_bytes);
@@ -775,14 +823,13 @@ ca_status run_forward_noalloc(const T *q, const T *k, const T *v, const Problem 
         CA_CUDA(cudaGetLastError());
         {
             Launch pl("kmeans_update", st, 0.0);
-            kmeans_update_kernel<<<(unsigned)NH, 256, 0, st>>>(K, sums, counts, mu,
+            kmeans_update_kernel<<<(unsigned)NH, 256, 0, st>>>(K, n_cta, sums, counts, mu,
                                                                 t == p.iters - 1 ? cent_out : nullptr);
             pl.after();
         }
         CA_CUDA(cudaGetLastError());
     }
     const size_t csmem = centroid_attn_smem_bytes(K);
-    CA_CUDA(cudaFuncSetAttribute(centroid_attn_partial_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem));
     {
         Launch pl("centroid_attn", st, 2.0 * head_bytes);
         centroid_attn_partial_kernel<T><<<dim3(n_chunks, (unsigned)NH), kCaThreads, csmem, st>>>(
@@ -797,7 +844,6 @@ ca_status run_forward_noalloc(const T *q, const T *k, const T *v, const Problem 
     }
     CA_CUDA(cudaGetLastError());
     const size_t wsmem = window_smem_bytes();
-    CA_CUDA(cudaFuncSetAttribute(window_blend_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem));
     {
         Launch pl("window_blend", st, 4.0 * head_bytes);
         window_blend_kernel<T><<<dim3((L + kWinQ - 1) / kWinQ, (unsigned)NH), kWinThreads, wsmem, st>>>(
@@ -819,6 +865,9 @@ extern "C" ca_status ca_forward_noalloc(const void *q, const void *k, const void
     if (s != CA_OK) return s;
     if (((uintptr_t)centroids_out & 15u) || ((uintptr_t)assign_out & 3u))
         return fail(CA_ERR_INVALID_ARG, "centroids_out must be 16-byte aligned, assign_out 4-byte aligned");
+    if (dtype != 0 && dtype != 1) return fail(CA_ERR_INVALID_ARG, "dtype must be 0 (fp32) or 1 (bf16), got %d", dtype);
+    s = ensure_kernel_attributes();
+    if (s != CA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
     if (dtype == 0)
         return run_forward_noalloc<float>((const float *)q, (const float *)k, (const float *)v, p, (float *)out,

@@ -36,6 +36,10 @@ __device__ __forceinline__ void record_error(int code, int where) {
     if (atomicCAS(&g_dev_error, 0, code) == 0) g_dev_error_where = where;
 }
 
+// Records code the way a kernel that detected a problem does (site 99), for
+// testing the host's error reporting without a fault.
+__global__ void debug_record_error_kernel(int code) { record_error(code, 99); }
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 

@@ -18,10 +18,16 @@
 //     e_j); otherwise every such candidate is re-measured in fp64 in the
 //     expanded form with index-order sums and separately rounded products
 //     and sums, and the lowest k with the smallest value wins.
-// Member sums of bf16 (or fp32) queries are exact in fp64 for every input
-// whose non-zero magnitudes stay within 2^-27 .. 16 (bf16, L <= 32768), so
-// the order of the additions (shared and global atomics here) does not
-// change any bit of the result.
+// Member sums are taken in a fixed order, with no floating-point atomics:
+// each CTA walks its token range in index order (thread j of a group of 64
+// owns coordinate j of the clusters k = group (mod 4)) and writes its partial
+// sums to its own slot; the update adds the CTA slots in CTA order.  The
+// result is therefore bitwise reproducible for any input.  When a head fits
+// one CTA (L <= 1024) the order is the oracle's index order, so the sums are
+// bit-identical to it for any fp32 or bf16 input; across CTAs they equal it
+// whenever the sums are exact in fp64, which holds for bf16 inputs whose
+// non-zero magnitudes lie within 2^-27 .. 16 (L <= 32768), and otherwise
+// differ by fp64 rounding only.
 #pragma once
 
 #include "common.cuh"
@@ -71,24 +77,26 @@ __device__ __forceinline__ double dot64_f64_ordered(const float (&x)[kD], const 
 
 // Shared-memory layout of the assignment kernel for K clusters.
 struct AssignSmem {
-    static __host__ __device__ size_t bytes(int K) {
+    static __host__ __device__ size_t bytes(int K, int tokens_per_cta) {
         return (size_t)K * kD * sizeof(double)    // member sums
                + (size_t)K * kD * sizeof(float)   // centroids
                + (size_t)K * sizeof(double)       // |mu_k|^2 in fp64, index order
                + (size_t)K * 2 * sizeof(float)    // |mu_k|^2 and |mu_k| in fp32
-               + (size_t)K * sizeof(int);         // member counts
+               + (size_t)K * sizeof(int)          // member counts
+               + (size_t)tokens_per_cta;          // the CTA's assignments
     }
 };
 
 // One Lloyd iteration's assignment step plus the per-CTA member sums.
 // Grid (ceil(L / tokens_per_cta), heads).  Writes c_i to assign (and to hist
-// when non-null) and adds exact member sums / counts into sums / counts.
+// when non-null) and the CTA's member sums / counts to its own slot of
+// part_sum [heads][ctas][K][64] / part_cnt [heads][ctas][K].
 template <typename T>
 __global__ void __launch_bounds__(kAssignThreads)
     kmeans_assign_kernel(const T *__restrict__ q, int L, int K, int tokens_per_cta,
                          const float *__restrict__ mu, int32_t *__restrict__ assign,
                          int32_t *__restrict__ hist, int64_t hist_head_stride,
-                         double *__restrict__ sums, int32_t *__restrict__ counts) {
+                         double *__restrict__ part_sum, int32_t *__restrict__ part_cnt) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     double *sum_s = reinterpret_cast<double *>(smem_raw);
     float *mu_s = reinterpret_cast<float *>(sum_s + (size_t)K * kD);
@@ -96,6 +104,7 @@ __global__ void __launch_bounds__(kAssignThreads)
     float *mm32_s = reinterpret_cast<float *>(mm64_s + K);
     float *mun_s = mm32_s + K;
     int *cnt_s = reinterpret_cast<int *>(mun_s + K);
+    uint8_t *c_s = reinterpret_cast<uint8_t *>(cnt_s + K);  // [tokens_per_cta]
 
     const int h = blockIdx.y;
     const int t0 = blockIdx.x * tokens_per_cta;
@@ -176,46 +185,51 @@ __global__ void __launch_bounds__(kAssignThreads)
             }
             assign[(int64_t)h * L + i] = best;
             if (hist) hist[(int64_t)h * hist_head_stride + i] = best;
+            c_s[i - t0] = (uint8_t)best;
             atomicAdd(&cnt_s[best], 1);
-        }
-        // Member sums: the warp walks its tokens one at a time, each lane
-        // adding two coordinates (exact fp64 additions).
-        const int n_here = min(32, t1 - base);
-        for (int tt = 0; tt < n_here; ++tt) {
-            const int c = __shfl_sync(0xffffffffu, best, tt);
-            const T *row = qh + (int64_t)(base + tt) * kD;
-            atomicAdd(&sum_s[(size_t)c * kD + lane], (double)to_f32(row[lane]));
-            atomicAdd(&sum_s[(size_t)c * kD + lane + 32], (double)to_f32(row[lane + 32]));
         }
     }
     __syncthreads();
-    double *sums_h = sums + (int64_t)h * K * kD;
-    for (int idx = threadIdx.x; idx < K * kD; idx += blockDim.x)
-        if (cnt_s[idx / kD] > 0) atomicAdd(&sums_h[idx], sum_s[idx]);
-    for (int k = threadIdx.x; k < K; k += blockDim.x)
-        if (cnt_s[k] > 0) atomicAdd(&counts[(int64_t)h * K + k], cnt_s[k]);
+    // Member sums in index order: thread (grp, j) adds coordinate j of every
+    // token of a cluster k = grp (mod 4), so each sum has one owner and a
+    // fixed order of additions.
+    {
+        const int grp = threadIdx.x >> 6, j = threadIdx.x & 63;
+        for (int i = t0; i < t1; ++i) {
+            const int c = c_s[i - t0];
+            if ((c & 3) == grp)
+                sum_s[(size_t)c * kD + j] = __dadd_rn(sum_s[(size_t)c * kD + j], (double)to_f32(qh[(int64_t)i * kD + j]));
+        }
+    }
+    __syncthreads();
+    const int64_t slot = (int64_t)h * gridDim.x + blockIdx.x;
+    for (int idx = threadIdx.x; idx < K * kD; idx += blockDim.x) part_sum[slot * K * kD + idx] = sum_s[idx];
+    for (int k = threadIdx.x; k < K; k += blockDim.x) part_cnt[slot * K + k] = cnt_s[k];
 }
 
 // mu_k = fp32(sum_k / max(1, count_k)) (an empty cluster keeps its previous
-// centroid when empty_keep); then clears sums / counts for the next
-// iteration.  One block per head.
-__global__ void kmeans_update_kernel(int K, double *__restrict__ sums, int32_t *__restrict__ counts,
-                                     float *__restrict__ mu, float *__restrict__ cent_out,
-                                     int empty_keep = 0) {
+// centroid when empty_keep), the CTA slots of the member sums added in CTA
+// order.  One block per head.
+__global__ void kmeans_update_kernel(int K, int n_cta, const double *__restrict__ part_sum,
+                                     const int32_t *__restrict__ part_cnt, float *__restrict__ mu,
+                                     float *__restrict__ cent_out, int empty_keep = 0) {
     const int64_t h = blockIdx.x;
-    double *s = sums + h * K * kD;
-    int32_t *cn = counts + h * K;
+    const double *ps = part_sum + h * n_cta * K * kD;
+    const int32_t *pc = part_cnt + h * n_cta * K;
     float *m = mu + h * K * kD;
     for (int idx = threadIdx.x; idx < K * kD; idx += blockDim.x) {
-        const int c = cn[idx / kD];
-        const double v = s[idx] / (double)(c > 1 ? c : 1);
+        const int k = idx / kD;
+        double s = 0.0;
+        int c = 0;
+        for (int b = 0; b < n_cta; ++b) {
+            s = __dadd_rn(s, ps[(int64_t)b * K * kD + idx]);
+            c += pc[(int64_t)b * K + k];
+        }
+        const double v = s / (double)(c > 1 ? c : 1);
         const float f = (empty_keep && c == 0) ? m[idx] : __double2float_rn(v);
         m[idx] = f;
         if (cent_out) cent_out[h * K * kD + idx] = f;
     }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < K * kD; idx += blockDim.x) s[idx] = 0.0;
-    for (int k = threadIdx.x; k < K; k += blockDim.x) cn[k] = 0;
 }
 
 }  // namespace ca

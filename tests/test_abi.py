@@ -133,3 +133,10 @@ def test_source_hash_ignores_comments_but_not_code():
     assert build._code_only(base) == build._code_only(commented)
     assert build._code_only(base) != build._code_only(changed)
     assert re.fullmatch(r"[0-9a-f]{16}", build.source_hash("fused_forward"))
+
+
+def test_debug_error_hook_validates_code_on_host(lib):
+    # only CA_ERR_TIMEOUT (4) and CA_ERR_DEVICE (5) may be recorded; anything
+    # else is rejected before a launch, so this needs no GPU
+    for bad in (0, 1, 2, 3, 6, -1):
+        assert lib.ca_debug_record_error(bad, None) == 1

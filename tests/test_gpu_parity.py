@@ -9,8 +9,10 @@ same seeded inputs, for the five workloads.
 * Centroids: bit-exact (fp32).
 * Outputs: max abs error against the oracle evaluated at the GPU's own
   assignments, 2e-3 for fp32 inputs and 2e-2 for bf16 inputs.
-The long-sequence workload is checked on sampled heads (full oracle chain per
-head) plus properties over every head.
+The long-sequence workload (forced ties and empty clusters) is checked on
+every one of its 16 heads against the full oracle chain, plus properties that
+hold for any head (centroid = exact mean of the GPU's own clusters, odd
+strided centroids empty after the first iteration).
 """
 
 import numpy as np
@@ -48,7 +50,7 @@ def test_workload_full_parity(name):
     print(f"{name}: max abs err {err:.3e}")
 
 
-def test_long_sequence_sampled_heads_and_properties():
+def test_long_sequence_every_head_and_properties():
     w = WORKLOADS["l32k_dup_bf16"]
     x = make_inputs(w)
     g = run_gpu(x, w.dtype, w.K, w.iters, w.W, w.alpha, hist=True)
@@ -68,8 +70,9 @@ def test_long_sequence_sampled_heads_and_properties():
         # Duplicated starting centroids: every odd cluster ties with the one
         # below it and loses, so it is empty after the first iteration.
         assert not np.isin(hist0[h], np.arange(1, w.K, 2)).any()
-    # Full oracle chain on sampled heads.
-    for heads in ([0, 7], [15]):
+    # Full oracle chain on every head, four heads per oracle call.
+    for h0 in range(0, B * H, 4):
+        heads = list(range(h0, min(B * H, h0 + 4)))
         xs = select_heads(x, heads)
         gs = {key: g[key].reshape((B * H,) + g[key].shape[2:])[heads][None] for key in ("out", "assign", "cent", "hist")}
         _check(w, xs, gs, heads_note=f" heads {heads}")

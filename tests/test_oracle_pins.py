@@ -427,3 +427,27 @@ def test_ex_grouped_kv_heads():
     ref, ref_a, ref_c, _ = oracle.forward(q, kr, vr, K=4, iters=2, W=6, alpha=0.5)
     np.testing.assert_array_equal(out, ref)
     np.testing.assert_array_equal(assign, ref_a)
+
+
+@pytest.mark.parametrize("name", ["card_gmm_f32", "l4k_gmm_bf16"])
+def test_fp32_stored_centroids_decide_like_plain_fp64(name):
+    """Reading of the precision of the decision: the oracle stores each
+    centroid rounded once to fp32 (as the module of "Hooshaai/svd-sst2-
+    roberta-cluster" section 5 casts its centroids to float before measuring
+    distances).  On the well-separated Gaussian-mixture workloads, where the
+    assignments must match bit for bit, that rounding must not change a single
+    assignment at any Lloyd iteration compared with the pages' plain fp64
+    formulas (Mathematical Formulation section 1 of "Hooshaai/distilbert-
+    sst2-cluster-attention"), so bit-exactness there rests on the pages and
+    not on this reading."""
+    from means_cluster_attention_b200.inputs import WORKLOADS, make_inputs
+    w = WORKLOADS[name]
+    x = make_inputs(w)
+    a32 = oracle.forward(x["q64"], x["k64"], x["v64"], K=w.K, iters=w.iters, W=w.W, alpha=w.alpha,
+                         mu_f32=True, hist=True)
+    a64 = oracle.forward(x["q64"], x["k64"], x["v64"], K=w.K, iters=w.iters, W=w.W, alpha=w.alpha,
+                         mu_f32=False, hist=True)
+    np.testing.assert_array_equal(a32[3], a64[3])
+    np.testing.assert_array_equal(a32[1], a64[1])
+    # the stored centroids differ from the fp64 ones only by that one rounding
+    np.testing.assert_allclose(a32[2], a64[2], rtol=2 ** -24, atol=0)
