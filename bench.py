@@ -35,9 +35,10 @@ DEFAULT_WORKLOAD = "l32k_dup_bf16"
 # Timed beside the headline: the other workloads the roofline target is stated on.
 DEFAULT_ALSO = "l4k_gmm_bf16,l512_bf16"
 FALLBACK_HBM_GBS = 6650.0
-# Heads of each workload the parity block re-checks against the fp64 oracle.
-PARITY_HEADS = {"small_f32": 24, "card_gmm_f32": 48, "l512_bf16": 64, "l4k_gmm_bf16": 12,
-                "l32k_dup_bf16": 8}
+# Heads of each workload the parity block re-checks against the fp64 oracle
+# (every head: the oracle needs about a second per 32k-token head per thread).
+PARITY_HEADS = {"small_f32": 24, "card_gmm_f32": 384, "l512_bf16": 768, "l4k_gmm_bf16": 96,
+                "l32k_dup_bf16": 16}
 PRECISION = {
     "bf16": ("bf16 Q/K/V and O in HBM; bf16 tensor-core operands with fp32 accumulation; "
              "k-means decisions exact on fp32 centroids (certified filter + fp64 re-measure, exact fp64 "

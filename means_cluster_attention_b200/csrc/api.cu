@@ -1,5 +1,7 @@
 // libclusterattn host layer: argument validation, stream-ordered scratch,
 // kernel launches.  The C ABI is declared in include/clusterattn.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -131,7 +133,9 @@ ca_status ensure_kernel_attributes() {
     if (done[dev]) return CA_OK;
     const int big = 227 * 1024;
     CA_CUDA(cudaFuncSetAttribute(fused::fused_forward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
@@ -178,6 +182,36 @@ ca_status run_fused(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     return CA_OK;
 }
 
+// TMA tensor map of a [NH, L, 64] bf16 tensor read in boxes of 256 rows of
+// one head, 128-byte swizzled (the layout the tcgen05 operand descriptors
+// read).  Rows past L (inside a box) are filled with zeros by the TMA unit.
+// The driver's encoder is looked up once through the runtime.
+ca_status encode_rows_map(CUtensorMap *map, const void *base, int64_t NH, int L) {
+    static std::mutex mu;
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    {
+        std::lock_guard<std::mutex> g(mu);
+        if (!encode) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+            cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
+            if (!fn || q != cudaDriverEntryPointSuccess)
+                return fail(CA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+            encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)ca::kD, (cuuint64_t)L, (cuuint64_t)NH};
+    const cuuint64_t strides[2] = {(cuuint64_t)ca::kD * 2u, (cuuint64_t)L * ca::kD * 2u};
+    const cuuint32_t box[3] = {(cuuint32_t)ca::kD, 256u, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(CA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return CA_OK;
+}
+
 // The tiled bf16 path serves the heads the fused kernel does not take, for
 // K <= 64 and a window radius floor(W/2) <= 128.
 bool tiled_eligible(int dtype, const Problem &p) {
@@ -197,9 +231,13 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     __nv_bfloat16 *hi = nullptr, *lo = nullptr;
     uint32_t *hash = nullptr;
     double *psum = nullptr;
-    int *pcnt = nullptr;
+    int *pcnt = nullptr, *done = nullptr;
+    float *mstat = nullptr, *qnorm = nullptr;
     int32_t *assign = assign_out;
     CA_CUDA(s.get((void **)&mu, sizeof(float) * NH * Kp * kD));
+    CA_CUDA(s.get((void **)&mstat, sizeof(float) * NH * 2));
+    CA_CUDA(s.get((void **)&done, sizeof(int) * NH));
+    CA_CUDA(s.get((void **)&qnorm, sizeof(float) * NH * L));
     CA_CUDA(s.get((void **)&hi, sizeof(__nv_bfloat16) * NH * Kp * kD));
     CA_CUDA(s.get((void **)&lo, sizeof(__nv_bfloat16) * NH * Kp * kD));
     CA_CUDA(s.get((void **)&mm, sizeof(float) * NH * Kp));
@@ -209,6 +247,12 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     CA_CUDA(s.get((void **)&cpart, sizeof(float) * NH * n_chunks * K * (kD + 2)));
     CA_CUDA(s.get((void **)&vcent, sizeof(float) * NH * K * kD));
     if (!assign) CA_CUDA(s.get((void **)&assign, sizeof(int32_t) * NH * L));
+    CA_CUDA(cudaMemsetAsync(done, 0, sizeof(int) * NH, st));
+    CUtensorMap qmap;
+    {
+        ca_status ms = encode_rows_map(&qmap, q, NH, L);
+        if (ms != CA_OK) return ms;
+    }
 
     const double head_bytes = (double)NH * L * kD * sizeof(__nv_bfloat16);
 
@@ -221,6 +265,8 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     mp.lo = lo;
     mp.mm = mm;
     mp.hash = hash;
+    mp.mstat = mstat;
+    mp.done = done;
     mp.L = L;
     mp.K = K;
     mp.Kp = Kp;
@@ -242,7 +288,8 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     ap.hi = hi;
     ap.lo = lo;
     ap.mm = mm;
-    ap.hash = hash;
+    ap.mstat = mstat;
+    ap.qnorm = qnorm;
     ap.assign = assign;
     ap.hist_stride = (int64_t)p.iters * L;
     ap.part_sum = psum;
@@ -256,7 +303,10 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         ap.first = t == 0;
         {
             Launch pl("tiled_assign", st, head_bytes);
-            tiled::tiled_assign_kernel<<<dim3(n_tiles, (unsigned)NH), tiled::kThreads, alay.total, st>>>(ap);
+            const dim3 grid(n_tiles, (unsigned)NH);
+            if (Kp == 16) tiled::tiled_assign_kernel<16><<<grid, tiled::kThreads, alay.total, st>>>(qmap, ap);
+            else if (Kp == 32) tiled::tiled_assign_kernel<32><<<grid, tiled::kThreads, alay.total, st>>>(qmap, ap);
+            else tiled::tiled_assign_kernel<64><<<grid, tiled::kThreads, alay.total, st>>>(qmap, ap);
             pl.after();
         }
         CA_CUDA(cudaGetLastError());

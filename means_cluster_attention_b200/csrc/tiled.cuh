@@ -23,7 +23,10 @@
 // roberta-cluster" sections 2.1 and 3.
 #pragma once
 
+#include <cuda.h>
+
 #include "fused.cuh"
+#include "umma.cuh"
 
 namespace ca {
 namespace tiled {
@@ -63,22 +66,32 @@ struct MuParams {
     const int *part_cnt;     // [NH][Kp][n_tiles]
     float *mu;               // [NH][Kp][64]
     __nv_bfloat16 *hi, *lo;  // [NH][Kp][64]
-    float *mm;               // [NH][Kp]
+    float *mm;               // [NH][Kp]: |mu_k|^2, then +inf for centroids that can never win
     uint32_t *hash;          // [NH][Kp]
+    float *mstat;            // [NH][2]: max_k |mu_k|^2 and its square root
+    int *done;               // [NH] arrival counters, zero between launches
     float *cent_out;         // [NH][K][64] or null
     int L, K, Kp, n_tiles, init;
 };
 
 // grid (Kp, NH), 256 threads: thread (g4, j) adds tiles g4, g4+4, ... of
 // coordinate j of centroid k; the four exact partial sums are then added in
-// fixed order by group 0, which finalises the centroid row.
+// fixed order by group 0, which finalises the centroid row.  The last CTA of
+// a head to finish (arrival counter, no waiting) then marks the centroids
+// that are bitwise copies of a lower-index one (they can never win an argmin
+// whose ties go to the lowest index: |mu|^2 := +inf) and records max |mu|^2.
 __global__ void __launch_bounds__(256) tiled_mu_kernel(MuParams P) {
     __shared__ double red_s[3][64];
     __shared__ int red_c[4];
     __shared__ float red_sq[2];
     __shared__ uint32_t red_h[2];
+    __shared__ int last_s;
+    __shared__ float mu_s[64 * 65];
+    __shared__ float mm_s[64];
+    __shared__ uint32_t hsh_s[64];
+    __shared__ uint8_t dead_s[64];
     const int k = blockIdx.x, j = threadIdx.x & 63, g4 = threadIdx.x >> 6;
-    const int lane = threadIdx.x & 31, wid = (threadIdx.x >> 5) & 1;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, wid = warp & 1;
     const int64_t head = blockIdx.y;
     const int64_t kb = head * P.Kp + k;
     double s = 0.0;
@@ -92,40 +105,74 @@ __global__ void __launch_bounds__(256) tiled_mu_kernel(MuParams P) {
     if (g4 > 0) red_s[g4 - 1][j] = s;
     if (j == 0) red_c[g4] = cnt;
     __syncthreads();
-    if (g4 != 0) return;
-    float x = 0.f;
-    if (k < P.K) {
-        if (P.init) {
-            const int64_t row = ((int64_t)k * P.L) / P.K;
-            x = __bfloat162float(P.q[(head * P.L + row) * kD + j]);
-        } else {
-            const double tot = ((s + red_s[0][j]) + red_s[1][j]) + red_s[2][j];
-            const int n = red_c[0] + red_c[1] + red_c[2] + red_c[3];
-            x = __double2float_rn(tot / (double)(n > 1 ? n : 1));
+    if (g4 == 0) {
+        float x = 0.f;
+        if (k < P.K) {
+            if (P.init) {
+                const int64_t row = ((int64_t)k * P.L) / P.K;
+                x = __bfloat162float(P.q[(head * P.L + row) * kD + j]);
+            } else {
+                const double tot = ((s + red_s[0][j]) + red_s[1][j]) + red_s[2][j];
+                const int n = red_c[0] + red_c[1] + red_c[2] + red_c[3];
+                x = __double2float_rn(tot / (double)(n > 1 ? n : 1));
+            }
+        }
+        const int64_t o = kb * kD + j;
+        P.mu[o] = x;
+        const __nv_bfloat16 h = __float2bfloat16_rn(x);
+        P.hi[o] = h;
+        P.lo[o] = __float2bfloat16_rn(x - __bfloat162float(h));
+        if (P.cent_out && k < P.K) P.cent_out[(head * P.K + k) * kD + j] = x;
+        float sq = x * x;
+        uint32_t hv = __float_as_uint(x) * (0x9E3779B1u + 2u * (uint32_t)j) + (uint32_t)j * 0xC2B2AE3Du;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            hv += __shfl_xor_sync(0xffffffffu, hv, off);
+        }
+        if (lane == 0) {
+            red_sq[wid] = sq;
+            red_h[wid] = hv;
+        }
+        asm volatile("bar.sync 1, 64;");
+        if (j == 0) {
+            P.mm[kb] = red_sq[0] + red_sq[1];
+            P.hash[kb] = red_h[0] + red_h[1];
         }
     }
-    const int64_t o = kb * kD + j;
-    P.mu[o] = x;
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    P.hi[o] = h;
-    P.lo[o] = __float2bfloat16_rn(x - __bfloat162float(h));
-    if (P.cent_out && k < P.K) P.cent_out[(head * P.K + k) * kD + j] = x;
-    float sq = x * x;
-    uint32_t hv = __float_as_uint(x) * (0x9E3779B1u + 2u * (uint32_t)j) + (uint32_t)j * 0xC2B2AE3Du;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        sq += __shfl_xor_sync(0xffffffffu, sq, off);
-        hv += __shfl_xor_sync(0xffffffffu, hv, off);
+    // arrival: the CTA that completes the head's set finishes it
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last_s = atomicAdd(&P.done[head], 1) == P.Kp - 1;
+    __syncthreads();
+    if (!last_s) return;
+    __threadfence();
+    const int Kp = P.Kp, K = P.K;
+    for (int e = threadIdx.x; e < Kp * kD; e += 256)
+        mu_s[(e / kD) * 65 + e % kD] = __ldcg(P.mu + head * Kp * kD + e);
+    for (int kk = threadIdx.x; kk < Kp; kk += 256) {
+        const float m = __ldcg(P.mm + head * Kp + kk);
+        mm_s[kk] = kk < K ? m : INFINITY;
+        hsh_s[kk] = __ldcg(P.hash + head * Kp + kk);
+        dead_s[kk] = kk < K ? 0 : 1;
     }
-    if (lane == 0) {
-        red_sq[wid] = sq;
-        red_h[wid] = hv;
+    __syncthreads();
+    if (warp == 0) {
+        // a copy has its original's norm, so the max over every k < K is the
+        // max over the live centroids
+        float mx = 0.f;
+        for (int k2 = lane; k2 < K; k2 += 32) mx = fmaxf(mx, mm_s[k2]);
+        mx = warp_max(mx);
+        if (lane == 0) {
+            P.mstat[head * 2 + 0] = mx;
+            P.mstat[head * 2 + 1] = sqrtf(mx);
+        }
     }
-    asm volatile("bar.sync 1, 64;");
-    if (j == 0) {
-        P.mm[kb] = red_sq[0] + red_sq[1];
-        P.hash[kb] = red_h[0] + red_h[1];
-    }
+    __syncthreads();
+    mark_copies(K, hsh_s, mu_s, 65, dead_s, mm_s, warp, 8, lane);
+    __syncthreads();
+    for (int kk = threadIdx.x; kk < Kp; kk += 256) P.mm[head * Kp + kk] = mm_s[kk];
+    if (threadIdx.x == 0) P.done[head] = 0;
 }
 
 // Centroid-attention combine for the tiled path: grid (K, NH), 64 threads.
@@ -147,47 +194,60 @@ __global__ void __launch_bounds__(64) tiled_combine_kernel(int K, int n_chunks, 
 
 // ---------------------------------------------------------------------------
 // One Lloyd assignment for a tile of up to 512 queries.
+//
+// Q tile: two TMA loads of 256 rows (128-byte swizzle) into shared memory.
+// Distances: one thread issues tcgen05.mma for each 128-token block,
+// D = Q [128 x 64] . (hi + lo)^T [64 x Kp] accumulated in fp32 in tensor
+// memory (4 k-steps with hi, then 4 with lo, into the same accumulator).
+// Epilogue: every thread owns one token row of a block (tcgen05.ld), forms
+// s_k = |mu_k|^2 - 2 D_k, takes the minimum m1 and the set of k with
+// s_k <= m1 + 2E; a single member is the certified argmin, several send the
+// token to the exact fp64 re-measure.
+//
+// Error bound: the split leaves |mu - hi - lo| <= 2^-18 |mu| per coordinate;
+// the products are exact and even an accumulator that truncates every one of
+// the 128 additions stays within 128 * 2^-23 (1 + 2^-8) |Q| |mu| of the
+// exact dot product, so |s_k error| <= 2^-14.6 (|Q| |mu_k| + |mu_k|^2) with
+// the fp32 |mu_k|^2 and the final fma included; E = 2^-13 (|Q| max|mu| +
+// max|mu|^2) covers it threefold.
 struct AssignLayout {
-    int Kp, Tp;
-    uint32_t q_off, sums_off, mu_off, hi_off, lo_off, mm_off, hash_off, cnt_off, dead_off,
-        c_off, sc_off, cprev_off, list_off, perm_off, misc_off, total;
+    int Kp;
+    uint32_t q_off, b_off, mu_off, sums_off, mm_off, dead_off, cnt_off, c_off, sc_off, cprev_off, list_off,
+        perm_off, misc_off, bar_off, total;
     __host__ __device__ AssignLayout(int K) {
         Kp = kpad(K);
-        Tp = kTileQ;
         uint32_t o = 0;
-        q_off = o;
-        o += (uint32_t)Tp * 128u;
+        q_off = o;  // 512 rows x 128 bytes, 1024-aligned (TMA / MMA swizzle)
+        o += (uint32_t)kTileQ * 128u;
+        b_off = o;  // [hi; lo]: 2 Kp rows x 128 bytes, 1024-aligned
+        o += 2u * (uint32_t)Kp * 128u;
+        mu_off = o;  // fp32 centroids, rows padded to 65 floats, for the exact re-measure
+        o += up((uint32_t)Kp * 65u * 4u, 16);
         // Member sums stay in shared memory when they fit beside two CTAs per
         // SM (Kp <= 32); for Kp = 64 they go straight to the tile's global slot.
         sums_off = o;
         if (Kp <= 32) o += (uint32_t)Kp * 64u * 8u;
-        mu_off = o;  // fp32 centroid copy (rows padded to 65) for the exact re-measure
-        o += up((uint32_t)Kp * 65u * 4u, 16);
-        hi_off = o;
-        o += (uint32_t)Kp * 128u;
-        lo_off = o;
-        o += (uint32_t)Kp * 128u;
         mm_off = o;
-        o += (uint32_t)Kp * 4u;
-        hash_off = o;
-        o += (uint32_t)Kp * 4u;
-        cnt_off = o;
         o += (uint32_t)Kp * 4u;
         dead_off = o;
         o += up((uint32_t)Kp, 16);
+        cnt_off = o;
+        o += (uint32_t)Kp * 4u;
         c_off = o;
-        o += (uint32_t)Tp;
+        o += (uint32_t)kTileQ;
         sc_off = o;
-        o += (uint32_t)Tp;
+        o += (uint32_t)kTileQ;
         cprev_off = o;
-        o += (uint32_t)Tp;
+        o += (uint32_t)kTileQ;
         list_off = o;
-        o += (uint32_t)Tp * 2u;
+        o += (uint32_t)kTileQ * 2u;
         perm_off = o;
-        o += (uint32_t)Tp * 2u;
+        o += (uint32_t)kTileQ * 2u;
         misc_off = o;
         o += 64;
-        total = up(o, 128);
+        bar_off = o;  // two mbarriers and the tensor-memory address
+        o += 32;
+        total = up(o, 128) + 1024;  // + slack to align the base to 1024 bytes
     }
 };
 
@@ -195,8 +255,9 @@ struct AssignParams {
     const __nv_bfloat16 *q;
     const float *mu;
     const __nv_bfloat16 *hi, *lo;
-    const float *mm;
-    const uint32_t *hash;
+    const float *mm;     // [NH][Kp], +inf for centroids that cannot win
+    const float *mstat;  // [NH][2]
+    float *qnorm;        // [NH][L] |Q_i| (written by the first iteration, read later)
     int32_t *assign;     // [NH][L]
     int32_t *hist;       // [NH][iters][L] or null (already offset by the iteration)
     int64_t hist_stride; // iters * L
@@ -206,22 +267,28 @@ struct AssignParams {
     int first;           // 1: first Lloyd iteration (full sums); 0: only changed tokens move
 };
 
-__global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams P) {
-    extern __shared__ __align__(1024) unsigned char smem[];
+template <int KP>
+__global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_constant__ CUtensorMap tmq,
+                                                                    AssignParams P) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const AssignLayout lay(P.K);
-    const int K = P.K, Kp = lay.Kp;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int K = P.K;
+    constexpr int Kp = KP;
+    constexpr uint32_t kCols = 4u * KP;  // four 128-token accumulators of KP columns
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tile = blockIdx.x;
     const int64_t head = blockIdx.y;
     const int t0 = tile * kTileQ;
     const int Lt = min(kTileQ, P.L - t0);  // tokens in this tile
-    const __nv_bfloat16 *qh = P.q + (head * P.L + t0) * kD;
+    const int nblk = (Lt + 127) / 128;
 
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t q_s = sbase + lay.q_off, hi_s = sbase + lay.hi_off, lo_s = sbase + lay.lo_off;
+    const uint32_t q_s = sbase + lay.q_off, b_s = sbase + lay.b_off;
+    const uint32_t bar_tma = sbase + lay.bar_off, bar_mma = bar_tma + 8;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + lay.bar_off + 16);
     unsigned char *qbytes = smem + lay.q_off;
     float *mm = reinterpret_cast<float *>(smem + lay.mm_off);
-    uint32_t *hsh = reinterpret_cast<uint32_t *>(smem + lay.hash_off);
     int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
     uint8_t *dead = smem + lay.dead_off;
     uint8_t *cs = smem + lay.c_off;
@@ -233,10 +300,19 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
     const bool smem_sums = Kp <= 32 && P.first;
     double *ssum = reinterpret_cast<double *>(smem + lay.sums_off);  // [Kp][64] when smem_sums
 
-    load_rows(q_s, qh, 0, kTileQ, Lt);
-    cp_async_commit();
+    if (threadIdx.x == 0) {
+        umma::mbar_init(bar_tma, 1);
+        umma::mbar_init(bar_mma, 1);
+        umma::mbar_init_fence();
+        const int nbox = Lt > 256 ? 2 : 1;
+        umma::mbar_expect_tx(bar_tma, (uint32_t)nbox * 256u * 128u);
+        umma::tma_load_3d(q_s, &tmq, 0, t0, (int)head, bar_tma);
+        if (nbox == 2) umma::tma_load_3d(q_s + 256u * 128u, &tmq, 0, t0 + 256, (int)head, bar_tma);
+    }
+    __syncwarp();
+    if (warp == 0) umma::tmem_alloc(smem_u32(tslot), kCols);
+
     const int64_t cb = head * Kp;
-    // [Kp][64] centroids: a shared-memory copy when it fits, else global (L2).
     float *mu = reinterpret_cast<float *>(smem + lay.mu_off);  // [Kp][65]
     constexpr int mu_ld = 65;
     for (int e = threadIdx.x; e < Kp * kD; e += kThreads) mu[(e / kD) * 65 + e % kD] = P.mu[cb * kD + e];
@@ -251,17 +327,18 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
     } else {
         for (int i = threadIdx.x; i < Lt; i += kThreads) cprev[i] = (uint8_t)P.assign[head * P.L + t0 + i];
     }
+    // B operand [hi; lo] in the swizzled K-major layout of the MMA
     for (int e = threadIdx.x; e < Kp * 8; e += kThreads) {
         const int kk = e >> 3, ch = e & 7;
         const uint4 vh = *reinterpret_cast<const uint4 *>(P.hi + (cb + kk) * kD + ch * 8);
         const uint4 vl = *reinterpret_cast<const uint4 *>(P.lo + (cb + kk) * kD + ch * 8);
-        *reinterpret_cast<uint4 *>(smem + lay.hi_off + swz(kk, ch)) = vh;
-        *reinterpret_cast<uint4 *>(smem + lay.lo_off + swz(kk, ch)) = vl;
+        *reinterpret_cast<uint4 *>(smem + lay.b_off + swz(kk, ch)) = vh;
+        *reinterpret_cast<uint4 *>(smem + lay.b_off + (uint32_t)Kp * 128u + swz(kk, ch)) = vl;
     }
     for (int kk = threadIdx.x; kk < Kp; kk += kThreads) {
-        mm[kk] = kk < K ? P.mm[cb + kk] : INFINITY;
-        hsh[kk] = P.hash[cb + kk];
-        dead[kk] = kk < K ? 0 : 1;
+        const float m = P.mm[cb + kk];
+        mm[kk] = m;
+        dead[kk] = (m < INFINITY) ? 0 : 1;
         cnt_s[kk] = 0;
     }
     for (int i = threadIdx.x; i < kTileQ; i += kThreads) cs[i] = i < Lt ? 0 : 0xFF;
@@ -269,53 +346,48 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
         misc[0] = 0;
         misc[3] = 0;
     }
+    const float mm_max = P.mstat[head * 2 + 0], mun_max = P.mstat[head * 2 + 1];
+    umma::fence_proxy_async_smem();
+    umma::tc_fence_before();
     __syncthreads();
-    // dead centroids: bitwise copies of a lower-index centroid (|mu|^2 = +inf);
-    // max |mu|^2 over the live ones (a copy has its original's norm, so the
-    // max over all k < K is the same) from L2.
-    mark_copies(K, hsh, mu, mu_ld, dead, mm, warp, kWarps, lane);
-    if (warp == 0) {
-        float mx = 0.f;
-        for (int k2 = lane; k2 < K; k2 += 32) mx = fmaxf(mx, P.mm[cb + k2]);
-        mx = warp_max(mx);
-        if (lane == 0) {
-            misc[1] = __float_as_int(mx);
-            misc[2] = __float_as_int(sqrtf(mx));
+    umma::tc_fence_after();
+    const uint32_t taddr = *tslot;
+
+    // Q tile in shared memory (every thread observes the TMA completion
+    // before reading it), then the distance MMAs.
+    const bool q_ok = __syncthreads_and(umma::mbar_wait(bar_tma, 0));
+    if (threadIdx.x == 0) {
+        if (q_ok) {
+            constexpr uint32_t idesc = umma::idesc_bf16_f32(128, KP);
+            for (int m = 0; m < nblk; ++m)
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma::mma_bf16(taddr + (uint32_t)(m * KP),
+                                       umma::desc_sw128(q_s + (uint32_t)m * 16384u + (uint32_t)ks * 32u),
+                                       umma::desc_sw128(b_s + (uint32_t)part * (uint32_t)Kp * 128u + (uint32_t)ks * 32u),
+                                       idesc, part > 0 || ks > 0);
+            umma::mma_commit(bar_mma);
+        } else {
+            record_error(4, 30);
         }
     }
-    cp_async_wait<0>();
-    __syncthreads();
-    const float mm_max = __int_as_float(misc[1]), mun_max = __int_as_float(misc[2]);
-    constexpr int kMtPerWarp = kTileQ / 16 / kWarps;  // 4
-    const int n_mt = (Lt + 15) / 16;
-
-    // assignment: tensor-core distances + certified argmin
+    // |Q_i| of this thread's rows: computed in the first iteration (from the
+    // tile in shared memory), read back in later ones.
+    const int wg = warp >> 2, q4 = warp & 3;
+    float qn[2];
 #pragma unroll
-    for (int jp = 0; jp < kMtPerWarp; jp += 2) {
-        const int mt0 = warp + jp * kWarps, mt1 = mt0 + kWarps;
-        if (mt0 >= n_mt) break;
-        const bool two = mt1 < n_mt;
-        uint32_t a0[4][4], a1[4][4];
-        float qn[2][2];
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const int m = lane >> 3;
-            const int rr = (lane & 7) + ((m & 1) ? 8 : 0);
-            ldmatrix_x4(a0[ks], q_s + swz(mt0 * 16 + rr, 2 * ks + (m >> 1)));
-            if (two) ldmatrix_x4(a1[ks], q_s + swz(mt1 * 16 + rr, 2 * ks + (m >> 1)));
-            else a1[ks][0] = a1[ks][1] = a1[ks][2] = a1[ks][3] = 0u;
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int mt = u ? mt1 : mt0;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
+    for (int mi = 0; mi < 2; ++mi) {
+        const int row = (2 * wg + mi) * 128 + q4 * 32 + lane;
+        qn[mi] = 0.f;
+        if (row < Lt) {
+            if (P.first) {
                 float a = 0.f;
-                const int row = mt * 16 + g + 8 * h;
-                if (u == 0 || two) {
+                if (q_ok) {
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const uint4 w = *reinterpret_cast<const uint4 *>(qbytes + swz(row, 2 * t + c));
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(qbytes + swz(row, c));
                         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -324,69 +396,68 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(AssignParams 
                         }
                     }
                 }
-                a += __shfl_xor_sync(0xffffffffu, a, 1);
-                a += __shfl_xor_sync(0xffffffffu, a, 2);
-                qn[u][h] = sqrtf(a);
-            }
-        }
-        Best b[2][2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) b[u][h] = Best{INFINITY, INFINITY, 0};
-        for (int nt = 0; nt < Kp / 8; ++nt) {
-            uint32_t bh[2][4], bl[2][4];
-#pragma unroll
-            for (int kp = 0; kp < 2; ++kp) {
-                const int row = nt * 8 + (lane & 7);
-                const int chunk = 4 * kp + (lane >> 3);
-                ldmatrix_x4(bh[kp], hi_s + swz(row, chunk));
-                ldmatrix_x4(bl[kp], lo_s + swz(row, chunk));
-            }
-            float acc[2][2][4];
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                for (int s = 0; s < 2; ++s)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[u][s][e] = 0.f;
-#pragma unroll
-            for (int kp = 0; kp < 2; ++kp) {
-                mma_16816(acc[0][0], a0[2 * kp], bh[kp][0], bh[kp][1]);
-                mma_16816(acc[0][1], a0[2 * kp], bl[kp][0], bl[kp][1]);
-                mma_16816(acc[1][0], a1[2 * kp], bh[kp][0], bh[kp][1]);
-                mma_16816(acc[1][1], a1[2 * kp], bl[kp][0], bl[kp][1]);
-                mma_16816(acc[0][0], a0[2 * kp + 1], bh[kp][2], bh[kp][3]);
-                mma_16816(acc[0][1], a0[2 * kp + 1], bl[kp][2], bl[kp][3]);
-                mma_16816(acc[1][0], a1[2 * kp + 1], bh[kp][2], bh[kp][3]);
-                mma_16816(acc[1][1], a1[2 * kp + 1], bl[kp][2], bl[kp][3]);
-            }
-            const int c0 = nt * 8 + 2 * t;
-            const float m0 = mm[c0], m1 = mm[c0 + 1];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                best_push(b[u][0], fmaf(-2.f, acc[u][0][0] + acc[u][1][0], m0), c0);
-                best_push(b[u][0], fmaf(-2.f, acc[u][0][1] + acc[u][1][1], m1), c0 + 1);
-                best_push(b[u][1], fmaf(-2.f, acc[u][0][2] + acc[u][1][2], m0), c0);
-                best_push(b[u][1], fmaf(-2.f, acc[u][0][3] + acc[u][1][3], m1), c0 + 1);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int mt = u ? mt1 : mt0;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const Best bb = best_quad(b[u][h]);
-                const int row = mt * 16 + g + 8 * h;
-                if (t == 0 && (u == 0 || two) && row < Lt) {
-                    const float E = kEps * fmaf(qn[u][h], mun_max, mm_max);
-                    cs[row] = (uint8_t)bb.k1;
-                    if (bb.m2 <= bb.m1 + 2.f * E) list[atomicAdd(&misc[0], 1)] = (uint16_t)row;
-                }
+                qn[mi] = sqrtf(a);
+                P.qnorm[head * P.L + t0 + row] = qn[mi];
+            } else {
+                qn[mi] = P.qnorm[head * P.L + t0 + row];
             }
         }
     }
+    const bool mma_ok = __syncthreads_and(q_ok && umma::mbar_wait(bar_mma, 0));
+    if (!mma_ok && q_ok && threadIdx.x == 0) record_error(4, 31);
+    umma::tc_fence_after();
+    if (mma_ok) {
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) {
+            const int m = 2 * wg + mi;
+            if (m >= nblk) break;  // uniform across the warp
+            const int row = m * 128 + q4 * 32 + lane;
+            float sv[KP];
+            const uint32_t ta = taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(m * KP);
+#pragma unroll
+            for (int c = 0; c < KP; c += 16) {
+                float v16[16];
+                umma::tmem_ld16(ta + (uint32_t)c, v16);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sv[c + i] = v16[i];
+            }
+            umma::tmem_ld_wait();
+            if (row < Lt) {
+                float m1a = INFINITY, m1b = INFINITY;
+#pragma unroll
+                for (int k4 = 0; k4 < KP / 4; ++k4) {
+                    const float4 m4 = reinterpret_cast<const float4 *>(mm)[k4];
+                    sv[4 * k4 + 0] = fmaf(-2.f, sv[4 * k4 + 0], m4.x);
+                    sv[4 * k4 + 1] = fmaf(-2.f, sv[4 * k4 + 1], m4.y);
+                    sv[4 * k4 + 2] = fmaf(-2.f, sv[4 * k4 + 2], m4.z);
+                    sv[4 * k4 + 3] = fmaf(-2.f, sv[4 * k4 + 3], m4.w);
+                    m1a = fminf(m1a, fminf(sv[4 * k4 + 0], sv[4 * k4 + 1]));
+                    m1b = fminf(m1b, fminf(sv[4 * k4 + 2], sv[4 * k4 + 3]));
+                }
+                const float m1 = fminf(m1a, m1b);
+                const float thr = m1 + 2.f * (kEps * fmaf(qn[mi], mun_max, mm_max));
+                uint32_t bits[(KP + 31) / 32];
+#pragma unroll
+                for (int w2 = 0; w2 < (KP + 31) / 32; ++w2) bits[w2] = 0u;
+#pragma unroll
+                for (int k = 0; k < KP; ++k) bits[k >> 5] |= (sv[k] <= thr ? 1u : 0u) << (k & 31);
+                int c = -1, n = 0;
+#pragma unroll
+                for (int w2 = (KP + 31) / 32 - 1; w2 >= 0; --w2) {
+                    n += __popc(bits[w2]);
+                    if (bits[w2]) c = w2 * 32 + __ffs(bits[w2]) - 1;
+                }
+                cs[row] = (uint8_t)(c < 0 ? 0 : c);
+                if (n != 1) list[atomicAdd(&misc[0], 1)] = (uint16_t)row;
+            }
+        }
+    }
+    umma::tc_fence_before();
     __syncthreads();
+    if (warp == 0) {
+        umma::tc_fence_after();
+        umma::tmem_dealloc(taddr, kCols);
+    }
     // exact re-measure of ambiguous tokens, one warp per token
     const int n_ref = misc[0];
     for (int e = warp; e < n_ref; e += kWarps) {

@@ -1,0 +1,133 @@
+// Blackwell (sm_100a) asynchronous primitives in inline PTX: mbarriers with
+// bounded waits, TMA tensor loads (no multicast), tcgen05 tensor-memory
+// allocation, single-thread tcgen05.mma issue with its commit, and
+// tensor-memory loads into registers.
+//
+// Operand layout used throughout: K-major bf16 rows of exactly 64 elements
+// (128 bytes), 128-byte swizzled in groups of 8 rows (1024 bytes, 1024-byte
+// aligned): 16-byte chunk c of row r sits at r * 128 + ((c ^ (r & 7)) << 4).
+// This is what a TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes, what swz()
+// in mma.cuh addresses, and what the SWIZZLE_128B shared-memory matrix
+// descriptor of tcgen05.mma reads.
+#pragma once
+
+#include <stdint.h>
+
+#include "common.cuh"
+#include "mma.cuh"
+
+namespace ca {
+namespace umma {
+
+// Iteration limit of every wait on an mbarrier; mbarrier.try_wait itself
+// suspends for a while, so this bounds a wait to well under a second.
+constexpr int kWaitLimit = 1 << 20;
+
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+
+// Makes mbarrier initialisation visible to the asynchronous proxy (TMA, MMA).
+__device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred P1;\n mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n selp.b32 %0, 1, 0, P1;\n}\n"
+        : "=r"(ok)
+        : "r"(mbar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete; false when the
+// iteration limit ran out (the caller records CA_ERR_TIMEOUT and carries on
+// without the guarded data).
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
+    for (int i = 0; i < kWaitLimit; ++i)
+        if (mbar_try_wait(mbar, parity)) return true;
+    return false;
+}
+
+// Generic-proxy writes to shared memory (st.shared) become visible to the
+// asynchronous proxy (tcgen05.mma operand reads) after this fence and a
+// barrier.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 3-D tiled TMA load (no multicast) of box {64, rows, 1} at coordinates
+// (x, y, z) into shared memory, completing on mbar.  x must be 0 here (the
+// inner coordinate stays 16-byte aligned); y may run past the tensor's
+// extent, in which case TMA writes zeros for the missing rows.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int x, int y, int z, uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(mbar)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major, 128-byte-swizzled operand
+// starting at saddr (the 8-row groups 1024 bytes apart).  Stepping K by 16
+// bf16 elements advances saddr by 32 bytes.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4)  // start address, 16-byte units
+           | ((uint64_t)1 << 16)                // leading byte offset (unused for swizzled K-major)
+           | ((uint64_t)(1024 >> 4) << 32)      // stride byte offset: 8 rows x 128 bytes
+           | ((uint64_t)1 << 46)                // descriptor version for sm_100
+           | ((uint64_t)2 << 61);               // 128-byte swizzle
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B (both K-major) and an
+// fp32 accumulator, for an M x N tile.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+    return (1u << 4)                            // D: fp32
+           | (1u << 7)                          // A: bf16
+           | (1u << 10)                         // B: bf16
+           | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(accumulate ? 1u : 0u));
+}
+
+// mbar receives one arrival once every tcgen05.mma this thread issued before
+// it has completed.
+__device__ __forceinline__ void mma_commit(uint32_t mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem), "r"(ncols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 16 consecutive fp32 columns of this warp's 32 tensor-memory lanes (lane i
+// of the warp receives row i of its quarter).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+}  // namespace umma
+}  // namespace ca
