@@ -231,12 +231,13 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     __nv_bfloat16 *hi = nullptr, *lo = nullptr;
     uint32_t *hash = nullptr;
     double *psum = nullptr;
-    int *pcnt = nullptr, *done = nullptr;
+    int *pcnt = nullptr;
+    uint8_t *dead = nullptr;
     float *mstat = nullptr, *qnorm = nullptr;
     int32_t *assign = assign_out;
     CA_CUDA(s.get((void **)&mu, sizeof(float) * NH * Kp * kD));
     CA_CUDA(s.get((void **)&mstat, sizeof(float) * NH * 2));
-    CA_CUDA(s.get((void **)&done, sizeof(int) * NH));
+    CA_CUDA(s.get((void **)&dead, sizeof(uint8_t) * NH * Kp));
     CA_CUDA(s.get((void **)&qnorm, sizeof(float) * NH * L));
     CA_CUDA(s.get((void **)&hi, sizeof(__nv_bfloat16) * NH * Kp * kD));
     CA_CUDA(s.get((void **)&lo, sizeof(__nv_bfloat16) * NH * Kp * kD));
@@ -244,10 +245,9 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     CA_CUDA(s.get((void **)&hash, sizeof(uint32_t) * NH * Kp));
     CA_CUDA(s.get((void **)&psum, sizeof(double) * NH * n_tiles * Kp * kD));
     CA_CUDA(s.get((void **)&pcnt, sizeof(int) * NH * n_tiles * Kp));
-    CA_CUDA(s.get((void **)&cpart, sizeof(float) * NH * n_chunks * K * (kD + 2)));
+    CA_CUDA(s.get((void **)&cpart, sizeof(float) * NH * n_chunks * K * tiled::kPartLd));
     CA_CUDA(s.get((void **)&vcent, sizeof(float) * NH * K * kD));
     if (!assign) CA_CUDA(s.get((void **)&assign, sizeof(int32_t) * NH * L));
-    CA_CUDA(cudaMemsetAsync(done, 0, sizeof(int) * NH, st));
     CUtensorMap qmap;
     {
         ca_status ms = encode_rows_map(&qmap, q, NH, L);
@@ -265,8 +265,6 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     mp.lo = lo;
     mp.mm = mm;
     mp.hash = hash;
-    mp.mstat = mstat;
-    mp.done = done;
     mp.L = L;
     mp.K = K;
     mp.Kp = Kp;
@@ -288,6 +286,7 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     ap.hi = hi;
     ap.lo = lo;
     ap.mm = mm;
+    ap.dead = dead;
     ap.mstat = mstat;
     ap.qnorm = qnorm;
     ap.assign = assign;
@@ -299,6 +298,12 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     ap.n_tiles = n_tiles;
     mp.init = 0;
     for (int t = 0; t < p.iters; ++t) {
+        {
+            Launch pl("tiled_dead", st, 0.0);
+            tiled::tiled_dead_kernel<<<dim3(Kp, (unsigned)NH), 64, 0, st>>>(K, Kp, mu, mm, hash, dead, mstat);
+            pl.after();
+        }
+        CA_CUDA(cudaGetLastError());
         ap.hist = hist ? hist + (int64_t)t * L : nullptr;
         ap.first = t == 0;
         {

@@ -66,32 +66,22 @@ struct MuParams {
     const int *part_cnt;     // [NH][Kp][n_tiles]
     float *mu;               // [NH][Kp][64]
     __nv_bfloat16 *hi, *lo;  // [NH][Kp][64]
-    float *mm;               // [NH][Kp]: |mu_k|^2, then +inf for centroids that can never win
+    float *mm;               // [NH][Kp] |mu_k|^2
     uint32_t *hash;          // [NH][Kp]
-    float *mstat;            // [NH][2]: max_k |mu_k|^2 and its square root
-    int *done;               // [NH] arrival counters, zero between launches
     float *cent_out;         // [NH][K][64] or null
     int L, K, Kp, n_tiles, init;
 };
 
 // grid (Kp, NH), 256 threads: thread (g4, j) adds tiles g4, g4+4, ... of
 // coordinate j of centroid k; the four exact partial sums are then added in
-// fixed order by group 0, which finalises the centroid row.  The last CTA of
-// a head to finish (arrival counter, no waiting) then marks the centroids
-// that are bitwise copies of a lower-index one (they can never win an argmin
-// whose ties go to the lowest index: |mu|^2 := +inf) and records max |mu|^2.
+// fixed order by group 0, which finalises the centroid row.
 __global__ void __launch_bounds__(256) tiled_mu_kernel(MuParams P) {
     __shared__ double red_s[3][64];
     __shared__ int red_c[4];
     __shared__ float red_sq[2];
     __shared__ uint32_t red_h[2];
-    __shared__ int last_s;
-    __shared__ float mu_s[64 * 65];
-    __shared__ float mm_s[64];
-    __shared__ uint32_t hsh_s[64];
-    __shared__ uint8_t dead_s[64];
     const int k = blockIdx.x, j = threadIdx.x & 63, g4 = threadIdx.x >> 6;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, wid = warp & 1;
+    const int lane = threadIdx.x & 31, wid = (threadIdx.x >> 5) & 1;
     const int64_t head = blockIdx.y;
     const int64_t kb = head * P.Kp + k;
     double s = 0.0;
@@ -105,7 +95,8 @@ __global__ void __launch_bounds__(256) tiled_mu_kernel(MuParams P) {
     if (g4 > 0) red_s[g4 - 1][j] = s;
     if (j == 0) red_c[g4] = cnt;
     __syncthreads();
-    if (g4 == 0) {
+    if (g4 != 0) return;
+    {
         float x = 0.f;
         if (k < P.K) {
             if (P.init) {
@@ -140,54 +131,96 @@ __global__ void __launch_bounds__(256) tiled_mu_kernel(MuParams P) {
             P.hash[kb] = red_h[0] + red_h[1];
         }
     }
-    // arrival: the CTA that completes the head's set finishes it
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) last_s = atomicAdd(&P.done[head], 1) == P.Kp - 1;
-    __syncthreads();
-    if (!last_s) return;
-    __threadfence();
-    const int Kp = P.Kp, K = P.K;
-    for (int e = threadIdx.x; e < Kp * kD; e += 256)
-        mu_s[(e / kD) * 65 + e % kD] = __ldcg(P.mu + head * Kp * kD + e);
-    for (int kk = threadIdx.x; kk < Kp; kk += 256) {
-        const float m = __ldcg(P.mm + head * Kp + kk);
-        mm_s[kk] = kk < K ? m : INFINITY;
-        hsh_s[kk] = __ldcg(P.hash + head * Kp + kk);
-        dead_s[kk] = kk < K ? 0 : 1;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        // a copy has its original's norm, so the max over every k < K is the
-        // max over the live centroids
-        float mx = 0.f;
-        for (int k2 = lane; k2 < K; k2 += 32) mx = fmaxf(mx, mm_s[k2]);
-        mx = warp_max(mx);
-        if (lane == 0) {
-            P.mstat[head * 2 + 0] = mx;
-            P.mstat[head * 2 + 1] = sqrtf(mx);
-        }
-    }
-    __syncthreads();
-    mark_copies(K, hsh_s, mu_s, 65, dead_s, mm_s, warp, 8, lane);
-    __syncthreads();
-    for (int kk = threadIdx.x; kk < Kp; kk += 256) P.mm[head * Kp + kk] = mm_s[kk];
-    if (threadIdx.x == 0) P.done[head] = 0;
 }
 
+// Centroids that can never win: grid (Kp, NH), 64 threads.  CTA k marks
+// centroid k dead when it is a bitwise copy of a lower-index centroid (its
+// distances equal that centroid's and ties go to the lowest index) or a
+// padding row (k >= K); lower indices with the same row hash are compared
+// coordinate by coordinate, lowest first.  CTA 0 also records max_k |mu_k|^2
+// over k < K (a copy has its original's norm).
+__global__ void __launch_bounds__(64) tiled_dead_kernel(int K, int Kp, const float *__restrict__ mu,
+                                                        const float *__restrict__ mm,
+                                                        const uint32_t *__restrict__ hash, uint8_t *__restrict__ dead,
+                                                        float *__restrict__ mstat) {
+    const int k = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int64_t head = blockIdx.y, hb = head * Kp;
+    if (k == 0 && w == 1) {
+        float mx = 0.f;
+        for (int k2 = lane; k2 < K; k2 += 32) mx = fmaxf(mx, mm[hb + k2]);
+        mx = warp_max(mx);
+        if (lane == 0) {
+            mstat[head * 2 + 0] = mx;
+            mstat[head * 2 + 1] = sqrtf(mx);
+        }
+    }
+    if (k >= K) {
+        if (t == 0) dead[hb + k] = 1;
+        return;
+    }
+    const uint32_t hk = hash[hb + k];
+    const float x = mu[(hb + k) * kD + t];
+    // Both warps form the same candidate masks, so every barrier below is
+    // reached by all 64 threads; the barrier's vote is the same everywhere.
+    bool found = false;
+    for (int a0 = 0; a0 < k && !found; a0 += 32) {
+        const int a = a0 + lane;
+        unsigned cand = __ballot_sync(0xffffffffu, a < k && hash[hb + a] == hk);
+        while (cand && !found) {
+            const int b = a0 + __ffs(cand) - 1;
+            cand &= cand - 1u;
+            found = __syncthreads_and(__float_as_uint(mu[(hb + b) * kD + t]) == __float_as_uint(x)) != 0;
+        }
+    }
+    if (t == 0) dead[hb + k] = found ? 1 : 0;
+}
+
+// Floats per chunk state of the centroid attention: 64 accumulator values,
+// the running max (natural-log units), the running denominator, and padding
+// to a 16-byte multiple.
+constexpr int kPartLd = kD + 4;
+
 // Centroid-attention combine for the tiled path: grid (K, NH), 64 threads.
+// Thread c takes chunk c of a group of 64 (all its loads in flight at once);
+// the group's states are rescaled to the group max and summed column by
+// column through shared memory, in chunk order.
 __global__ void __launch_bounds__(64) tiled_combine_kernel(int K, int n_chunks, const float *__restrict__ part,
                                                             float *__restrict__ vcent) {
-    const int k = blockIdx.x, t = threadIdx.x;
+    __shared__ float rows[64][65];
+    __shared__ float red_m[2], red_l[2];
+    const int k = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int64_t h = blockIdx.y;
-    float M = -INFINITY;
-    for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, part[((h * n_chunks + c) * K + k) * (kD + 2) + kD]);
-    float lsum = 0.f, acc = 0.f;
-    for (int c = 0; c < n_chunks; ++c) {
-        const float *p = part + ((h * n_chunks + c) * K + k) * (kD + 2);
-        const float w = expf(p[kD] - M);
-        lsum = fmaf(p[kD + 1], w, lsum);
-        acc = fmaf(p[t], w, acc);
+    float M = -INFINITY, lsum = 0.f, acc = 0.f;
+    for (int c0 = 0; c0 < n_chunks; c0 += 64) {
+        const int c = c0 + t;
+        const bool ok = c < n_chunks;
+        const float *p = part + ((h * n_chunks + (ok ? c : 0)) * K + k) * kPartLd;
+        float4 r[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) r[u] = ok ? reinterpret_cast<const float4 *>(p)[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float2 ml = ok ? *reinterpret_cast<const float2 *>(p + kD) : make_float2(-INFINITY, 0.f);
+        const float gm = warp_max(ml.x);
+        if (lane == 0) red_m[w] = gm;
+        __syncthreads();
+        const float Mn = fmaxf(M, fmaxf(red_m[0], red_m[1]));
+        const float f_old = (M == -INFINITY) ? 0.f : expf(M - Mn);
+        const float wc = (ml.x == -INFINITY) ? 0.f : expf(ml.x - Mn);
+        const float gl = warp_sum(wc * ml.y);
+        if (lane == 0) red_l[w] = gl;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            rows[t][4 * u + 0] = wc * r[u].x;
+            rows[t][4 * u + 1] = wc * r[u].y;
+            rows[t][4 * u + 2] = wc * r[u].z;
+            rows[t][4 * u + 3] = wc * r[u].w;
+        }
+        __syncthreads();
+        float col = 0.f;
+        for (int cc = 0; cc < 64; ++cc) col += rows[cc][t];
+        acc = fmaf(acc, f_old, col);
+        lsum = fmaf(lsum, f_old, red_l[0] + red_l[1]);
+        M = Mn;
+        __syncthreads();
     }
     vcent[(h * K + k) * kD + t] = acc / lsum;
 }
@@ -212,21 +245,22 @@ __global__ void __launch_bounds__(64) tiled_combine_kernel(int K, int n_chunks, 
 // max|mu|^2) covers it threefold.
 struct AssignLayout {
     int Kp;
-    uint32_t q_off, b_off, mu_off, sums_off, mm_off, dead_off, cnt_off, c_off, sc_off, cprev_off, list_off,
-        perm_off, misc_off, bar_off, total;
+    uint32_t q_off, r_off, mu_off, mm_off, dead_off, cnt_off, c_off, sc_off, cprev_off, list_off, perm_off,
+        misc_off, bar_off, total;
     __host__ __device__ AssignLayout(int K) {
         Kp = kpad(K);
         uint32_t o = 0;
         q_off = o;  // 512 rows x 128 bytes, 1024-aligned (TMA / MMA swizzle)
         o += (uint32_t)kTileQ * 128u;
-        b_off = o;  // [hi; lo]: 2 Kp rows x 128 bytes, 1024-aligned
-        o += 2u * (uint32_t)Kp * 128u;
-        mu_off = o;  // fp32 centroids, rows padded to 65 floats, for the exact re-measure
-        o += up((uint32_t)Kp * 65u * 4u, 16);
-        // Member sums stay in shared memory when they fit beside two CTAs per
-        // SM (Kp <= 32); for Kp = 64 they go straight to the tile's global slot.
-        sums_off = o;
-        if (Kp <= 32) o += (uint32_t)Kp * 64u * 8u;
+        // Region R, reused in turn: the MMA's B operand [hi; lo] (2 Kp rows of
+        // 128 bytes, 1024-aligned) beside the fp32 centroids (rows padded to
+        // 65 floats) for the exact re-measure; then the tile's fp64 member
+        // sums [Kp][64].
+        r_off = o;
+        mu_off = o + 2u * (uint32_t)Kp * 128u;
+        const uint32_t r_a = 2u * (uint32_t)Kp * 128u + (uint32_t)Kp * 65u * 4u;
+        const uint32_t r_b = (uint32_t)Kp * 64u * 8u;
+        o += up(r_a > r_b ? r_a : r_b, 16);
         mm_off = o;
         o += (uint32_t)Kp * 4u;
         dead_off = o;
@@ -255,7 +289,8 @@ struct AssignParams {
     const __nv_bfloat16 *q;
     const float *mu;
     const __nv_bfloat16 *hi, *lo;
-    const float *mm;     // [NH][Kp], +inf for centroids that cannot win
+    const float *mm;     // [NH][Kp] |mu_k|^2
+    const uint8_t *dead; // [NH][Kp] 1 for centroids that can never win
     const float *mstat;  // [NH][2]
     float *qnorm;        // [NH][L] |Q_i| (written by the first iteration, read later)
     int32_t *assign;     // [NH][L]
@@ -264,8 +299,16 @@ struct AssignParams {
     double *part_sum;    // [NH][Kp][n_tiles][64]
     int *part_cnt;       // [NH][Kp][n_tiles]
     int L, K, n_tiles;
-    int first;           // 1: first Lloyd iteration (full sums); 0: only changed tokens move
+    int first;           // 1: first Lloyd iteration; 0: the slots hold the previous iteration's sums
 };
+
+// Later iterations move at most this many tokens of a tile by exact fp64
+// subtract / add on the tile's slot; more movers recompute the tile's sums.
+constexpr int kMoverMax = 96;
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src));
+}
 
 template <int KP>
 __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_constant__ CUtensorMap tmq,
@@ -284,10 +327,12 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     const int nblk = (Lt + 127) / 128;
 
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t q_s = sbase + lay.q_off, b_s = sbase + lay.b_off;
+    const uint32_t q_s = sbase + lay.q_off, b_s = sbase + lay.r_off;
     const uint32_t bar_tma = sbase + lay.bar_off, bar_mma = bar_tma + 8;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + lay.bar_off + 16);
     unsigned char *qbytes = smem + lay.q_off;
+    float *mu = reinterpret_cast<float *>(smem + lay.mu_off);        // [Kp][65] until the re-measure ends
+    double *ssum = reinterpret_cast<double *>(smem + lay.r_off);     // [Kp][64] after it
     float *mm = reinterpret_cast<float *>(smem + lay.mm_off);
     int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
     uint8_t *dead = smem + lay.dead_off;
@@ -297,8 +342,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     uint16_t *list = reinterpret_cast<uint16_t *>(smem + lay.list_off);
     uint16_t *perm = reinterpret_cast<uint16_t *>(smem + lay.perm_off);
     int *misc = reinterpret_cast<int *>(smem + lay.misc_off);
-    const bool smem_sums = Kp <= 32 && P.first;
-    double *ssum = reinterpret_cast<double *>(smem + lay.sums_off);  // [Kp][64] when smem_sums
+    constexpr int mu_ld = 65;
 
     if (threadIdx.x == 0) {
         umma::mbar_init(bar_tma, 1);
@@ -312,33 +356,39 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     __syncwarp();
     if (warp == 0) umma::tmem_alloc(smem_u32(tslot), kCols);
 
+    // Staging, all of it asynchronous or issued before it is waited for:
+    // [hi; lo] in the swizzled K-major layout of the MMA, and the fp32
+    // centroids for the re-measure.
     const int64_t cb = head * Kp;
-    float *mu = reinterpret_cast<float *>(smem + lay.mu_off);  // [Kp][65]
-    constexpr int mu_ld = 65;
-    for (int e = threadIdx.x; e < Kp * kD; e += kThreads) mu[(e / kD) * 65 + e % kD] = P.mu[cb * kD + e];
-    // This tile's slots of the partial sums, cleared before the run sums add in.
-    double *psum = P.part_sum;
-    if (P.first) {
-        for (int e = threadIdx.x; e < Kp * kD; e += kThreads) {
-            const int kk = e / kD, j = e % kD;
-            if (smem_sums) ssum[e] = 0.0;
-            else psum[((cb + kk) * P.n_tiles + tile) * kD + j] = 0.0;
-        }
-    } else {
-        for (int i = threadIdx.x; i < Lt; i += kThreads) cprev[i] = (uint8_t)P.assign[head * P.L + t0 + i];
-    }
-    // B operand [hi; lo] in the swizzled K-major layout of the MMA
     for (int e = threadIdx.x; e < Kp * 8; e += kThreads) {
         const int kk = e >> 3, ch = e & 7;
-        const uint4 vh = *reinterpret_cast<const uint4 *>(P.hi + (cb + kk) * kD + ch * 8);
-        const uint4 vl = *reinterpret_cast<const uint4 *>(P.lo + (cb + kk) * kD + ch * 8);
-        *reinterpret_cast<uint4 *>(smem + lay.b_off + swz(kk, ch)) = vh;
-        *reinterpret_cast<uint4 *>(smem + lay.b_off + (uint32_t)Kp * 128u + swz(kk, ch)) = vl;
+        cp_async16(b_s + swz(kk, ch), P.hi + (cb + kk) * kD + ch * 8, 16);
+        cp_async16(b_s + (uint32_t)Kp * 128u + swz(kk, ch), P.lo + (cb + kk) * kD + ch * 8, 16);
+    }
+    for (int e = threadIdx.x; e < Kp * kD; e += kThreads)
+        cp_async4(smem_u32(mu + (e / kD) * mu_ld + e % kD), P.mu + cb * kD + e);
+    cp_async_commit();
+    float qn_g[2] = {0.f, 0.f};
+    const int wg = warp >> 2, q4 = warp & 3;
+    if (!P.first) {
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) {
+            const int row = (2 * wg + mi) * 128 + q4 * 32 + lane;
+            if (row < Lt) qn_g[mi] = P.qnorm[head * P.L + t0 + row];
+        }
+        int pv[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int i = threadIdx.x + u * kThreads;
+            pv[u] = i < Lt ? P.assign[head * P.L + t0 + i] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) cprev[threadIdx.x + u * kThreads] = (uint8_t)pv[u];
     }
     for (int kk = threadIdx.x; kk < Kp; kk += kThreads) {
-        const float m = P.mm[cb + kk];
-        mm[kk] = m;
-        dead[kk] = (m < INFINITY) ? 0 : 1;
+        const uint8_t dd = P.dead[cb + kk];
+        mm[kk] = dd ? INFINITY : P.mm[cb + kk];
+        dead[kk] = dd;
         cnt_s[kk] = 0;
     }
     for (int i = threadIdx.x; i < kTileQ; i += kThreads) cs[i] = i < Lt ? 0 : 0xFF;
@@ -347,6 +397,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
         misc[3] = 0;
     }
     const float mm_max = P.mstat[head * 2 + 0], mun_max = P.mstat[head * 2 + 1];
+    cp_async_wait<0>();
     umma::fence_proxy_async_smem();
     umma::tc_fence_before();
     __syncthreads();
@@ -373,16 +424,14 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
             record_error(4, 30);
         }
     }
-    // |Q_i| of this thread's rows: computed in the first iteration (from the
-    // tile in shared memory), read back in later ones.
-    const int wg = warp >> 2, q4 = warp & 3;
-    float qn[2];
+    // |Q_i| of this thread's rows: computed in the first iteration from the
+    // tile in shared memory (and stored), read back in later ones.
+    float qn[2] = {qn_g[0], qn_g[1]};
+    if (P.first) {
 #pragma unroll
-    for (int mi = 0; mi < 2; ++mi) {
-        const int row = (2 * wg + mi) * 128 + q4 * 32 + lane;
-        qn[mi] = 0.f;
-        if (row < Lt) {
-            if (P.first) {
+        for (int mi = 0; mi < 2; ++mi) {
+            const int row = (2 * wg + mi) * 128 + q4 * 32 + lane;
+            if (row < Lt) {
                 float a = 0.f;
                 if (q_ok) {
 #pragma unroll
@@ -398,8 +447,6 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
                 }
                 qn[mi] = sqrtf(a);
                 P.qnorm[head * P.L + t0 + row] = qn[mi];
-            } else {
-                qn[mi] = P.qnorm[head * P.L + t0 + row];
             }
         }
     }
@@ -527,8 +574,9 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
         if (P.hist) P.hist[head * P.hist_stride + t0 + i] = cs[i];
     }
     if (!P.first) {
-        // Later iterations: only tokens whose cluster changed move between the
-        // tile's member sums (exact fp64 subtract / add) and counts.
+        // Later iterations list the tokens whose cluster changed; when they
+        // are few, only they move between the tile's member sums (exact fp64
+        // subtract / add on the slot) and counts.
         for (int ch = warp; ch < kTileQ / 32; ch += kWarps) {
             const int i = ch * 32 + lane;
             const bool mv = i < Lt && cs[i] != cprev[i];
@@ -540,24 +588,31 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
         }
         __syncthreads();
         const int n_mv = misc[3];
-        for (int e = warp; e < n_mv; e += kWarps) {
-            const int row = list[e];
-            const int co = cprev[row], cn = cs[row];
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(qbytes + swz(row, lane >> 2) + (lane & 3) * 4);
-            const double d0 = bf16_to_f64(w & 0xffffu), d1 = bf16_to_f64(w >> 16);
-            double *so = psum + ((cb + co) * P.n_tiles + tile) * kD;
-            double *sn = psum + ((cb + cn) * P.n_tiles + tile) * kD;
-            atomicAdd(&so[2 * lane], -d0);
-            atomicAdd(&so[2 * lane + 1], -d1);
-            atomicAdd(&sn[2 * lane], d0);
-            atomicAdd(&sn[2 * lane + 1], d1);
-            if (lane == 0) {
-                atomicSub(&P.part_cnt[(cb + co) * P.n_tiles + tile], 1);
-                atomicAdd(&P.part_cnt[(cb + cn) * P.n_tiles + tile], 1);
+        if (n_mv <= kMoverMax) {
+            double *psum = P.part_sum;
+            for (int e = warp; e < n_mv; e += kWarps) {
+                const int row = list[e];
+                const int co = cprev[row], cn = cs[row];
+                const uint32_t w = *reinterpret_cast<const uint32_t *>(qbytes + swz(row, lane >> 2) + (lane & 3) * 4);
+                const double d0 = bf16_to_f64(w & 0xffffu), d1 = bf16_to_f64(w >> 16);
+                double *so = psum + ((cb + co) * P.n_tiles + tile) * kD;
+                double *sn = psum + ((cb + cn) * P.n_tiles + tile) * kD;
+                atomicAdd(&so[2 * lane], -d0);
+                atomicAdd(&so[2 * lane + 1], -d1);
+                atomicAdd(&sn[2 * lane], d0);
+                atomicAdd(&sn[2 * lane + 1], d1);
+                if (lane == 0) {
+                    atomicSub(&P.part_cnt[(cb + co) * P.n_tiles + tile], 1);
+                    atomicAdd(&P.part_cnt[(cb + cn) * P.n_tiles + tile], 1);
+                }
             }
+            return;
         }
-        return;
     }
+    // Full member sums of the tile into shared memory (region R is free now
+    // that the MMA and the re-measure are done).
+    for (int e = threadIdx.x; e < Kp * kD / 2; e += kThreads)
+        reinterpret_cast<double2 *>(ssum)[e] = make_double2(0.0, 0.0);
     // counting sort of the tile's tokens by cluster (order inside a cluster
     // is free: the sums are exact).  Peers of one cluster in a 32-token chunk
     // take their offsets with one atomic on the count; every warp then scans
@@ -600,7 +655,10 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
         }
     }
     __syncthreads();
-    // exact member sums, run by run over the sorted tokens
+    // exact member sums, run by run over the sorted tokens: each warp walks a
+    // contiguous eighth of them, lane l adding coordinates 2l and 2l+1 into
+    // four chains; a run's sum goes into its cluster's row with an fp64
+    // shared-memory atomic
     {
         const int seg = (Lt + kWarps - 1) / kWarps;
         const int p1 = min(Lt, (warp + 1) * seg);
@@ -646,15 +704,15 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
                 p += n;
                 if (n < 32) break;
             }
-            double *dst = smem_sums ? ssum + c * kD : psum + ((cb + c) * P.n_tiles + tile) * kD;
-            atomicAdd(&dst[2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
-            atomicAdd(&dst[2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
+            atomicAdd(&ssum[c * kD + 2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
+            atomicAdd(&ssum[c * kD + 2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
         }
     }
-    if (smem_sums) {
-        __syncthreads();
-        for (int e = threadIdx.x; e < Kp * kD; e += kThreads)
-            psum[((cb + e / kD) * P.n_tiles + tile) * kD + e % kD] = ssum[e];
+    __syncthreads();
+    for (int e = threadIdx.x; e < Kp * kD / 2; e += kThreads) {
+        const int kk = (2 * e) / kD, j = (2 * e) % kD;
+        *reinterpret_cast<double2 *>(P.part_sum + ((cb + kk) * P.n_tiles + tile) * kD + j) =
+            reinterpret_cast<const double2 *>(ssum)[e];
     }
     for (int kk = threadIdx.x; kk < Kp; kk += kThreads) P.part_cnt[(cb + kk) * P.n_tiles + tile] = cnt_s[kk];
 }
@@ -687,7 +745,7 @@ struct CentroidLayout {
 struct CentroidParams {
     const __nv_bfloat16 *k, *v;
     const __nv_bfloat16 *hi, *lo;  // [NH][Kp][64]
-    float *part;                   // [NH][n_chunks][K][66]
+    float *part;                   // [NH][n_chunks][K][kPartLd]
     int L, K, n_chunks;
     float scale;
 };
@@ -863,14 +921,16 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_centroid_kernel(CentroidPar
         ml[(warp * 16 + g + 8) * 2 + 1] = rl[1];
     }
     __syncthreads();
-    float *outp = P.part + ((head * P.n_chunks + chunk) * (int64_t)K) * (kD + 2);
-    for (int e = threadIdx.x; e < K * (kD + 2); e += kThreads) {
-        const int row = e / (kD + 2), col = e % (kD + 2);
+    float *outp = P.part + ((head * P.n_chunks + chunk) * (int64_t)K) * kPartLd;
+    for (int e = threadIdx.x; e < K * kPartLd; e += kThreads) {
+        const int row = e / kPartLd, col = e % kPartLd;
         const int mt = row / 16, rr = row % 16;
         float M = -INFINITY;
         for (int w = mt * G; w < mt * G + G; ++w) M = fmaxf(M, ml[(w * 16 + rr) * 2]);
         float val;
-        if (col == kD) {
+        if (col >= kD + 2) {
+            val = 0.f;  // padding
+        } else if (col == kD) {
             val = M * P.scale;  // running max in natural-log units
         } else {
             float acc = 0.f;
