@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "clusterattn.h"
 #include "common.cuh"
@@ -212,6 +213,26 @@ ca_status encode_rows_map(CUtensorMap *map, const void *base, int64_t NH, int L)
     return CA_OK;
 }
 
+// Launches a kernel that may start before the previous kernel on the stream
+// completes (programmatic dependent launch); the kernel itself waits for
+// its predecessor (pdl_wait) before touching anything the predecessor
+// writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // The tiled bf16 path serves the heads the fused kernel does not take, for
 // K <= 64 and a window radius floor(W/2) <= 128.
 bool tiled_eligible(int dtype, const Problem &p) {
@@ -300,7 +321,8 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     for (int t = 0; t < p.iters; ++t) {
         {
             Launch pl("tiled_dead", st, 0.0);
-            tiled::tiled_dead_kernel<<<dim3(Kp, (unsigned)NH), 64, 0, st>>>(K, Kp, mu, mm, hash, dead, mstat);
+            CA_CUDA(launch_pdl(tiled::tiled_dead_kernel, dim3(Kp, (unsigned)NH), dim3(64), 0, st, K, Kp,
+                               (const float *)mu, (const float *)mm, (const uint32_t *)hash, dead, mstat));
             pl.after();
         }
         CA_CUDA(cudaGetLastError());
@@ -309,16 +331,16 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         {
             Launch pl("tiled_assign", st, head_bytes);
             const dim3 grid(n_tiles, (unsigned)NH);
-            if (Kp == 16) tiled::tiled_assign_kernel<16><<<grid, tiled::kThreads, alay.total, st>>>(qmap, ap);
-            else if (Kp == 32) tiled::tiled_assign_kernel<32><<<grid, tiled::kThreads, alay.total, st>>>(qmap, ap);
-            else tiled::tiled_assign_kernel<64><<<grid, tiled::kThreads, alay.total, st>>>(qmap, ap);
+            auto kern = Kp == 16 ? tiled::tiled_assign_kernel<16>
+                                 : (Kp == 32 ? tiled::tiled_assign_kernel<32> : tiled::tiled_assign_kernel<64>);
+            CA_CUDA(launch_pdl(kern, grid, dim3(tiled::kThreads), alay.total, st, qmap, ap));
             pl.after();
         }
         CA_CUDA(cudaGetLastError());
         mp.cent_out = t == p.iters - 1 ? cent_out : nullptr;
         {
             Launch pl("tiled_update", st, 0.0);
-            tiled::tiled_mu_kernel<<<dim3(Kp, (unsigned)NH), 256, 0, st>>>(mp);
+            CA_CUDA(launch_pdl(tiled::tiled_mu_kernel, dim3(Kp, (unsigned)NH), dim3(256), 0, st, mp));
             pl.after();
         }
         CA_CUDA(cudaGetLastError());
@@ -337,13 +359,15 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     cp.scale = scale;
     {
         Launch pl("tiled_centroid", st, 2.0 * head_bytes);
-        tiled::tiled_centroid_kernel<<<dim3(n_chunks, (unsigned)NH), tiled::kThreads, clay.total, st>>>(cp);
+        CA_CUDA(launch_pdl(tiled::tiled_centroid_kernel, dim3(n_chunks, (unsigned)NH), dim3(tiled::kThreads), clay.total,
+                           st, cp));
         pl.after();
     }
     CA_CUDA(cudaGetLastError());
     {
         Launch pl("tiled_combine", st, 0.0);
-        tiled::tiled_combine_kernel<<<dim3(K, (unsigned)NH), 64, 0, st>>>(K, n_chunks, cpart, vcent);
+        CA_CUDA(launch_pdl(tiled::tiled_combine_kernel, dim3(K, (unsigned)NH), dim3(64), 0, st, K, n_chunks,
+                           (const float *)cpart, vcent));
         pl.after();
     }
     CA_CUDA(cudaGetLastError());
@@ -363,7 +387,8 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     wp.scale = scale;
     {
         Launch pl("tiled_window", st, 4.0 * head_bytes);
-        tiled::tiled_window_kernel<<<dim3((L + tiled::kWinQ - 1) / tiled::kWinQ, (unsigned)NH), tiled::kThreads, wlay.total, st>>>(wp);
+        CA_CUDA(launch_pdl(tiled::tiled_window_kernel, dim3((L + tiled::kWinQ - 1) / tiled::kWinQ, (unsigned)NH),
+                           dim3(tiled::kThreads), wlay.total, st, wp));
         pl.after();
     }
     CA_CUDA(cudaGetLastError());

@@ -32,6 +32,15 @@ struct Variant {
     __host__ __device__ int64_t batch(int64_t h) const { return h / H; }
 };
 
+// Programmatic dependent launch.  pdl_launch lets the next kernel of the
+// stream be scheduled before this one completes; pdl_wait blocks until the
+// previous kernel of the stream has completed and its writes are visible
+// (no-ops when the launch did not ask for it).  A kernel touches nothing its
+// predecessor writes, and writes nothing its predecessor reads, before
+// pdl_wait: only the forward's inputs and its own shared memory.
+__device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void record_error(int code, int where) {
     if (atomicCAS(&g_dev_error, 0, code) == 0) g_dev_error_where = where;
 }

@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(256) tiled_mu_kernel(MuParams P) {
     const int lane = threadIdx.x & 31, wid = (threadIdx.x >> 5) & 1;
     const int64_t head = blockIdx.y;
     const int64_t kb = head * P.Kp + k;
+    pdl_launch();
+    pdl_wait();
     double s = 0.0;
     int cnt = 0;
     if (!P.init && k < P.K) {
@@ -145,6 +147,8 @@ __global__ void __launch_bounds__(64) tiled_dead_kernel(int K, int Kp, const flo
                                                         float *__restrict__ mstat) {
     const int k = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int64_t head = blockIdx.y, hb = head * Kp;
+    pdl_launch();
+    pdl_wait();
     if (k == 0 && w == 1) {
         float mx = 0.f;
         for (int k2 = lane; k2 < K; k2 += 32) mx = fmaxf(mx, mm[hb + k2]);
@@ -190,6 +194,8 @@ __global__ void __launch_bounds__(64) tiled_combine_kernel(int K, int n_chunks, 
     __shared__ float red_m[2], red_l[2];
     const int k = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int64_t h = blockIdx.y;
+    pdl_launch();
+    pdl_wait();
     float M = -INFINITY, lsum = 0.f, acc = 0.f;
     for (int c0 = 0; c0 < n_chunks; c0 += 64) {
         const int c = c0 + t;
@@ -344,6 +350,9 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     int *misc = reinterpret_cast<int *>(smem + lay.misc_off);
     constexpr int mu_ld = 65;
 
+    pdl_launch();
+    // The query tile is an input of the forward: its load starts before the
+    // previous kernel (the centroid update) has finished.
     if (threadIdx.x == 0) {
         umma::mbar_init(bar_tma, 1);
         umma::mbar_init(bar_mma, 1);
@@ -353,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
         umma::tma_load_3d(q_s, &tmq, 0, t0, (int)head, bar_tma);
         if (nbox == 2) umma::tma_load_3d(q_s + 256u * 128u, &tmq, 0, t0 + 256, (int)head, bar_tma);
     }
+    pdl_wait();
     __syncwarp();
     if (warp == 0) umma::tmem_alloc(smem_u32(tslot), kCols);
 
@@ -766,6 +776,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_centroid_kernel(CentroidPar
     const uint32_t slot_s = sbase + lay.slots_off, hi_s = sbase + lay.hi_off, lo_s = sbase + lay.lo_off;
     float *ml = reinterpret_cast<float *>(smem + lay.ml_off);
 
+    pdl_launch();
     for (int s = 0; s < kSlots; ++s) {
         if (s < nT) {
             const uint32_t slot = slot_s + s * 2 * kTile * 128;
@@ -774,6 +785,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_centroid_kernel(CentroidPar
         }
         cp_async_commit();
     }
+    pdl_wait();  // the centroids come from the previous kernel
     const int64_t cb = head * Kp;
     for (int e = threadIdx.x; e < Kp * 8; e += kThreads) {
         const int kk = e >> 3, ch = e & 7;
@@ -995,9 +1007,11 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
     const int ks0 = max(0, qb - r) & ~7;
     const int ke = min(L - 1, qb + kWinQ - 1 + r);
     const int nrows = (ke - ks0 + 1 + 7) & ~7;
+    pdl_launch();
     load_rows(kw_s, kh, ks0, nrows, ke + 1);
     load_rows(vw_s, vh, ks0, nrows, ke + 1);
     cp_async_commit();
+    pdl_wait();  // V_cent and the assignments come from earlier kernels
     const float *vch = P.vcent + head * (int64_t)K * kD;
     const float be = 1.f - P.alpha;
     for (int e = threadIdx.x; e < K * kD / 4; e += kThreads) {
