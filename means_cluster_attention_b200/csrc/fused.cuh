@@ -38,6 +38,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "kmeans_tile.cuh"
 #include "mma.cuh"
 
 namespace ca {
@@ -186,28 +187,7 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Exact fp64 value of a bf16 bit pattern (low 16 bits of b) built with
-// integer operations: the 8-bit exponent is rebiased (+896) into the 11-bit
-// field and the 7 fraction bits become the top fraction bits.  Zero and
-// subnormal inputs take the (exact) conversion path.  Inputs are finite.
-__device__ __forceinline__ double bf16_to_f64(uint32_t b) {
-    if ((b & 0x7F80u) == 0u) return (double)__uint_as_float(b << 16);
-    const uint32_t hi = ((b & 0x8000u) << 16) | (((b & 0x7FFFu) << 13) + 0x38000000u);
-    return __hiloint2double((int)hi, 0);
-}
-
-// Both bf16 halves of a 32-bit word as exact doubles, for words whose two
-// exponent fields are non-zero (the caller checks; see bf16_to_f64).
-__device__ __forceinline__ void bf16x2_to_f64_normal(uint32_t w, double &lo, double &hi) {
-    const uint32_t h0 = ((w << 16) & 0x80000000u) | (((w & 0x7FFFu) << 13) + 0x38000000u);
-    const uint32_t h1 = (w & 0x80000000u) | (((w >> 3) & 0x0FFFE000u) + 0x38000000u);
-    lo = __hiloint2double((int)h0, 0);
-    hi = __hiloint2double((int)h1, 0);
-}
-
-__device__ __forceinline__ bool bf16x2_has_zero_exp(uint32_t w) {
-    return ((w & 0x7F80u) == 0u) || ((w & 0x7F800000u) == 0u);
-}
+using tile::bf16_to_f64;
 
 __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -422,69 +402,11 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         if (threadIdx.x == 0) misc[1] = 0;
         // Lane k holds centroid k (and k + 32 when Kp = 64); the chains of
         // the second set are only run when that set exists.
-        auto remeasure = [&](int row, auto two_c, double &bd, int &bk) {
-            constexpr bool two = decltype(two_c)::value;
-            double qq = 0.0, qm0 = 0.0, qm1 = 0.0, m20 = 0.0, m21 = 0.0;
-            const int k0 = lane, k1 = lane + 32;
-            const bool v0 = k0 < Kp, v1 = two && k1 < Kp;
-#pragma unroll 2
-            for (int jb = 0; jb < kD; jb += 8) {
-                const uint4 w = *reinterpret_cast<const uint4 *>(qbytes + swz(row, jb >> 3));
-                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                double qj[8], mj0[8], mj1[8];
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                    qj[2 * e2] = bf16_to_f64(ws[e2] & 0xffffu);
-                    qj[2 * e2 + 1] = bf16_to_f64(ws[e2] >> 16);
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    mj0[u] = v0 ? mu64[k0 * 65 + jb + u] : 0.0;
-                    if constexpr (two) mj1[u] = v1 ? mu64[k1 * 65 + jb + u] : 0.0;
-                }
-                // Every product (bf16 x bf16, bf16 x fp32, fp32 x fp32) is
-                // exact in fp64, so one fused multiply-add rounds exactly as
-                // a separately rounded product followed by a rounded sum.
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    qq = __fma_rn(qj[u], qj[u], qq);
-                    qm0 = __fma_rn(qj[u], mj0[u], qm0);
-                    m20 = __fma_rn(mj0[u], mj0[u], m20);
-                    if constexpr (two) {
-                        qm1 = __fma_rn(qj[u], mj1[u], qm1);
-                        m21 = __fma_rn(mj1[u], mj1[u], m21);
-                    }
-                }
-            }
-            bd = INFINITY;
-            bk = 0x7fffffff;
-            if (v0 && !dead[k0]) {
-                bd = __dsub_rn(__dadd_rn(qq, m20), __dmul_rn(2.0, qm0));
-                bk = k0;
-            }
-            if (v1 && !dead[k1]) {
-                const double D = __dsub_rn(__dadd_rn(qq, m21), __dmul_rn(2.0, qm1));
-                if (D < bd) {
-                    bd = D;
-                    bk = k1;
-                }
-            }
-        };
+        auto mu_at = [&](int k, int j) { return mu64[k * 65 + j]; };
         for (int e = warp; e < n_ref; e += kWarps) {
             const int row = list[e];
-            double bd;
-            int bk;
-            if (Kp > 32) remeasure(row, std::true_type{}, bd, bk);
-            else remeasure(row, std::false_type{}, bd, bk);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const double od = __shfl_xor_sync(0xffffffffu, bd, o);
-                const int ok = __shfl_xor_sync(0xffffffffu, bk, o);
-                if (od < bd || (od == bd && ok < bk)) {
-                    bd = od;
-                    bk = ok;
-                }
-            }
+            int bk = Kp > 32 ? tile::remeasure_token<true>(qbytes, row, Kp, dead, mu_at, lane)
+                             : tile::remeasure_token<false>(qbytes, row, Kp, dead, mu_at, lane);
             if (bk >= K) {
                 if (lane == 0) record_error(5, 2);
                 bk = 0;
@@ -530,103 +452,11 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                 if (threadIdx.x < Kp) cnt_s[threadIdx.x] = 0;
                 __syncthreads();
             }
-            // Counting sort by cluster (order inside a cluster is free: the
-            // sums are exact).  Peers of one cluster in a 32-token chunk take
-            // their offsets with one atomic on the count; every warp then
-            // scans the counts itself.
-            int my_c[2], my_off[2];
-#pragma unroll
-            for (int s2 = 0; s2 < 2; ++s2) {
-                const int ch = warp + s2 * kWarps;
-                my_c[s2] = 0xFF;
-                my_off[s2] = 0;
-                if (ch < nch) {
-                    const int c = cs[ch * 32 + lane];
-                    const unsigned peers = __match_any_sync(0xffffffffu, c);
-                    const int leader = __ffs(peers) - 1;
-                    int off = 0;
-                    if (c != 0xFF && lane == leader) off = atomicAdd(&cnt_s[c], __popc(peers));
-                    off = __shfl_sync(0xffffffffu, off, leader);
-                    my_c[s2] = c;
-                    my_off[s2] = off + __popc(peers & ((1u << lane) - 1u));
-                }
-            }
-            __syncthreads();
-            {
-                const int c0 = lane < Kp ? cnt_s[lane] : 0, c1 = lane + 32 < Kp ? cnt_s[lane + 32] : 0;
-                int s0 = c0, s1 = c1;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int x0 = __shfl_up_sync(0xffffffffu, s0, o), x1 = __shfl_up_sync(0xffffffffu, s1, o);
-                    if (lane >= o) {
-                        s0 += x0;
-                        s1 += x1;
-                    }
-                }
-                const int b0 = s0 - c0, b1 = __shfl_sync(0xffffffffu, s0, 31) + s1 - c1;
-#pragma unroll
-                for (int s2 = 0; s2 < 2; ++s2) {
-                    const int c = my_c[s2];
-                    const int x0 = __shfl_sync(0xffffffffu, b0, c & 31), x1 = __shfl_sync(0xffffffffu, b1, c & 31);
-                    if (c != 0xFF) {
-                        const int pos = (c < 32 ? x0 : x1) + my_off[s2];
-                        perm[pos] = (uint16_t)((warp + s2 * kWarps) * 32 + lane);
-                        sc[pos] = (uint8_t)c;
-                    }
-                }
-            }
-            __syncthreads();
-            // Each warp walks a contiguous slice of the sorted tokens run by
-            // run (one cluster per run), lane holding coordinates 2*lane and
-            // 2*lane+1, four independent accumulators; a run's sum is added
-            // into the cluster's row with an fp64 shared-memory atomic.
+            // Counting sort by cluster, then exact fp64 member sums over a
+            // contiguous eighth of the sorted tokens per warp.
+            tile::counting_sort(cs, nch, Kp, cnt_s, perm, sc, warp, kWarps, lane);
             const int seg = (L + kWarps - 1) / kWarps;
-            const int p1 = min(L, (warp + 1) * seg);
-            int p = warp * seg;
-            while (p < p1) {
-                const int c = sc[p];
-                double s0[4] = {0.0, 0.0, 0.0, 0.0}, s1[4] = {0.0, 0.0, 0.0, 0.0};
-                for (;;) {
-                    const int q = p + lane;
-                    const unsigned same = __ballot_sync(0xffffffffu, q < p1 && sc[q] == c);
-                    const int n = __ffs(~same) ? __ffs(~same) - 1 : 32;
-                    const int rowl = (lane < n) ? perm[p + lane] : 0;
-                    for (int j = 0; j < n; j += 4) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int rr = __shfl_sync(0xffffffffu, rowl, (j + u) & 31);
-                            w[u] = (j + u < n) ? *reinterpret_cast<const uint32_t *>(qbytes + swz(rr, lane >> 2) + (lane & 3) * 4) : 0u;
-                        }
-                        bool slow = false;
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) slow |= (j + u < n) && bf16x2_has_zero_exp(w[u]);
-                        if (__any_sync(0xffffffffu, slow)) {
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                if (j + u < n) {
-                                    s0[u] += bf16_to_f64(w[u] & 0xffffu);
-                                    s1[u] += bf16_to_f64(w[u] >> 16);
-                                }
-                            }
-                        } else {
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                if (j + u < n) {
-                                    double d0, d1;
-                                    bf16x2_to_f64_normal(w[u], d0, d1);
-                                    s0[u] += d0;
-                                    s1[u] += d1;
-                                }
-                            }
-                        }
-                    }
-                    p += n;
-                    if (n < 32) break;
-                }
-                atomicAdd(&sums[c * kD + 2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
-                atomicAdd(&sums[c * kD + 2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
-            }
+            tile::member_sums(qbytes, sc, perm, warp * seg, min(L, (warp + 1) * seg), sums, lane);
         }
         __syncthreads();
         for (int i = threadIdx.x; i < Lp; i += kThreads) cprev[i] = cs[i];

@@ -26,21 +26,16 @@
 #include <cuda.h>
 
 #include "fused.cuh"
+#include "kmeans_tile.cuh"
 #include "umma.cuh"
 
 namespace ca {
 namespace tiled {
 
-using fused::Best;
-using fused::best_merge;
-using fused::best_push;
-using fused::best_quad;
-using fused::bf16_to_f64;
 using fused::bf16hi;
 using fused::bf16lo;
-using fused::bf16x2_has_zero_exp;
-using fused::bf16x2_to_f64_normal;
 using fused::ex2;
+using tile::bf16_to_f64;
 using fused::kEps;
 using fused::kLog2e;
 using fused::load_rows;
@@ -519,57 +514,8 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     const int n_ref = misc[0];
     for (int e = warp; e < n_ref; e += kWarps) {
         const int row = list[e];
-        double qq = 0.0, qm0 = 0.0, qm1 = 0.0, m20 = 0.0, m21 = 0.0;
-        const int k0 = lane, k1 = lane + 32;
-        const bool v0 = k0 < Kp, v1 = k1 < Kp;
-#pragma unroll 2
-        for (int jb = 0; jb < kD; jb += 8) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(qbytes + swz(row, jb >> 3));
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-            double qj[8], mj0[8], mj1[8];
-#pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) {
-                qj[2 * e2] = bf16_to_f64(ws[e2] & 0xffffu);
-                qj[2 * e2 + 1] = bf16_to_f64(ws[e2] >> 16);
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                mj0[u] = v0 ? (double)mu[k0 * mu_ld + jb + u] : 0.0;
-                mj1[u] = v1 ? (double)mu[k1 * mu_ld + jb + u] : 0.0;
-            }
-            // every product is exact in fp64: one fused multiply-add rounds
-            // exactly as a rounded product followed by a rounded sum
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                qq = __fma_rn(qj[u], qj[u], qq);
-                qm0 = __fma_rn(qj[u], mj0[u], qm0);
-                m20 = __fma_rn(mj0[u], mj0[u], m20);
-                qm1 = __fma_rn(qj[u], mj1[u], qm1);
-                m21 = __fma_rn(mj1[u], mj1[u], m21);
-            }
-        }
-        double bd = INFINITY;
-        int bk = 0x7fffffff;
-        if (v0 && !dead[k0]) {
-            bd = __dsub_rn(__dadd_rn(qq, m20), __dmul_rn(2.0, qm0));
-            bk = k0;
-        }
-        if (v1 && !dead[k1]) {
-            const double D = __dsub_rn(__dadd_rn(qq, m21), __dmul_rn(2.0, qm1));
-            if (D < bd) {
-                bd = D;
-                bk = k1;
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double od = __shfl_xor_sync(0xffffffffu, bd, o);
-            const int ok = __shfl_xor_sync(0xffffffffu, bk, o);
-            if (od < bd || (od == bd && ok < bk)) {
-                bd = od;
-                bk = ok;
-            }
-        }
+        int bk = tile::remeasure_token<(KP > 32)>(qbytes, row, Kp, dead,
+                                                  [&](int k, int j) { return (double)mu[k * mu_ld + j]; }, lane);
         if (lane == 0) {
             if (bk >= K) {
                 record_error(5, 3);
@@ -623,100 +569,10 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     // that the MMA and the re-measure are done).
     for (int e = threadIdx.x; e < Kp * kD / 2; e += kThreads)
         reinterpret_cast<double2 *>(ssum)[e] = make_double2(0.0, 0.0);
-    // counting sort of the tile's tokens by cluster (order inside a cluster
-    // is free: the sums are exact).  Peers of one cluster in a 32-token chunk
-    // take their offsets with one atomic on the count; every warp then scans
-    // the counts itself.
-    {
-        int my_c[2], my_off[2];
-#pragma unroll
-        for (int s2 = 0; s2 < 2; ++s2) {
-            const int ch = warp + s2 * kWarps;
-            const int c = cs[ch * 32 + lane];
-            const unsigned peers = __match_any_sync(0xffffffffu, c);
-            const int leader = __ffs(peers) - 1;
-            int off = 0;
-            if (c != 0xFF && lane == leader) off = atomicAdd(&cnt_s[c], __popc(peers));
-            off = __shfl_sync(0xffffffffu, off, leader);
-            my_c[s2] = c;
-            my_off[s2] = off + __popc(peers & ((1u << lane) - 1u));
-        }
-        __syncthreads();
-        const int c0 = lane < Kp ? cnt_s[lane] : 0, c1 = lane + 32 < Kp ? cnt_s[lane + 32] : 0;
-        int s0 = c0, s1 = c1;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int x0 = __shfl_up_sync(0xffffffffu, s0, o), x1 = __shfl_up_sync(0xffffffffu, s1, o);
-            if (lane >= o) {
-                s0 += x0;
-                s1 += x1;
-            }
-        }
-        const int b0 = s0 - c0, b1 = __shfl_sync(0xffffffffu, s0, 31) + s1 - c1;
-#pragma unroll
-        for (int s2 = 0; s2 < 2; ++s2) {
-            const int c = my_c[s2];
-            const int x0 = __shfl_sync(0xffffffffu, b0, c & 31), x1 = __shfl_sync(0xffffffffu, b1, c & 31);
-            if (c != 0xFF) {
-                const int pos = (c < 32 ? x0 : x1) + my_off[s2];
-                perm[pos] = (uint16_t)((warp + s2 * kWarps) * 32 + lane);
-                sc[pos] = (uint8_t)c;
-            }
-        }
-    }
-    __syncthreads();
-    // exact member sums, run by run over the sorted tokens: each warp walks a
-    // contiguous eighth of them, lane l adding coordinates 2l and 2l+1 into
-    // four chains; a run's sum goes into its cluster's row with an fp64
-    // shared-memory atomic
+    tile::counting_sort(cs, kTileQ / 32, Kp, cnt_s, perm, sc, warp, kWarps, lane);
     {
         const int seg = (Lt + kWarps - 1) / kWarps;
-        const int p1 = min(Lt, (warp + 1) * seg);
-        int p = warp * seg;
-        while (p < p1) {
-            const int c = sc[p];
-            double s0[4] = {0.0, 0.0, 0.0, 0.0}, s1[4] = {0.0, 0.0, 0.0, 0.0};
-            for (;;) {
-                const int qq = p + lane;
-                const unsigned same = __ballot_sync(0xffffffffu, qq < p1 && sc[qq] == c);
-                const int n = __ffs(~same) ? __ffs(~same) - 1 : 32;
-                const int rowl = (lane < n) ? perm[p + lane] : 0;
-                for (int j = 0; j < n; j += 4) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int rr = __shfl_sync(0xffffffffu, rowl, (j + u) & 31);
-                        w[u] = (j + u < n) ? *reinterpret_cast<const uint32_t *>(qbytes + swz(rr, lane >> 2) + (lane & 3) * 4) : 0u;
-                    }
-                    bool slow = false;
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) slow |= (j + u < n) && bf16x2_has_zero_exp(w[u]);
-                    if (__any_sync(0xffffffffu, slow)) {
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            if (j + u < n) {
-                                s0[u] += bf16_to_f64(w[u] & 0xffffu);
-                                s1[u] += bf16_to_f64(w[u] >> 16);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            if (j + u < n) {
-                                double d0, d1;
-                                bf16x2_to_f64_normal(w[u], d0, d1);
-                                s0[u] += d0;
-                                s1[u] += d1;
-                            }
-                        }
-                    }
-                }
-                p += n;
-                if (n < 32) break;
-            }
-            atomicAdd(&ssum[c * kD + 2 * lane], (s0[0] + s0[1]) + (s0[2] + s0[3]));
-            atomicAdd(&ssum[c * kD + 2 * lane + 1], (s1[0] + s1[1]) + (s1[2] + s1[3]));
-        }
+        tile::member_sums(qbytes, sc, perm, warp * seg, min(Lt, (warp + 1) * seg), ssum, lane);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < Kp * kD / 2; e += kThreads) {
