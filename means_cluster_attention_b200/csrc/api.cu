@@ -139,6 +139,8 @@ ca_status ensure_kernel_attributes() {
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(centroid_attn_partial_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
@@ -183,11 +185,11 @@ ca_status run_fused(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     return CA_OK;
 }
 
-// TMA tensor map of a [NH, L, 64] bf16 tensor read in boxes of 256 rows of
-// one head, 128-byte swizzled (the layout the tcgen05 operand descriptors
+// TMA tensor map of a [NH, L, 64] bf16 tensor read in boxes of box_rows
+// (<= 256) rows of one head, 128-byte swizzled (the layout the tcgen05 operand descriptors
 // read).  Rows past L (inside a box) are filled with zeros by the TMA unit.
 // The driver's encoder is looked up once through the runtime.
-ca_status encode_rows_map(CUtensorMap *map, const void *base, int64_t NH, int L) {
+ca_status encode_rows_map(CUtensorMap *map, const void *base, int64_t NH, int L, int box_rows = 256) {
     static std::mutex mu;
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     {
@@ -204,7 +206,7 @@ ca_status encode_rows_map(CUtensorMap *map, const void *base, int64_t NH, int L)
     }
     const cuuint64_t dims[3] = {(cuuint64_t)ca::kD, (cuuint64_t)L, (cuuint64_t)NH};
     const cuuint64_t strides[2] = {(cuuint64_t)ca::kD * 2u, (cuuint64_t)L * ca::kD * 2u};
-    const cuuint32_t box[3] = {(cuuint32_t)ca::kD, 256u, 1u};
+    const cuuint32_t box[3] = {(cuuint32_t)ca::kD, (cuuint32_t)box_rows, 1u};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
     const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -372,7 +374,6 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     }
     CA_CUDA(cudaGetLastError());
 
-    const tiled::WindowLayout wlay(K, p.W / 2);
     tiled::WindowParams wp{};
     wp.q = q;
     wp.k = k;
@@ -385,7 +386,21 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     wp.r = p.W / 2;
     wp.alpha = p.alpha;
     wp.scale = scale;
-    {
+    if (wp.r <= 64) {
+        // tensor-core window kernel: the key window [q0 - RP, q0 + 127 + RP]
+        const int RP = wp.r <= 32 ? 32 : 64;
+        const tiled::WindowTcLayout tlay(RP);
+        CUtensorMap kmap, vmap, q128;
+        ca_status ms = encode_rows_map(&q128, q, NH, L, 128);
+        if (ms == CA_OK) ms = encode_rows_map(&kmap, k, NH, L, tlay.NK);
+        if (ms == CA_OK) ms = encode_rows_map(&vmap, v, NH, L, tlay.NK);
+        if (ms != CA_OK) return ms;
+        Launch pl("tiled_window", st, 4.0 * head_bytes);
+        CA_CUDA(launch_pdl(RP == 32 ? tiled::tiled_window_tc_kernel<32> : tiled::tiled_window_tc_kernel<64>,
+                           dim3((L + 127) / 128, (unsigned)NH), dim3(128), tlay.total, st, q128, kmap, vmap, wp));
+        pl.after();
+    } else {
+        const tiled::WindowLayout wlay(K, p.W / 2);
         Launch pl("tiled_window", st, 4.0 * head_bytes);
         CA_CUDA(launch_pdl(tiled::tiled_window_kernel, dim3((L + tiled::kWinQ - 1) / tiled::kWinQ, (unsigned)NH),
                            dim3(tiled::kThreads), wlay.total, st, wp));

@@ -1038,5 +1038,199 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
     }
 }
 
+// ---------------------------------------------------------------------------
+// Window attention + gather + blend for 128 queries on tcgen05, radius
+// r <= RP (RP = 32 or 64).  Keys of the CTA's window: [q0 - RP, q0 + 127 +
+// RP], NK = 128 + 2 RP of them, TMA-loaded with the query block (rows outside
+// [0, L) arrive as zeros and are masked).
+//
+//   S = Q K^T           one thread issues 4 MMAs (M = 128, N = NK, K = 64),
+//                       fp32 scores in tensor memory;
+//   softmax             thread i owns query row i (tensor-memory lane i): its
+//                       warp's 32 + 2 RP columns are read twice (row max,
+//                       then exp2), keys outside |i - j| <= r or [0, L) get
+//                       weight 0; P is rounded to bf16 into shared memory
+//                       (over the dead Q and K tiles, K-major, 128-byte
+//                       swizzled blocks of 64 keys);
+//   O = P V             NK / 16 MMAs (M = 128, N = 64), V read N-major as
+//                       loaded, accumulated over the first 64 columns of S;
+//   epilogue            O = (1 - alpha) V_cent[c_i] + (alpha / l_i) o_i,
+//                       rounded once to bf16, one 128-byte row per thread.
+struct WindowTcLayout {
+    int NK;
+    uint32_t qk_off, v_off, bar_off, total;
+    __host__ __device__ WindowTcLayout(int RP) {
+        NK = 128 + 2 * RP;
+        qk_off = 0;  // Q (16 KB) then K (NK rows); afterwards P (NK / 64 blocks of 16 KB)
+        const uint32_t qk = 16384u + (uint32_t)NK * 128u, pb = (uint32_t)NK / 64u * 16384u;
+        v_off = up(qk > pb ? qk : pb, 1024);
+        bar_off = v_off + (uint32_t)NK * 128u;
+        total = up(bar_off + 32u, 128) + 1024;  // + slack to align the base to 1024 bytes
+    }
+};
+
+template <int RP>
+__global__ void __launch_bounds__(128, 2) tiled_window_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+                                                                  const __grid_constant__ CUtensorMap tmk,
+                                                                  const __grid_constant__ CUtensorMap tmv,
+                                                                  WindowParams P) {
+    constexpr int NK = 128 + 2 * RP;
+    constexpr int NC = RP / 16 + 1;  // 32-column chunks of one warp's window
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const WindowTcLayout lay(RP);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int L = P.L, K = P.K, r = P.r;
+    const int64_t head = blockIdx.y;
+    const int q0 = blockIdx.x * 128;
+    const int kb0 = q0 - RP;  // key of window column 0
+    const uint32_t sb = smem_u32(smem);
+    const uint32_t q_s = sb + lay.qk_off, k_s = q_s + 16384u, v_s = sb + lay.v_off, p_s = q_s;
+    const uint32_t bar_ld = sb + lay.bar_off, bar_s = bar_ld + 8, bar_o = bar_ld + 16;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + lay.bar_off + 24);
+
+    pdl_launch();
+    if (tid == 0) {
+        umma::mbar_init(bar_ld, 1);
+        umma::mbar_init(bar_s, 1);
+        umma::mbar_init(bar_o, 1);
+        umma::mbar_init_fence();
+        umma::mbar_expect_tx(bar_ld, (uint32_t)(128 + 2 * NK) * 128u);
+        umma::tma_load_3d(q_s, &tmq, 0, q0, (int)head, bar_ld);
+        umma::tma_load_3d(k_s, &tmk, 0, kb0, (int)head, bar_ld);
+        umma::tma_load_3d(v_s, &tmv, 0, kb0, (int)head, bar_ld);
+    }
+    pdl_wait();  // V_cent and the assignments come from earlier kernels
+    __syncwarp();
+    if (warp == 0) umma::tmem_alloc(smem_u32(tslot), 256u);
+    // gather inputs of this thread's row, fetched early
+    const int i = tid, qi = q0 + i;
+    const int ci = qi < L ? P.assign[head * L + qi] : 0;
+    const float4 *vrow = reinterpret_cast<const float4 *>(P.vcent + (head * K + ci) * kD);
+    umma::tc_fence_before();
+    __syncthreads();
+    umma::tc_fence_after();
+    const uint32_t taddr = *tslot;
+
+    const bool ld_ok = __syncthreads_and(umma::mbar_wait(bar_ld, 0));
+    if (tid == 0) {
+        if (ld_ok) {
+            constexpr uint32_t idesc = umma::idesc_bf16_f32(128, NK);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                umma::mma_bf16(taddr, umma::desc_sw128(q_s + (uint32_t)ks * 32u), umma::desc_sw128(k_s + (uint32_t)ks * 32u),
+                               idesc, ks > 0);
+            umma::mma_commit(bar_s);
+        } else {
+            record_error(4, 40);
+        }
+    }
+    const bool s_ok = __syncthreads_and(ld_ok && umma::mbar_wait(bar_s, 0));
+    if (!s_ok && ld_ok && tid == 0) record_error(4, 41);
+    umma::tc_fence_after();
+
+    // Row i's keys: window columns [lo, hi] (inclusive); the warp reads
+    // columns [32 warp, 32 warp + 32 NC).
+    const float csc = P.scale * fused::kLog2e;
+    const int lo = max(i + RP - r, RP - q0), hi = min(i + RP + r, L - 1 - kb0);
+    const int cw = 32 * warp;
+    const uint32_t trow = taddr + ((uint32_t)(32 * warp) << 16);
+    float m = -INFINITY;
+    if (s_ok) {
+#pragma unroll
+        for (int ch = 0; ch < NC; ++ch) {
+            float v[32];
+            umma::tmem_ld32(trow + (uint32_t)(cw + 32 * ch), v);
+            umma::tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int c = cw + 32 * ch + j;
+                if (c >= lo && c <= hi) m = fmaxf(m, v[j]);
+            }
+        }
+    }
+    const float mc = (m == -INFINITY) ? 0.f : m * csc;
+    float l = 0.f;
+    // P row i: zeros outside the warp's columns, exp2 weights inside
+    auto p_chunk = [&](int c8) -> uint32_t {  // byte address of 8-key chunk c8 of row i
+        return p_s + (uint32_t)(c8 >> 3) * 16384u + swz(i, c8 & 7);
+    };
+    if (s_ok) {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        for (int c8 = 0; c8 < NK / 8; ++c8) {
+            if (c8 * 8 >= cw && c8 * 8 < cw + 32 * NC) continue;
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(p_chunk(c8)), "r"(z.x), "r"(z.y), "r"(z.z), "r"(z.w)
+                         : "memory");
+        }
+#pragma unroll
+        for (int ch = 0; ch < NC; ++ch) {
+            float v[32];
+            umma::tmem_ld32(trow + (uint32_t)(cw + 32 * ch), v);
+            umma::tmem_ld_wait();
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                const int c = cw + 32 * ch + j;
+                const float p0 = (c >= lo && c <= hi) ? fused::ex2(fmaf(v[j], csc, -mc)) : 0.f;
+                const float p1 = (c + 1 >= lo && c + 1 <= hi) ? fused::ex2(fmaf(v[j + 1], csc, -mc)) : 0.f;
+                l += p0 + p1;
+                pk[j >> 1] = pack_bf16(p0, p1);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(p_chunk((cw + 32 * ch) / 8 + q)),
+                             "r"(pk[4 * q]), "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
+                             : "memory");
+        }
+    }
+    umma::fence_proxy_async_smem();
+    umma::tc_fence_before();
+    __syncthreads();
+    umma::tc_fence_after();
+    if (tid == 0 && s_ok) {
+        constexpr uint32_t idesc = umma::idesc_bf16_f32_bmn(128, 64);
+#pragma unroll
+        for (int ks = 0; ks < NK / 16; ++ks)
+            umma::mma_bf16(taddr, umma::desc_sw128(p_s + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u),
+                           umma::desc_sw128(v_s + (uint32_t)ks * 2048u), idesc, ks > 0);
+        umma::mma_commit(bar_o);
+    }
+    // V_cent row of this token, pre-scaled by (1 - alpha)
+    float4 g[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) g[u] = __ldg(vrow + u);
+    const bool o_ok = __syncthreads_and(s_ok && umma::mbar_wait(bar_o, 0));
+    if (!o_ok && s_ok && tid == 0) record_error(4, 42);
+    umma::tc_fence_after();
+    if (o_ok) {
+        const float be = 1.f - P.alpha, f = l > 0.f ? P.alpha / l : 0.f;
+        __nv_bfloat16 *orow = P.out + (head * L + qi) * kD;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float o[32];
+            umma::tmem_ld32(trow + (uint32_t)(32 * half), o);
+            umma::tmem_ld_wait();
+            uint32_t w[16];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float4 gv = g[8 * half + u];
+                w[2 * u] = pack_bf16(fmaf(f, o[4 * u + 0], be * gv.x), fmaf(f, o[4 * u + 1], be * gv.y));
+                w[2 * u + 1] = pack_bf16(fmaf(f, o[4 * u + 2], be * gv.z), fmaf(f, o[4 * u + 3], be * gv.w));
+            }
+            if (qi < L) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(orow + 32 * half + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            }
+        }
+    }
+    umma::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        umma::tc_fence_after();
+        umma::tmem_dealloc(taddr, 256u);
+    }
+}
+
 }  // namespace tiled
 }  // namespace ca
