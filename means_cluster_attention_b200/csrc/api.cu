@@ -397,7 +397,7 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         if (ms != CA_OK) return ms;
         Launch pl("tiled_window", st, 4.0 * head_bytes);
         CA_CUDA(launch_pdl(RP == 32 ? tiled::tiled_window_tc_kernel<32> : tiled::tiled_window_tc_kernel<64>,
-                           dim3((L + 127) / 128, (unsigned)NH), dim3(128), tlay.total, st, q128, kmap, vmap, wp));
+                           dim3((L + 127) / 128, (unsigned)NH), dim3(256), tlay.total, st, q128, kmap, vmap, wp));
         pl.after();
     } else {
         const tiled::WindowLayout wlay(K, p.W / 2);

@@ -1046,10 +1046,14 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
 //
 //   S = Q K^T           one thread issues 4 MMAs (M = 128, N = NK, K = 64),
 //                       fp32 scores in tensor memory;
-//   softmax             thread i owns query row i (tensor-memory lane i): its
-//                       warp's 32 + 2 RP columns are read twice (row max,
-//                       then exp2), keys outside |i - j| <= r or [0, L) get
-//                       weight 0; P is rounded to bf16 into shared memory
+//   softmax             query row i is tensor-memory lane i; the 32 + 2 RP
+//                       columns of its warp quarter are split between two
+//                       threads (one per warpgroup) and read twice (row
+//                       max, then exp2), with the partial maxima and sums
+//                       exchanged through shared memory; keys outside
+//                       |i - j| <= r or [0, L) get weight 0, and chunks
+//                       inside every row's band skip the mask; P is
+//                       rounded to bf16 into shared memory
 //                       (over the dead Q and K tiles, K-major, 128-byte
 //                       swizzled blocks of 64 keys);
 //   O = P V             NK / 16 MMAs (M = 128, N = 64), V read N-major as
@@ -1058,28 +1062,30 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
 //                       rounded once to bf16, one 128-byte row per thread.
 struct WindowTcLayout {
     int NK;
-    uint32_t qk_off, v_off, bar_off, total;
+    uint32_t qk_off, v_off, red_off, bar_off, total;
     __host__ __device__ WindowTcLayout(int RP) {
         NK = 128 + 2 * RP;
         qk_off = 0;  // Q (16 KB) then K (NK rows); afterwards P (NK / 64 blocks of 16 KB)
         const uint32_t qk = 16384u + (uint32_t)NK * 128u, pb = (uint32_t)NK / 64u * 16384u;
         v_off = up(qk > pb ? qk : pb, 1024);
-        bar_off = v_off + (uint32_t)NK * 128u;
+        red_off = v_off + (uint32_t)NK * 128u;  // [4][128] floats: partial row maxima and sums
+        bar_off = red_off + 4u * 128u * 4u;
         total = up(bar_off + 32u, 128) + 1024;  // + slack to align the base to 1024 bytes
     }
 };
 
 template <int RP>
-__global__ void __launch_bounds__(128, 2) tiled_window_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+__global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                                                                   const __grid_constant__ CUtensorMap tmk,
                                                                   const __grid_constant__ CUtensorMap tmv,
                                                                   WindowParams P) {
     constexpr int NK = 128 + 2 * RP;
-    constexpr int NC = RP / 16 + 1;  // 32-column chunks of one warp's window
+    constexpr int NC = RP / 16 + 1;    // 32-column chunks of one warp's window
+    constexpr int NC0 = (NC + 1) / 2;  // chunks of warpgroup 0; warpgroup 1 takes the rest
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const WindowTcLayout lay(RP);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, wg = warp >> 2, q4 = warp & 3;
     const int L = P.L, K = P.K, r = P.r;
     const int64_t head = blockIdx.y;
     const int q0 = blockIdx.x * 128;
@@ -1088,6 +1094,7 @@ __global__ void __launch_bounds__(128, 2) tiled_window_tc_kernel(const __grid_co
     const uint32_t q_s = sb + lay.qk_off, k_s = q_s + 16384u, v_s = sb + lay.v_off, p_s = q_s;
     const uint32_t bar_ld = sb + lay.bar_off, bar_s = bar_ld + 8, bar_o = bar_ld + 16;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + lay.bar_off + 24);
+    float *red = reinterpret_cast<float *>(smem + lay.red_off);  // [2][128] partial max, then [2][128] partial sums
 
     pdl_launch();
     if (tid == 0) {
@@ -1103,10 +1110,12 @@ __global__ void __launch_bounds__(128, 2) tiled_window_tc_kernel(const __grid_co
     pdl_wait();  // V_cent and the assignments come from earlier kernels
     __syncwarp();
     if (warp == 0) umma::tmem_alloc(smem_u32(tslot), 256u);
-    // gather inputs of this thread's row, fetched early
-    const int i = tid, qi = q0 + i;
+    // Thread (wg, q4, lane) serves query row i = 32 q4 + lane: warpgroup wg
+    // reads its share of the row's score columns and writes half of its
+    // output row.
+    const int i = 32 * q4 + (tid & 31), qi = q0 + i;
     const int ci = qi < L ? P.assign[head * L + qi] : 0;
-    const float4 *vrow = reinterpret_cast<const float4 *>(P.vcent + (head * K + ci) * kD);
+    const float4 *vrow = reinterpret_cast<const float4 *>(P.vcent + (head * K + ci) * kD) + 8 * wg;
     umma::tc_fence_before();
     __syncthreads();
     umma::tc_fence_after();
@@ -1129,60 +1138,81 @@ __global__ void __launch_bounds__(128, 2) tiled_window_tc_kernel(const __grid_co
     if (!s_ok && ld_ok && tid == 0) record_error(4, 41);
     umma::tc_fence_after();
 
-    // Row i's keys: window columns [lo, hi] (inclusive); the warp reads
-    // columns [32 warp, 32 warp + 32 NC).
+    // Row i's keys: window columns [lo, hi] (inclusive).  The rows of warp
+    // quarter q4 lie in columns [32 q4, 32 q4 + 32 NC); a chunk inside
+    // [lo, hi] needs no mask.
     const float csc = P.scale * fused::kLog2e;
     const int lo = max(i + RP - r, RP - q0), hi = min(i + RP + r, L - 1 - kb0);
-    const int cw = 32 * warp;
-    const uint32_t trow = taddr + ((uint32_t)(32 * warp) << 16);
+    const int cw = 32 * q4;
+    const int ch0 = wg == 0 ? 0 : NC0, ch1 = wg == 0 ? NC0 : NC;
+    const uint32_t trow = taddr + ((uint32_t)(32 * q4) << 16);
     float m = -INFINITY;
     if (s_ok) {
 #pragma unroll
-        for (int ch = 0; ch < NC; ++ch) {
+        for (int ch = 0; ch < NC0; ++ch) {
+            if (ch0 + ch >= ch1) break;  // uniform
+            const int cb = cw + 32 * (ch0 + ch);
             float v[32];
-            umma::tmem_ld32(trow + (uint32_t)(cw + 32 * ch), v);
+            umma::tmem_ld32(trow + (uint32_t)cb, v);
             umma::tmem_ld_wait();
+            if (cb >= lo && cb + 31 <= hi) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int c = cw + 32 * ch + j;
-                if (c >= lo && c <= hi) m = fmaxf(m, v[j]);
+                for (int j = 0; j < 32; ++j) m = fmaxf(m, v[j]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if ((unsigned)(cb + j - lo) <= (unsigned)(hi - lo)) m = fmaxf(m, v[j]);
             }
         }
     }
+    red[wg * 128 + i] = m;
+    __syncthreads();
+    m = fmaxf(red[i], red[128 + i]);
     const float mc = (m == -INFINITY) ? 0.f : m * csc;
     float l = 0.f;
-    // P row i: zeros outside the warp's columns, exp2 weights inside
     auto p_chunk = [&](int c8) -> uint32_t {  // byte address of 8-key chunk c8 of row i
         return p_s + (uint32_t)(c8 >> 3) * 16384u + swz(i, c8 & 7);
     };
     if (s_ok) {
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        for (int c8 = 0; c8 < NK / 8; ++c8) {
-            if (c8 * 8 >= cw && c8 * 8 < cw + 32 * NC) continue;
-            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(p_chunk(c8)), "r"(z.x), "r"(z.y), "r"(z.z), "r"(z.w)
-                         : "memory");
-        }
+        // zeros outside the warp quarter's columns (warpgroup 0 before them,
+        // warpgroup 1 after them)
+        const int z0 = wg == 0 ? 0 : (cw + 32 * NC) / 8, z1 = wg == 0 ? cw / 8 : NK / 8;
+        for (int c8 = z0; c8 < z1; ++c8)
+            asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(p_chunk(c8)), "r"(0u) : "memory");
 #pragma unroll
-        for (int ch = 0; ch < NC; ++ch) {
+        for (int ch = 0; ch < NC0; ++ch) {
+            if (ch0 + ch >= ch1) break;  // uniform
+            const int cb = cw + 32 * (ch0 + ch);
             float v[32];
-            umma::tmem_ld32(trow + (uint32_t)(cw + 32 * ch), v);
+            umma::tmem_ld32(trow + (uint32_t)cb, v);
             umma::tmem_ld_wait();
             uint32_t pk[16];
+            if (cb >= lo && cb + 31 <= hi) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                const int c = cw + 32 * ch + j;
-                const float p0 = (c >= lo && c <= hi) ? fused::ex2(fmaf(v[j], csc, -mc)) : 0.f;
-                const float p1 = (c + 1 >= lo && c + 1 <= hi) ? fused::ex2(fmaf(v[j + 1], csc, -mc)) : 0.f;
-                l += p0 + p1;
-                pk[j >> 1] = pack_bf16(p0, p1);
+                for (int j = 0; j < 32; j += 2) {
+                    const float p0 = fused::ex2(fmaf(v[j], csc, -mc)), p1 = fused::ex2(fmaf(v[j + 1], csc, -mc));
+                    l += p0 + p1;
+                    pk[j >> 1] = pack_bf16(p0, p1);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const bool in0 = (unsigned)(cb + j - lo) <= (unsigned)(hi - lo);
+                    const bool in1 = (unsigned)(cb + j + 1 - lo) <= (unsigned)(hi - lo);
+                    const float p0 = in0 ? fused::ex2(fmaf(v[j], csc, -mc)) : 0.f;
+                    const float p1 = in1 ? fused::ex2(fmaf(v[j + 1], csc, -mc)) : 0.f;
+                    l += p0 + p1;
+                    pk[j >> 1] = pack_bf16(p0, p1);
+                }
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(p_chunk((cw + 32 * ch) / 8 + q)),
-                             "r"(pk[4 * q]), "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(p_chunk(cb / 8 + q)), "r"(pk[4 * q]),
+                             "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
                              : "memory");
         }
     }
+    red[256 + wg * 128 + i] = l;
     umma::fence_proxy_async_smem();
     umma::tc_fence_before();
     __syncthreads();
@@ -1195,33 +1225,30 @@ __global__ void __launch_bounds__(128, 2) tiled_window_tc_kernel(const __grid_co
                            umma::desc_sw128(v_s + (uint32_t)ks * 2048u), idesc, ks > 0);
         umma::mma_commit(bar_o);
     }
-    // V_cent row of this token, pre-scaled by (1 - alpha)
-    float4 g[16];
+    // this thread's half of the token's V_cent row
+    float4 g[8];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) g[u] = __ldg(vrow + u);
+    for (int u = 0; u < 8; ++u) g[u] = __ldg(vrow + u);
+    l = red[256 + i] + red[384 + i];
     const bool o_ok = __syncthreads_and(s_ok && umma::mbar_wait(bar_o, 0));
     if (!o_ok && s_ok && tid == 0) record_error(4, 42);
     umma::tc_fence_after();
     if (o_ok) {
         const float be = 1.f - P.alpha, f = l > 0.f ? P.alpha / l : 0.f;
-        __nv_bfloat16 *orow = P.out + (head * L + qi) * kD;
+        float o[32];
+        umma::tmem_ld32(trow + (uint32_t)(32 * wg), o);
+        umma::tmem_ld_wait();
+        uint32_t w[16];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float o[32];
-            umma::tmem_ld32(trow + (uint32_t)(32 * half), o);
-            umma::tmem_ld_wait();
-            uint32_t w[16];
+        for (int u = 0; u < 8; ++u) {
+            w[2 * u] = pack_bf16(fmaf(f, o[4 * u + 0], be * g[u].x), fmaf(f, o[4 * u + 1], be * g[u].y));
+            w[2 * u + 1] = pack_bf16(fmaf(f, o[4 * u + 2], be * g[u].z), fmaf(f, o[4 * u + 3], be * g[u].w));
+        }
+        if (qi < L) {
+            __nv_bfloat16 *orow = P.out + (head * L + qi) * kD + 32 * wg;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float4 gv = g[8 * half + u];
-                w[2 * u] = pack_bf16(fmaf(f, o[4 * u + 0], be * gv.x), fmaf(f, o[4 * u + 1], be * gv.y));
-                w[2 * u + 1] = pack_bf16(fmaf(f, o[4 * u + 2], be * gv.z), fmaf(f, o[4 * u + 3], be * gv.w));
-            }
-            if (qi < L) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(orow + 32 * half + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-            }
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
     }
     umma::tc_fence_before();
