@@ -353,7 +353,6 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     cp.k = k;
     cp.v = v;
     cp.hi = hi;
-    cp.lo = lo;
     cp.part = cpart;
     cp.L = L;
     cp.K = K;

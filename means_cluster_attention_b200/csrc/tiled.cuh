@@ -590,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
 // centroid_attn_combine_kernel: part[head][chunk][K][64 + 2].
 struct CentroidLayout {
     int Kp;
-    uint32_t slots_off, hi_off, lo_off, ml_off, total;
+    uint32_t slots_off, hi_off, ml_off, total;
     __host__ __device__ CentroidLayout(int K) {
         Kp = kpad(K);
         uint32_t o = 0;
@@ -600,8 +600,6 @@ struct CentroidLayout {
         o += up(slots > comb ? slots : comb, 1024);
         hi_off = o;
         o += (uint32_t)Kp * 128u;
-        lo_off = o;
-        o += (uint32_t)Kp * 128u;
         ml_off = o;
         o += (uint32_t)kWarps * 16u * 2u * 4u;
         total = up(o, 128);
@@ -610,7 +608,7 @@ struct CentroidLayout {
 
 struct CentroidParams {
     const __nv_bfloat16 *k, *v;
-    const __nv_bfloat16 *hi, *lo;  // [NH][Kp][64]
+    const __nv_bfloat16 *hi;       // [NH][Kp][64] centroids rounded to bf16
     float *part;                   // [NH][n_chunks][K][kPartLd]
     int L, K, n_chunks;
     float scale;
@@ -629,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_centroid_kernel(CentroidPar
     const __nv_bfloat16 *kh = P.k + (head * P.L + k0) * kD;
     const __nv_bfloat16 *vh = P.v + (head * P.L + k0) * kD;
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t slot_s = sbase + lay.slots_off, hi_s = sbase + lay.hi_off, lo_s = sbase + lay.lo_off;
+    const uint32_t slot_s = sbase + lay.slots_off, hi_s = sbase + lay.hi_off;
     float *ml = reinterpret_cast<float *>(smem + lay.ml_off);
 
     pdl_launch();
@@ -646,18 +644,20 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_centroid_kernel(CentroidPar
     for (int e = threadIdx.x; e < Kp * 8; e += kThreads) {
         const int kk = e >> 3, ch = e & 7;
         *reinterpret_cast<uint4 *>(smem + lay.hi_off + swz(kk, ch)) = *reinterpret_cast<const uint4 *>(P.hi + (cb + kk) * kD + ch * 8);
-        *reinterpret_cast<uint4 *>(smem + lay.lo_off + swz(kk, ch)) = *reinterpret_cast<const uint4 *>(P.lo + (cb + kk) * kD + ch * 8);
     }
     __syncthreads();
     const int n_cm = Kp / 16, G = kWarps / n_cm, cm = warp / G, kb = warp % G, keys_w = kTile / G;
     const float csc = P.scale * kLog2e;
-    uint32_t ahi[4][4], alo[4][4];
+    // Scores use the centroids rounded once to bf16: the weights P are
+    // rounded to bf16 as well, and the error this adds to a logit
+    // (|mu| |K| 2^-9 / sqrt(d) at worst, far less on average) stays well
+    // below the output tolerance.
+    uint32_t ahi[4][4];
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
         const int m = lane >> 3;
         const int row = cm * 16 + (lane & 7) + ((m & 1) ? 8 : 0);
         ldmatrix_x4(ahi[ks], hi_s + swz(row, 2 * ks + (m >> 1)));
-        ldmatrix_x4(alo[ks], lo_s + swz(row, 2 * ks + (m >> 1)));
     }
     float o_acc[8][4];
 #pragma unroll
@@ -685,8 +685,6 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_centroid_kernel(CentroidPar
                 ldmatrix_x4(bk, kt + swz(key0 + (lane & 7), 4 * kp + (lane >> 3)));
                 mma_16816(sacc[n], ahi[2 * kp], bk[0], bk[1]);
                 mma_16816(sacc[n], ahi[2 * kp + 1], bk[2], bk[3]);
-                mma_16816(sacc[n], alo[2 * kp], bk[0], bk[1]);
-                mma_16816(sacc[n], alo[2 * kp + 1], bk[2], bk[3]);
             }
         }
         float tmax[2] = {-INFINITY, -INFINITY};
@@ -1148,20 +1146,30 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
     const uint32_t trow = taddr + ((uint32_t)(32 * q4) << 16);
     float m = -INFINITY;
     if (s_ok) {
+        // two tensor-memory loads in flight per wait
 #pragma unroll
-        for (int ch = 0; ch < NC0; ++ch) {
-            if (ch0 + ch >= ch1) break;  // uniform
-            const int cb = cw + 32 * (ch0 + ch);
-            float v[32];
-            umma::tmem_ld32(trow + (uint32_t)cb, v);
+        for (int c2 = 0; c2 < NC0; c2 += 2) {
+            const int chA = ch0 + c2, chB = ch0 + c2 + 1;
+            if (chA >= ch1) break;  // uniform
+            float va[32], vb[32];
+            umma::tmem_ld32(trow + (uint32_t)(cw + 32 * chA), va);
+            if (chB < ch1) umma::tmem_ld32(trow + (uint32_t)(cw + 32 * chB), vb);
             umma::tmem_ld_wait();
-            if (cb >= lo && cb + 31 <= hi) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) m = fmaxf(m, v[j]);
-            } else {
+            for (int u = 0; u < 2; ++u) {
+                if (u == 1 && chB >= ch1) break;
+                float *v = u ? vb : va;
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if ((unsigned)(cb + j - lo) <= (unsigned)(hi - lo)) m = fmaxf(m, v[j]);
+                for (int t = 0; t < 32; ++t) asm volatile("" : "+f"(v[t]));  // used only after the wait
+                const int cb = cw + 32 * (u ? chB : chA);
+                if (cb >= lo && cb + 31 <= hi) {
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) m = fmaxf(m, v[t]);
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 32; ++t)
+                        if ((unsigned)(cb + t - lo) <= (unsigned)(hi - lo)) m = fmaxf(m, v[t]);
+                }
             }
         }
     }
@@ -1180,36 +1188,45 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
         for (int c8 = z0; c8 < z1; ++c8)
             asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(p_chunk(c8)), "r"(0u) : "memory");
 #pragma unroll
-        for (int ch = 0; ch < NC0; ++ch) {
-            if (ch0 + ch >= ch1) break;  // uniform
-            const int cb = cw + 32 * (ch0 + ch);
-            float v[32];
-            umma::tmem_ld32(trow + (uint32_t)cb, v);
+        for (int c2 = 0; c2 < NC0; c2 += 2) {
+            const int chA = ch0 + c2, chB = ch0 + c2 + 1;
+            if (chA >= ch1) break;  // uniform
+            float va[32], vb[32];
+            umma::tmem_ld32(trow + (uint32_t)(cw + 32 * chA), va);
+            if (chB < ch1) umma::tmem_ld32(trow + (uint32_t)(cw + 32 * chB), vb);
             umma::tmem_ld_wait();
-            uint32_t pk[16];
-            if (cb >= lo && cb + 31 <= hi) {
 #pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    const float p0 = fused::ex2(fmaf(v[j], csc, -mc)), p1 = fused::ex2(fmaf(v[j + 1], csc, -mc));
-                    l += p0 + p1;
-                    pk[j >> 1] = pack_bf16(p0, p1);
-                }
-            } else {
+            for (int u = 0; u < 2; ++u) {
+                if (u == 1 && chB >= ch1) break;
+                float *v = u ? vb : va;
 #pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    const bool in0 = (unsigned)(cb + j - lo) <= (unsigned)(hi - lo);
-                    const bool in1 = (unsigned)(cb + j + 1 - lo) <= (unsigned)(hi - lo);
-                    const float p0 = in0 ? fused::ex2(fmaf(v[j], csc, -mc)) : 0.f;
-                    const float p1 = in1 ? fused::ex2(fmaf(v[j + 1], csc, -mc)) : 0.f;
-                    l += p0 + p1;
-                    pk[j >> 1] = pack_bf16(p0, p1);
+                for (int t = 0; t < 32; ++t) asm volatile("" : "+f"(v[t]));
+                const int cb = cw + 32 * (u ? chB : chA);
+                uint32_t pk[16];
+                if (cb >= lo && cb + 31 <= hi) {
+#pragma unroll
+                    for (int t = 0; t < 32; t += 2) {
+                        const float p0 = fused::ex2(fmaf(v[t], csc, -mc)), p1 = fused::ex2(fmaf(v[t + 1], csc, -mc));
+                        l += p0 + p1;
+                        pk[t >> 1] = pack_bf16(p0, p1);
+                    }
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 32; t += 2) {
+                        const bool in0 = (unsigned)(cb + t - lo) <= (unsigned)(hi - lo);
+                        const bool in1 = (unsigned)(cb + t + 1 - lo) <= (unsigned)(hi - lo);
+                        const float p0 = in0 ? fused::ex2(fmaf(v[t], csc, -mc)) : 0.f;
+                        const float p1 = in1 ? fused::ex2(fmaf(v[t + 1], csc, -mc)) : 0.f;
+                        l += p0 + p1;
+                        pk[t >> 1] = pack_bf16(p0, p1);
+                    }
                 }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(p_chunk(cb / 8 + q)), "r"(pk[4 * q]),
+                                 "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
+                                 : "memory");
             }
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(p_chunk(cb / 8 + q)), "r"(pk[4 * q]),
-                             "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
-                             : "memory");
         }
     }
     red[256 + wg * 128 + i] = l;
@@ -1238,6 +1255,8 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
         float o[32];
         umma::tmem_ld32(trow + (uint32_t)(32 * wg), o);
         umma::tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) asm volatile("" : "+f"(o[t]));
         uint32_t w[16];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
