@@ -25,7 +25,20 @@
  * those fp32 centroids exactly: an fp32 pass with a rigorous error bound
  * settles almost every token, and the few whose two best candidates lie
  * within that bound are re-measured in fp64, in the expanded form above with
- * index-order sums.
+ * index-order sums.  On the bf16 paths the contractions run on tensor cores
+ * with bf16 operands and fp32 accumulation: the distance pass splits each
+ * fp32 centroid into two bf16 terms; the centroid-attention scores use the
+ * centroids split in two terms (one CTA per head) or rounded once to bf16
+ * (long sequences); the attention weights are rounded to bf16 for the P V
+ * products.
+ *
+ * Execution.  On sm_100a the long-sequence bf16 path stages query, key and
+ * value tiles with TMA (tensor maps over the caller's q, k, v) and issues its
+ * distance and window-attention contractions as tcgen05.mma with tensor-
+ * memory accumulators; its kernels are chained with programmatic dependent
+ * launch (a kernel may start before its predecessor on the stream ends and
+ * waits for it before reading its results; the first kernel of a call waits
+ * for all earlier work on the stream).
  *
  * Conventions for every entry point below:
  *   - Tensors are dense, row-major [B, H, L, d] (d fastest), as produced by
@@ -200,7 +213,8 @@ const char *ca_version(void);
  * output the kernel must touch).  Kernel names: the fused one-CTA-per-head
  * kernel (bf16, L <= 512, K <= 64, floor(W/2) <= 16) is "fused_forward";
  * the tiled bf16 path (K <= 64, floor(W/2) <= 128) launches "tiled_init",
- * "tiled_assign", "tiled_update", "tiled_centroid", "tiled_combine" and
+ * then per Lloyd iteration "tiled_dead", "tiled_assign" and
+ * "tiled_update", then "tiled_centroid", "tiled_combine" and
  * "tiled_window"; every other case runs the general path "kmeans_init",
  * "kmeans_assign", "kmeans_update", "centroid_attn", "centroid_combine" and
  * "window_blend". */

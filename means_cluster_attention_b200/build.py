@@ -37,11 +37,12 @@ def sources() -> list:
 
 # Source files each profiled kernel is built from (its own code and the
 # headers it includes), for deciding whether recorded counters still apply.
+_TILED = ["tiled.cuh", "fused.cuh", "kmeans_tile.cuh", "umma.cuh", "mma.cuh", "common.cuh"]
 KERNEL_SOURCES = {
-    "fused_forward": ["fused.cuh", "mma.cuh", "common.cuh"],
-    "tiled_assign": ["tiled.cuh", "fused.cuh", "mma.cuh", "common.cuh"],
-    "tiled_window": ["tiled.cuh", "fused.cuh", "mma.cuh", "common.cuh"],
-    "tiled_centroid": ["tiled.cuh", "fused.cuh", "mma.cuh", "common.cuh"],
+    "fused_forward": ["fused.cuh", "kmeans_tile.cuh", "mma.cuh", "common.cuh"],
+    "tiled_assign": _TILED,
+    "tiled_window": _TILED,
+    "tiled_centroid": _TILED,
 }
 
 

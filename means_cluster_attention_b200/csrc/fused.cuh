@@ -26,13 +26,13 @@
 // copies of a lower-index centroid can never win (their distances are equal
 // and the lower index takes the tie) and are excluded up front.
 //
-// Member sums: tokens are grouped by cluster with a counting sort and each
-// warp walks a contiguous slice of the sorted tokens, turning bf16 values
-// into doubles with integer operations and adding in fp64; a later iteration
-// in which few tokens change cluster only subtracts / adds those.  The sums
-// are exact for any input whose non-zero magnitudes lie within 2^-27 .. 16,
-// so the centroid mu_k = fp32(sum / max(1, count)) does not depend on the
-// order of the adds.
+// Member sums (kmeans_tile.cuh): tokens are grouped by cluster with a
+// counting sort and each warp walks a contiguous slice of the sorted tokens,
+// two tokens per step, adding exact doubles in fp64; a later iteration in
+// which few tokens change cluster only subtracts / adds those.  The sums are
+// exact for any input whose non-zero magnitudes lie within 2^-27 .. 16, so
+// the centroid mu_k = fp32(sum / max(1, count)) does not depend on the order
+// of the adds.
 #pragma once
 
 #include <type_traits>

@@ -1,22 +1,35 @@
-// Tiled cluster-attention kernels for long sequences (bf16): the same phase
-// code as the fused one-CTA-per-head kernel, cut into launches that split a
-// head over several CTAs.
+// Tiled cluster-attention kernels for long sequences (bf16): a head is split
+// over several CTAs.
 //
-//   tiled_mu_kernel        (K, heads)      mu = strided init, or the update
+//   tiled_mu_kernel        (Kp, heads)     mu = strided init, or the update
 //                                          mu_k = fp32(sum_k / max(1, count_k))
 //                                          from per-tile exact partial sums;
 //                                          also the bf16 hi/lo split, |mu|^2
 //                                          and a row hash for each centroid.
+//   tiled_dead_kernel      (Kp, heads)     marks centroids that are bitwise
+//                                          copies of a lower-index one (they
+//                                          can never win the argmin) and
+//                                          records max |mu|^2 per head.
 //   tiled_assign_kernel    (tiles, heads)  one Lloyd assignment for a tile of
-//                                          512 queries (tensor-core distances,
-//                                          exact argmin) and the tile's exact
-//                                          fp64 member sums.
+//                                          512 queries: TMA-staged queries,
+//                                          distances on tcgen05 (tensor-memory
+//                                          accumulators), certified argmin,
+//                                          exact fp64 re-measure of ambiguous
+//                                          tokens, the tile's exact member sums.
 //   tiled_centroid_kernel  (chunks, heads) partial softmax state of every
 //                                          centroid over 512 keys;
 //   tiled_combine_kernel   (K, heads)      combines the chunk states into
 //                                          V_cent.
-//   tiled_window_kernel    (blocks, heads) clipped window attention for 128
-//                                          queries, gather V_cent[c_i], blend.
+//   tiled_window_tc_kernel (blocks, heads) clipped window attention for 128
+//                                          queries on tcgen05 (radius <= 64),
+//                                          gather V_cent[c_i], blend;
+//   tiled_window_kernel    (blocks, heads) the same on mma.sync for radii up
+//                                          to 128.
+//
+// Consecutive kernels are chained with programmatic dependent launch: each
+// lets its successor start early, and the successor touches only the
+// forward's inputs (q, k, v) and its own shared / tensor memory before
+// waiting for its predecessor (pdl_wait).
 //
 // Model card "Hooshaai/distilbert-sst2-cluster-attention", Architecture
 // Overview and Mathematical Formulation section 1; "Hooshaai/svd-sst2-
