@@ -92,6 +92,59 @@ __device__ __forceinline__ int remeasure_token(const unsigned char *qbytes, int 
     return bk;
 }
 
+// Fast exact decision among a token's candidate centroids (bit k of cand
+// set, lowest first).  Each distance D_k = (|Q|^2 + |mu_k|^2) - 2 Q.mu_k is
+// formed in fp64 with warp-tree sums (lane l holds coordinates 2l, 2l+1;
+// every product is exact).  Whatever the order of its sums, a computed D_k
+// lies within 2^-45 (|Q|^2 + |mu_k|^2) of the exact value: 64 summands
+// give at most 64 u of the sum of magnitudes per dot product (u = 2^-53),
+// |Q.mu| <= (|Q|^2 + |mu|^2) / 2, and two more roundings add u each, so
+// 67 u (|Q| + |mu|)^2 <= 2^-45 (|Q|^2 + |mu|^2); E_k takes twice that
+// (2^-44) to cover the roundings of the gap tests themselves.  The
+// index-order distances of the re-measure (and of the fp64 oracle) obey the
+// same bound, so when min over k != b of (D_k - 2 E_k) exceeds D_b + 2 E_b
+// the lowest-k argmin
+// b of the tree distances is the argmin of the index-order ones, with no
+// tie.  Returns b and sets certain; when certain is false the caller takes
+// the index-order re-measure.  The result is the same on every lane.
+template <typename MuAt>
+__device__ __forceinline__ int decide_candidates(const unsigned char *qbytes, int row, const uint32_t *cand, int n_words,
+                                                 const uint8_t *dead, MuAt mu, int lane, bool &certain) {
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(qbytes + swz(row, lane >> 2) + (lane & 3) * 4);
+    const double q0 = bf16_to_f64(w & 0xffffu), q1 = bf16_to_f64(w >> 16);
+    auto tree = [](double x) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        return x;
+    };
+    const double qq = tree(__fma_rn(q0, q0, q1 * q1));
+    double bd = INFINITY, be = 0.0, chall = INFINITY;
+    int bk = -1;
+    for (int wi = 0; wi < n_words; ++wi) {
+        uint32_t bits = cand[wi];
+        while (bits) {
+            const int k = wi * 32 + __ffs(bits) - 1;
+            bits &= bits - 1u;
+            if (dead[k]) continue;
+            const double m0 = mu(k, 2 * lane), m1 = mu(k, 2 * lane + 1);
+            const double qm = tree(__fma_rn(q0, m0, q1 * m1));
+            const double mm = tree(__fma_rn(m0, m0, m1 * m1));
+            const double D = __dsub_rn(__dadd_rn(qq, mm), __dmul_rn(2.0, qm));
+            const double E = ldexp(qq + mm, -44);  // twice the bound: room for the roundings of the gap tests
+            if (D < bd) {
+                if (bk >= 0) chall = fmin(chall, bd - 2.0 * be);
+                bd = D;
+                be = E;
+                bk = k;
+            } else {
+                chall = fmin(chall, D - 2.0 * E);
+            }
+        }
+    }
+    certain = bk >= 0 && chall > bd + 2.0 * be;
+    return bk;
+}
+
 // Counting sort of up to 32 * (number of chunks) tokens by cluster: cs[i] is
 // token i's cluster (0xFF for no token), cnt[] (Kp <= 64 entries, zero on
 // entry) receives the counts; perm[] and sc[] receive the tokens and their

@@ -259,8 +259,8 @@ __global__ void __launch_bounds__(64) tiled_combine_kernel(int K, int n_chunks, 
 // max|mu|^2) covers it threefold.
 struct AssignLayout {
     int Kp;
-    uint32_t q_off, r_off, mu_off, mm_off, dead_off, cnt_off, c_off, sc_off, cprev_off, list_off, perm_off,
-        misc_off, bar_off, total;
+    uint32_t q_off, r_off, mu_off, mm_off, dead_off, cnt_off, c_off, sc_off, cprev_off, list_off, lmask_off,
+        perm_off, misc_off, bar_off, total;
     __host__ __device__ AssignLayout(int K) {
         Kp = kpad(K);
         uint32_t o = 0;
@@ -289,6 +289,8 @@ struct AssignLayout {
         o += (uint32_t)kTileQ;
         list_off = o;
         o += (uint32_t)kTileQ * 2u;
+        lmask_off = o;  // candidate bits of each listed token (two words)
+        o += (uint32_t)kTileQ * 8u;
         perm_off = o;
         o += (uint32_t)kTileQ * 2u;
         misc_off = o;
@@ -354,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     uint8_t *sc = smem + lay.sc_off;
     uint8_t *cprev = smem + lay.cprev_off;
     uint16_t *list = reinterpret_cast<uint16_t *>(smem + lay.list_off);
+    uint32_t *lmask = reinterpret_cast<uint32_t *>(smem + lay.lmask_off);
     uint16_t *perm = reinterpret_cast<uint16_t *>(smem + lay.perm_off);
     int *misc = reinterpret_cast<int *>(smem + lay.misc_off);
     constexpr int mu_ld = 65;
@@ -500,7 +503,8 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
                     m1b = fminf(m1b, fminf(sv[4 * k4 + 2], sv[4 * k4 + 3]));
                 }
                 const float m1 = fminf(m1a, m1b);
-                const float thr = m1 + 2.f * (kEps * fmaf(qn[mi], mun_max, mm_max));
+                const float E = kEps * fmaf(qn[mi], mun_max, mm_max);
+                const float thr = m1 + 2.f * E;
                 uint32_t bits[(KP + 31) / 32];
 #pragma unroll
                 for (int w2 = 0; w2 < (KP + 31) / 32; ++w2) bits[w2] = 0u;
@@ -513,7 +517,22 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
                     if (bits[w2]) c = w2 * 32 + __ffs(bits[w2]) - 1;
                 }
                 cs[row] = (uint8_t)(c < 0 ? 0 : c);
-                if (n != 1) list[atomicAdd(&misc[0], 1)] = (uint16_t)row;
+                if (n != 1) {
+                    // ambiguous: the candidates for the exact decision are
+                    // every k with s_k <= m1 + 3E, so any other centroid is
+                    // worse than the fp32 winner by at least E in exact
+                    // arithmetic
+                    const float thr3 = m1 + 3.f * E;
+                    uint32_t b3[(KP + 31) / 32];
+#pragma unroll
+                    for (int w2 = 0; w2 < (KP + 31) / 32; ++w2) b3[w2] = 0u;
+#pragma unroll
+                    for (int k = 0; k < KP; ++k) b3[k >> 5] |= (sv[k] <= thr3 ? 1u : 0u) << (k & 31);
+                    const int e = atomicAdd(&misc[0], 1);
+                    list[e] = (uint16_t)row;
+#pragma unroll
+                    for (int w2 = 0; w2 < (KP + 31) / 32; ++w2) lmask[e * 2 + w2] = b3[w2];
+                }
             }
         }
     }
@@ -527,8 +546,10 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     const int n_ref = misc[0];
     for (int e = warp; e < n_ref; e += kWarps) {
         const int row = list[e];
-        int bk = tile::remeasure_token<(KP > 32)>(qbytes, row, Kp, dead,
-                                                  [&](int k, int j) { return (double)mu[k * mu_ld + j]; }, lane);
+        auto mu_at = [&](int k, int j) { return (double)mu[k * mu_ld + j]; };
+        bool certain;
+        int bk = tile::decide_candidates(qbytes, row, lmask + 2 * e, (KP + 31) / 32, dead, mu_at, lane, certain);
+        if (!certain) bk = tile::remeasure_token<(KP > 32)>(qbytes, row, Kp, dead, mu_at, lane);
         if (lane == 0) {
             if (bk >= K) {
                 record_error(5, 3);

@@ -242,3 +242,45 @@ def test_tiled_forced_ties_across_tiles():
                                                       iters=w.iters, W=w.W, alpha=w.alpha, hist=True)
     np.testing.assert_array_equal(g["hist"], ref_hist)
     np.testing.assert_array_equal(g["cent"], ref_cent)
+
+
+# Window radii around the tensor-core window kernel's key windows (radius
+# <= 32 and <= 64) and the mma.sync kernel beyond, with a ragged last block;
+# alpha = 1 leaves only the window branch in the output.
+@pytest.mark.parametrize("W", [2, 62, 63, 64, 66, 127, 128, 129, 130])
+def test_tiled_window_radius_boundaries(W):
+    w = Workload("tiled_win", 1, 2, 700, 64, 8, 1, W, 1.0, "bf16", "normal")
+    x = make_inputs(w, seed=W)
+    g = run_gpu(x, "bf16", w.K, w.iters, w.W, w.alpha)
+    ref_out, _, _, _ = oracle.forward(x["q64"], x["k64"], x["v64"], K=w.K, iters=w.iters, W=w.W, alpha=w.alpha)
+    err = float(np.abs(g["out"] - ref_out).max())
+    assert err <= TOL["bf16"], f"W={W}: {err}"
+
+
+def test_tiled_exact_ties_between_distinct_centroids():
+    """Strided starting centroids e1, -e1, 3e3, -3e3 and tokens e2 or 0:
+    every token is exactly equidistant from the first two centroids, so the
+    exact decision cannot be certified from rounded distances and must fall
+    back to the index-order comparison, where the lower index wins."""
+    from means_cluster_attention_b200.inputs import bf16_bits_to_f64, bf16_round_bits
+    L, K = 600, 4
+    q = np.zeros((1, 1, L, 64), dtype=np.float32)
+    q[0, 0, 1::2, 1] = 1.0                      # e2 on odd positions, 0 on even ones
+    rows = [(k * L) // K for k in range(K)]
+    for r_, (dim, val) in zip(rows, [(0, 1.0), (0, -1.0), (2, 3.0), (2, -3.0)]):
+        q[0, 0, r_, :] = 0.0
+        q[0, 0, r_, dim] = val
+    rng = np.random.default_rng(5)
+    x = {}
+    for name, a in (("q", q), ("k", rng.standard_normal(q.shape, dtype=np.float32)),
+                    ("v", rng.standard_normal(q.shape, dtype=np.float32))):
+        x[name] = bf16_round_bits(a)
+        x[name + "64"] = bf16_bits_to_f64(x[name])
+    g = run_gpu(x, "bf16", K, 1, 8, 0.5, hist=True)
+    _, ref_assign, ref_cent, ref_hist = oracle.forward(x["q64"], x["k64"], x["v64"], K=K, iters=1, W=8,
+                                                      alpha=0.5, hist=True)
+    np.testing.assert_array_equal(g["hist"], ref_hist)
+    np.testing.assert_array_equal(g["assign"], ref_assign)
+    np.testing.assert_array_equal(g["cent"], ref_cent)
+    tokens = [i for i in range(L) if i not in rows]
+    assert (ref_assign[0, 0, tokens] == 0).all()
