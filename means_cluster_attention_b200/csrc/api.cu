@@ -389,14 +389,15 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         // tensor-core window kernel: the key window [q0 - RP, q0 + 127 + RP]
         const int RP = wp.r <= 32 ? 32 : 64;
         const tiled::WindowTcLayout tlay(RP);
-        CUtensorMap kmap, vmap, q128;
+        CUtensorMap kmap, vmap, q128, o128;
         ca_status ms = encode_rows_map(&q128, q, NH, L, 128);
         if (ms == CA_OK) ms = encode_rows_map(&kmap, k, NH, L, tlay.NK);
         if (ms == CA_OK) ms = encode_rows_map(&vmap, v, NH, L, tlay.NK);
+        if (ms == CA_OK) ms = encode_rows_map(&o128, out, NH, L, 128);
         if (ms != CA_OK) return ms;
         Launch pl("tiled_window", st, 4.0 * head_bytes);
         CA_CUDA(launch_pdl(RP == 32 ? tiled::tiled_window_tc_kernel<32> : tiled::tiled_window_tc_kernel<64>,
-                           dim3((L + 127) / 128, (unsigned)NH), dim3(256), tlay.total, st, q128, kmap, vmap, wp));
+                           dim3((L + 127) / 128, (unsigned)NH), dim3(256), tlay.total, st, q128, kmap, vmap, o128, wp));
         pl.after();
     } else {
         const tiled::WindowLayout wlay(K, p.W / 2);

@@ -92,8 +92,8 @@ __device__ __forceinline__ int remeasure_token(const unsigned char *qbytes, int 
     return bk;
 }
 
-// Fast exact decision among a token's candidate centroids (bit k of cand
-// set, lowest first).  Each distance D_k = (|Q|^2 + |mu_k|^2) - 2 Q.mu_k is
+// Fast exact decision among a token's candidate centroids (bit k of the
+// 64-bit set cand1:cand0, lowest first).  Each distance D_k = (|Q|^2 + |mu_k|^2) - 2 Q.mu_k is
 // formed in fp64 with warp-tree sums (lane l holds coordinates 2l, 2l+1;
 // every product is exact).  Whatever the order of its sums, a computed D_k
 // lies within 2^-45 (|Q|^2 + |mu_k|^2) of the exact value: 64 summands
@@ -108,7 +108,7 @@ __device__ __forceinline__ int remeasure_token(const unsigned char *qbytes, int 
 // tie.  Returns b and sets certain; when certain is false the caller takes
 // the index-order re-measure.  The result is the same on every lane.
 template <typename MuAt>
-__device__ __forceinline__ int decide_candidates(const unsigned char *qbytes, int row, const uint32_t *cand, int n_words,
+__device__ __forceinline__ int decide_candidates(const unsigned char *qbytes, int row, uint32_t cand0, uint32_t cand1,
                                                  const uint8_t *dead, MuAt mu, int lane, bool &certain) {
     const uint32_t w = *reinterpret_cast<const uint32_t *>(qbytes + swz(row, lane >> 2) + (lane & 3) * 4);
     const double q0 = bf16_to_f64(w & 0xffffu), q1 = bf16_to_f64(w >> 16);
@@ -120,8 +120,9 @@ __device__ __forceinline__ int decide_candidates(const unsigned char *qbytes, in
     const double qq = tree(__fma_rn(q0, q0, q1 * q1));
     double bd = INFINITY, be = 0.0, chall = INFINITY;
     int bk = -1;
-    for (int wi = 0; wi < n_words; ++wi) {
-        uint32_t bits = cand[wi];
+#pragma unroll
+    for (int wi = 0; wi < 2; ++wi) {
+        uint32_t bits = wi ? cand1 : cand0;
         while (bits) {
             const int k = wi * 32 + __ffs(bits) - 1;
             bits &= bits - 1u;

@@ -548,7 +548,8 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
         const int row = list[e];
         auto mu_at = [&](int k, int j) { return (double)mu[k * mu_ld + j]; };
         bool certain;
-        int bk = tile::decide_candidates(qbytes, row, lmask + 2 * e, (KP + 31) / 32, dead, mu_at, lane, certain);
+        int bk = tile::decide_candidates(qbytes, row, lmask[2 * e], KP > 32 ? lmask[2 * e + 1] : 0u, dead, mu_at, lane,
+                                         certain);
         if (!certain) bk = tile::remeasure_token<(KP > 32)>(qbytes, row, Kp, dead, mu_at, lane);
         if (lane == 0) {
             if (bk >= K) {
@@ -1110,6 +1111,7 @@ template <int RP>
 __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                                                                   const __grid_constant__ CUtensorMap tmk,
                                                                   const __grid_constant__ CUtensorMap tmv,
+                                                                  const __grid_constant__ CUtensorMap tmo,
                                                                   WindowParams P) {
     constexpr int NK = 128 + 2 * RP;
     constexpr int NC = RP / 16 + 1;    // 32-column chunks of one warp's window
@@ -1297,19 +1299,26 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
             w[2 * u] = pack_bf16(fmaf(f, o[4 * u + 0], be * g[u].x), fmaf(f, o[4 * u + 1], be * g[u].y));
             w[2 * u + 1] = pack_bf16(fmaf(f, o[4 * u + 2], be * g[u].z), fmaf(f, o[4 * u + 3], be * g[u].w));
         }
-        if (qi < L) {
-            __nv_bfloat16 *orow = P.out + (head * L + qi) * kD + 32 * wg;
+        // the output tile, 128-byte swizzled over the dead P block 0, then
+        // one TMA store (rows past L are clipped)
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4 *>(orow + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-        }
+        for (int q = 0; q < 4; ++q)
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(p_s + swz(i, 4 * wg + q)), "r"(w[4 * q]),
+                         "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
+                         : "memory");
     }
+    umma::fence_proxy_async_smem();
     umma::tc_fence_before();
     __syncthreads();
+    if (tid == 0 && o_ok) {
+        umma::tma_store_3d(&tmo, 0, q0, (int)head, p_s);
+        umma::tma_store_commit();
+    }
     if (warp == 0) {
         umma::tc_fence_after();
         umma::tmem_dealloc(taddr, 256u);
     }
+    if (tid == 0 && o_ok) umma::tma_store_wait_read();  // shared memory stays live until read
 }
 
 }  // namespace tiled

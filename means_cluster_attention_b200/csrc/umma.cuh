@@ -69,6 +69,19 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int 
         : "memory");
 }
 
+// 3-D tiled TMA store of box {64, rows, 1} from shared memory to (x, y, z),
+// x = 0 and y >= 0; rows past the tensor's extent are not written.  Groups
+// with the stores issued before it by this thread (commit / wait below).
+__device__ __forceinline__ void tma_store_3d(const void *tmap, int x, int y, int z, uint32_t src) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(x), "r"(y), "r"(z), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until every committed store has finished reading shared memory.
+__device__ __forceinline__ void tma_store_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 // Shared-memory matrix descriptor of a K-major, 128-byte-swizzled operand
 // starting at saddr (the 8-row groups 1024 bytes apart).  Stepping K by 16
 // bf16 elements advances saddr by 32 bytes.
