@@ -402,8 +402,6 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         if (threadIdx.x == 0) misc[1] = 0;
         // Lane k holds centroid k (and k + 32 when Kp = 64); the chains of
         // the second set are only run when that set exists.
-        // Lane k holds centroid k (and k + 32 when Kp = 64); the chains of
-        // the second set are only run when that set exists.
         auto mu_at = [&](int k, int j) { return mu64[k * 65 + j]; };
         for (int e = warp; e < n_ref; e += kWarps) {
             const int row = list[e];
