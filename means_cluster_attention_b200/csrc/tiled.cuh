@@ -80,66 +80,73 @@ struct MuParams {
     int L, K, Kp, n_tiles, init;
 };
 
-// grid (Kp, NH), 256 threads: thread (g4, j) adds tiles g4, g4+4, ... of
-// coordinate j of centroid k; the four exact partial sums are then added in
-// fixed order by group 0, which finalises the centroid row.
+// grid (Kp, NH), 256 threads: thread (g8, jp) adds tiles g8, g8+8, ... of
+// coordinates 2 jp and 2 jp + 1 of centroid k (16-byte loads); thread j of
+// the first 64 then adds the eight exact partial sums of coordinate j in
+// group order and finalises it.
 __global__ void __launch_bounds__(256) tiled_mu_kernel(MuParams P) {
-    __shared__ double red_s[3][64];
-    __shared__ int red_c[4];
+    __shared__ double2 red_s[8][32];
+    __shared__ int red_c[8];
     __shared__ float red_sq[2];
     __shared__ uint32_t red_h[2];
-    const int k = blockIdx.x, j = threadIdx.x & 63, g4 = threadIdx.x >> 6;
-    const int lane = threadIdx.x & 31, wid = (threadIdx.x >> 5) & 1;
+    const int k = blockIdx.x, jp = threadIdx.x & 31, g8 = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
     const int64_t head = blockIdx.y;
     const int64_t kb = head * P.Kp + k;
     pdl_launch();
     pdl_wait();
-    double s = 0.0;
+    double2 s = make_double2(0.0, 0.0);
     int cnt = 0;
     if (!P.init && k < P.K) {
-        for (int tt = g4; tt < P.n_tiles; tt += 4) {
-            s += P.part_sum[(kb * P.n_tiles + tt) * kD + j];
-            if (j == 0) cnt += P.part_cnt[kb * P.n_tiles + tt];
+        for (int tt = g8; tt < P.n_tiles; tt += 8) {
+            const double2 v = reinterpret_cast<const double2 *>(P.part_sum + (kb * P.n_tiles + tt) * kD)[jp];
+            s.x += v.x;
+            s.y += v.y;
+            if (jp == 0) cnt += P.part_cnt[kb * P.n_tiles + tt];
         }
     }
-    if (g4 > 0) red_s[g4 - 1][j] = s;
-    if (j == 0) red_c[g4] = cnt;
+    red_s[g8][jp] = s;
+    if (jp == 0) red_c[g8] = cnt;
     __syncthreads();
-    if (g4 != 0) return;
-    {
-        float x = 0.f;
-        if (k < P.K) {
-            if (P.init) {
-                const int64_t row = ((int64_t)k * P.L) / P.K;
-                x = __bfloat162float(P.q[(head * P.L + row) * kD + j]);
-            } else {
-                const double tot = ((s + red_s[0][j]) + red_s[1][j]) + red_s[2][j];
-                const int n = red_c[0] + red_c[1] + red_c[2] + red_c[3];
-                x = __double2float_rn(tot / (double)(n > 1 ? n : 1));
-            }
-        }
-        const int64_t o = kb * kD + j;
-        P.mu[o] = x;
-        const __nv_bfloat16 h = __float2bfloat16_rn(x);
-        P.hi[o] = h;
-        P.lo[o] = __float2bfloat16_rn(x - __bfloat162float(h));
-        if (P.cent_out && k < P.K) P.cent_out[(head * P.K + k) * kD + j] = x;
-        float sq = x * x;
-        uint32_t hv = __float_as_uint(x) * (0x9E3779B1u + 2u * (uint32_t)j) + (uint32_t)j * 0xC2B2AE3Du;
+    if (threadIdx.x >= 64) return;
+    // thread j (< 64) finalises coordinate j
+    const int j = threadIdx.x, wid = j >> 5;
+    float x = 0.f;
+    if (k < P.K) {
+        if (P.init) {
+            const int64_t row = ((int64_t)k * P.L) / P.K;
+            x = __bfloat162float(P.q[(head * P.L + row) * kD + j]);
+        } else {
+            double tot = 0.0;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            sq += __shfl_xor_sync(0xffffffffu, sq, off);
-            hv += __shfl_xor_sync(0xffffffffu, hv, off);
+            for (int g = 0; g < 8; ++g) tot += (j & 1) ? red_s[g][j >> 1].y : red_s[g][j >> 1].x;
+            int n = 0;
+#pragma unroll
+            for (int g = 0; g < 8; ++g) n += red_c[g];
+            x = __double2float_rn(tot / (double)(n > 1 ? n : 1));
         }
-        if (lane == 0) {
-            red_sq[wid] = sq;
-            red_h[wid] = hv;
-        }
-        asm volatile("bar.sync 1, 64;");
-        if (j == 0) {
-            P.mm[kb] = red_sq[0] + red_sq[1];
-            P.hash[kb] = red_h[0] + red_h[1];
-        }
+    }
+    const int64_t o = kb * kD + j;
+    P.mu[o] = x;
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    P.hi[o] = h;
+    P.lo[o] = __float2bfloat16_rn(x - __bfloat162float(h));
+    if (P.cent_out && k < P.K) P.cent_out[(head * P.K + k) * kD + j] = x;
+    float sq = x * x;
+    uint32_t hv = __float_as_uint(x) * (0x9E3779B1u + 2u * (uint32_t)j) + (uint32_t)j * 0xC2B2AE3Du;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        hv += __shfl_xor_sync(0xffffffffu, hv, off);
+    }
+    if (lane == 0) {
+        red_sq[wid] = sq;
+        red_h[wid] = hv;
+    }
+    asm volatile("bar.sync 1, 64;");
+    if (j == 0) {
+        P.mm[kb] = red_sq[0] + red_sq[1];
+        P.hash[kb] = red_h[0] + red_h[1];
     }
 }
 
