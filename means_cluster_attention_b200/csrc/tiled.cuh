@@ -1121,8 +1121,7 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
                                                                   const __grid_constant__ CUtensorMap tmo,
                                                                   WindowParams P) {
     constexpr int NK = 128 + 2 * RP;
-    constexpr int NC = RP / 16 + 1;    // 32-column chunks of one warp's window
-    constexpr int NC0 = (NC + 1) / 2;  // chunks of warpgroup 0; warpgroup 1 takes the rest
+    constexpr int NC = RP / 16 + 1;    // 32-column chunks of one warp quarter's window
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const WindowTcLayout lay(RP);
@@ -1180,39 +1179,39 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
     umma::tc_fence_after();
 
     // Row i's keys: window columns [lo, hi] (inclusive).  The rows of warp
-    // quarter q4 lie in columns [32 q4, 32 q4 + 32 NC); a chunk inside
-    // [lo, hi] needs no mask.
+    // quarter q4 lie in columns [32 q4, 32 q4 + 32 NC); warpgroup wg takes
+    // the half [32 q4 + HALF wg, + HALF) and reads it from tensor memory
+    // once (16-column pieces, one wait); a piece inside [lo, hi] needs no
+    // mask.
+    constexpr int HALF = 16 * NC;         // 80 (RP = 64) or 48 (RP = 32) columns per thread
+    constexpr int NP = HALF / 16;         // 16-column pieces per thread
     const float csc = P.scale * fused::kLog2e;
     const int lo = max(i + RP - r, RP - q0), hi = min(i + RP + r, L - 1 - kb0);
-    const int cw = 32 * q4;
-    const int ch0 = wg == 0 ? 0 : NC0, ch1 = wg == 0 ? NC0 : NC;
+    const int cw = 32 * q4, cb0 = cw + HALF * wg;
     const uint32_t trow = taddr + ((uint32_t)(32 * q4) << 16);
+    float v[HALF];
     float m = -INFINITY;
     if (s_ok) {
-        // two tensor-memory loads in flight per wait
 #pragma unroll
-        for (int c2 = 0; c2 < NC0; c2 += 2) {
-            const int chA = ch0 + c2, chB = ch0 + c2 + 1;
-            if (chA >= ch1) break;  // uniform
-            float va[32], vb[32];
-            umma::tmem_ld32(trow + (uint32_t)(cw + 32 * chA), va);
-            if (chB < ch1) umma::tmem_ld32(trow + (uint32_t)(cw + 32 * chB), vb);
-            umma::tmem_ld_wait();
+        for (int pc = 0; pc < NP; ++pc) {
+            float t16[16];
+            umma::tmem_ld16(trow + (uint32_t)(cb0 + 16 * pc), t16);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                if (u == 1 && chB >= ch1) break;
-                float *v = u ? vb : va;
+            for (int t = 0; t < 16; ++t) v[16 * pc + t] = t16[t];
+        }
+        umma::tmem_ld_wait();
 #pragma unroll
-                for (int t = 0; t < 32; ++t) asm volatile("" : "+f"(v[t]));  // used only after the wait
-                const int cb = cw + 32 * (u ? chB : chA);
-                if (cb >= lo && cb + 31 <= hi) {
+        for (int t = 0; t < HALF; ++t) asm volatile("" : "+f"(v[t]));  // used only after the wait
 #pragma unroll
-                    for (int t = 0; t < 32; ++t) m = fmaxf(m, v[t]);
-                } else {
+        for (int pc = 0; pc < NP; ++pc) {
+            const int cb = cb0 + 16 * pc;
+            if (cb >= lo && cb + 15 <= hi) {
 #pragma unroll
-                    for (int t = 0; t < 32; ++t)
-                        if ((unsigned)(cb + t - lo) <= (unsigned)(hi - lo)) m = fmaxf(m, v[t]);
-                }
+                for (int t = 0; t < 16; ++t) m = fmaxf(m, v[16 * pc + t]);
+            } else {
+#pragma unroll
+                for (int t = 0; t < 16; ++t)
+                    if ((unsigned)(cb + t - lo) <= (unsigned)(hi - lo)) m = fmaxf(m, v[16 * pc + t]);
             }
         }
     }
@@ -1231,45 +1230,33 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
         for (int c8 = z0; c8 < z1; ++c8)
             asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(p_chunk(c8)), "r"(0u) : "memory");
 #pragma unroll
-        for (int c2 = 0; c2 < NC0; c2 += 2) {
-            const int chA = ch0 + c2, chB = ch0 + c2 + 1;
-            if (chA >= ch1) break;  // uniform
-            float va[32], vb[32];
-            umma::tmem_ld32(trow + (uint32_t)(cw + 32 * chA), va);
-            if (chB < ch1) umma::tmem_ld32(trow + (uint32_t)(cw + 32 * chB), vb);
-            umma::tmem_ld_wait();
+        for (int pc = 0; pc < NP; ++pc) {
+            const int cb = cb0 + 16 * pc;
+            uint32_t pk[8];
+            if (cb >= lo && cb + 15 <= hi) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                if (u == 1 && chB >= ch1) break;
-                float *v = u ? vb : va;
-#pragma unroll
-                for (int t = 0; t < 32; ++t) asm volatile("" : "+f"(v[t]));
-                const int cb = cw + 32 * (u ? chB : chA);
-                uint32_t pk[16];
-                if (cb >= lo && cb + 31 <= hi) {
-#pragma unroll
-                    for (int t = 0; t < 32; t += 2) {
-                        const float p0 = fused::ex2(fmaf(v[t], csc, -mc)), p1 = fused::ex2(fmaf(v[t + 1], csc, -mc));
-                        l += p0 + p1;
-                        pk[t >> 1] = pack_bf16(p0, p1);
-                    }
-                } else {
-#pragma unroll
-                    for (int t = 0; t < 32; t += 2) {
-                        const bool in0 = (unsigned)(cb + t - lo) <= (unsigned)(hi - lo);
-                        const bool in1 = (unsigned)(cb + t + 1 - lo) <= (unsigned)(hi - lo);
-                        const float p0 = in0 ? fused::ex2(fmaf(v[t], csc, -mc)) : 0.f;
-                        const float p1 = in1 ? fused::ex2(fmaf(v[t + 1], csc, -mc)) : 0.f;
-                        l += p0 + p1;
-                        pk[t >> 1] = pack_bf16(p0, p1);
-                    }
+                for (int t = 0; t < 16; t += 2) {
+                    const float p0 = fused::ex2(fmaf(v[16 * pc + t], csc, -mc));
+                    const float p1 = fused::ex2(fmaf(v[16 * pc + t + 1], csc, -mc));
+                    l += p0 + p1;
+                    pk[t >> 1] = pack_bf16(p0, p1);
                 }
+            } else {
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(p_chunk(cb / 8 + q)), "r"(pk[4 * q]),
-                                 "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
-                                 : "memory");
+                for (int t = 0; t < 16; t += 2) {
+                    const bool in0 = (unsigned)(cb + t - lo) <= (unsigned)(hi - lo);
+                    const bool in1 = (unsigned)(cb + t + 1 - lo) <= (unsigned)(hi - lo);
+                    const float p0 = in0 ? fused::ex2(fmaf(v[16 * pc + t], csc, -mc)) : 0.f;
+                    const float p1 = in1 ? fused::ex2(fmaf(v[16 * pc + t + 1], csc, -mc)) : 0.f;
+                    l += p0 + p1;
+                    pk[t >> 1] = pack_bf16(p0, p1);
+                }
             }
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(p_chunk(cb / 8 + q)), "r"(pk[4 * q]),
+                             "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
+                             : "memory");
         }
     }
     red[256 + wg * 128 + i] = l;
