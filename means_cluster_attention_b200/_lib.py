@@ -13,6 +13,9 @@ from typing import Optional, Tuple
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libclusterattn.so")
+# CA_CHECKED=1 selects the bounds-checked build (same ABI; index checks on the
+# device report CA_ERR_DEVICE through ca_sync_status instead of faulting).
+LIB_CHECKED_PATH = os.path.join(PKG, "libclusterattn_checked.so")
 
 CA_OK = 0
 STATUS_NAMES = {0: "CA_OK", 1: "CA_ERR_INVALID_ARG", 2: "CA_ERR_UNSUPPORTED", 3: "CA_ERR_CUDA",
@@ -62,7 +65,7 @@ def load(path: Optional[str] = None):
     global _lib
     if _lib is not None and path is None:
         return _lib
-    p = path or LIB_PATH
+    p = path or (LIB_CHECKED_PATH if os.environ.get("CA_CHECKED") == "1" else LIB_PATH)
     if not os.path.exists(p):
         raise OSError(f"libclusterattn.so not found at {p}; build it with "
                       "`python -m means_cluster_attention_b200.build`")

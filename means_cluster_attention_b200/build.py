@@ -19,6 +19,11 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libclusterattn.so")
+# The bounds-checked build (-DCA_CHECKED): every computed index that addresses
+# memory is checked on the device; a bad one records CA_ERR_DEVICE (read by
+# ca_sync_status) and is clamped, so nothing faults.  Selected at load time
+# with the environment variable CA_CHECKED=1.
+LIB_CHECKED = os.path.join(PKG, "libclusterattn_checked.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -66,19 +71,22 @@ def source_hash(kernel: str = None) -> str:
     return h.hexdigest()[:16]
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
-    if not force and not needs_build():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+def build(force: bool = False, verbose: bool = False, extra_flags=None, checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
+    if not force and not needs_build(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
            "-I", INCLUDE, "-I", CSRC, "-o", tmp, os.path.join(CSRC, "api.cu"), "-cudart", "static"]
+    if checked:
+        cmd.insert(1, "-DCA_CHECKED")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     if extra_flags:
@@ -88,9 +96,10 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
     if verbose:
         sys.stderr.write(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, checked=True))

@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdarg>
@@ -44,6 +45,13 @@ ca_status cuda_fail(cudaError_t e, const char *what) {
         cudaError_t e_ = (call);                               \
         if (e_ != cudaSuccess) return cuda_fail(e_, #call);    \
     } while (0)
+
+// NVTX range around one forward (header-only NVTX: free unless a profiler
+// that records ranges is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
 
 struct Problem {
     int B, H, L, d, K, iters, W;
@@ -518,12 +526,17 @@ ca_status dispatch(const void *q, const void *k, const void *v, int dtype, const
     s = ensure_kernel_attributes();
     if (s != CA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
-    if (fused_eligible(dtype, p))
+    if (fused_eligible(dtype, p)) {
+        NvtxRange range("ca_forward fused");
         return run_fused((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, p,
                          (__nv_bfloat16 *)out, assign_out, cent_out, hist, st);
-    if (tiled_eligible(dtype, p))
+    }
+    if (tiled_eligible(dtype, p)) {
+        NvtxRange range("ca_forward tiled");
         return run_tiled((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, p,
                          (__nv_bfloat16 *)out, assign_out, cent_out, hist, st);
+    }
+    NvtxRange range("ca_forward general");
     if (dtype == 0)
         return run_forward<float>((const float *)q, (const float *)k, (const float *)v, p, (float *)out,
                                   assign_out, cent_out, hist, st);

@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(kWinThreads)
     // gathered global context: hard V_cent[c_i], or the soft assignment
     float gv[16];
     if (!var.soft) {
-        const int c = assign[(int64_t)h * L + qi];
+        const int c = CA_IDX(assign[(int64_t)h * L + qi], 0, K, 75);
         const float *g = vcent + ((int64_t)h * K + c) * kD + 16 * sub;
 #pragma unroll
         for (int t = 0; t < 16; ++t) gv[t] = g[t];

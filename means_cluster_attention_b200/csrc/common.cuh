@@ -45,6 +45,24 @@ __device__ __forceinline__ void record_error(int code, int where) {
     if (atomicCAS(&g_dev_error, 0, code) == 0) g_dev_error_where = where;
 }
 
+// Bounds-checked build (compiled with -DCA_CHECKED): CA_IDX(v, lo, hi, site)
+// checks a computed index at a point where it addresses memory; an index
+// outside [lo, hi) records CA_ERR_DEVICE with the site and is replaced by lo,
+// so nothing is accessed out of bounds and nothing faults.  In the normal
+// build CA_IDX is the index itself.
+#ifdef CA_CHECKED
+__device__ __forceinline__ int ca_checked_index(int v, int lo, int hi, int site) {
+    if (v < lo || v >= hi) {
+        record_error(5, site);
+        return lo;
+    }
+    return v;
+}
+#define CA_IDX(v, lo, hi, site) ca_checked_index((v), (lo), (hi), (site))
+#else
+#define CA_IDX(v, lo, hi, site) (v)
+#endif
+
 // Records code the way a kernel that detected a problem does (site 99), for
 // testing the host's error reporting without a fault.
 __global__ void debug_record_error_kernel(int code) { record_error(code, 99); }

@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
                     if (t == 0 && (u == 0 || two) && row < L) {
                         const float E = kEps * fmaf(qn[jp + u][h], mun_max, mm_max);
                         cs[row] = (uint8_t)bb.k1;
-                        if (bb.m2 <= bb.m1 + 2.f * E) list[atomicAdd(&misc[0], 1)] = (uint16_t)row;
+                        if (bb.m2 <= bb.m1 + 2.f * E) list[CA_IDX(atomicAdd(&misc[0], 1), 0, kMaxL, 70)] = (uint16_t)row;
                     }
                 }
             }
@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         // the second set are only run when that set exists.
         auto mu_at = [&](int k, int j) { return mu64[k * 65 + j]; };
         for (int e = warp; e < n_ref; e += kWarps) {
-            const int row = list[e];
+            const int row = CA_IDX(list[e], 0, L, 71);
             int bk = Kp > 32 ? tile::remeasure_token<true>(qbytes, row, Kp, dead, mu_at, lane)
                              : tile::remeasure_token<false>(qbytes, row, Kp, dead, mu_at, lane);
             if (bk >= K) {
@@ -433,8 +433,8 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
         }
         if (n_mv <= (L >> 2)) {
             for (int e = warp; e < n_mv; e += kWarps) {
-                const int row = list[e];
-                const int co = cprev[row], cn = cs[row];
+                const int row = CA_IDX(list[e], 0, L, 72);
+                const int co = CA_IDX(cprev[row], 0, Kp, 73), cn = CA_IDX(cs[row], 0, Kp, 73);
                 const uint32_t w = *reinterpret_cast<const uint32_t *>(qbytes + swz(row, lane >> 2) + (lane & 3) * 4);
                 const double d0 = bf16_to_f64(w & 0xffffu), d1 = bf16_to_f64(w >> 16);
                 atomicAdd(&sums[co * kD + 2 * lane], -d0);
@@ -836,7 +836,7 @@ __global__ void __launch_bounds__(kThreads, 2) fused_forward_kernel(Params P) {
             for (int hh = 0; hh < 2; ++hh) {
                 const int i = i0 + g + 8 * hh;
                 const float f = hh ? f1 : f0;
-                const float *vrow = vc + (i < L ? cs[i] : 0) * kVcStride + 2 * t;
+                const float *vrow = vc + (i < L ? CA_IDX(cs[i], 0, K, 74) : 0) * kVcStride + 2 * t;
                 uint32_t wv[8];
 #pragma unroll
                 for (int d = 0; d < 8; ++d) {

@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kAssignThreads)
     {
         const int grp = threadIdx.x >> 6, j = threadIdx.x & 63;
         for (int i = t0; i < t1; ++i) {
-            const int c = c_s[i - t0];
+            const int c = CA_IDX(c_s[i - t0], 0, K, 76);
             if ((c & 3) == grp)
                 sum_s[(size_t)c * kD + j] = __dadd_rn(sum_s[(size_t)c * kD + j], (double)to_f32(qh[(int64_t)i * kD + j]));
         }

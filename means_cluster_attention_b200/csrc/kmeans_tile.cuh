@@ -17,6 +17,9 @@
 namespace ca {
 namespace tile {
 
+// Largest number of query rows a tile holds in shared memory (both kernels).
+constexpr int kMaxTileRows = 512;
+
 // Exact fp64 value of a bf16 bit pattern (low 16 bits of b) built with
 // integer operations: the 8-bit exponent is rebiased (+896) into the 11-bit
 // field and the 7 fraction bits become the top fraction bits.  Zero and
@@ -189,7 +192,7 @@ __device__ __forceinline__ void counting_sort(const uint8_t *cs, int n_chunks, i
         const int c = my_c[s2];
         const int x0 = __shfl_sync(0xffffffffu, b0, c & 31), x1 = __shfl_sync(0xffffffffu, b1, c & 31);
         if (c != 0xFF) {
-            const int pos = (c < 32 ? x0 : x1) + my_off[s2];
+            const int pos = CA_IDX((c < 32 ? x0 : x1) + my_off[s2], 0, n_chunks * 32, 60);
             perm[pos] = (uint16_t)((warp + s2 * nwarps) * 32 + lane);
             sc[pos] = (uint8_t)c;
         }
@@ -211,13 +214,13 @@ __device__ __forceinline__ void member_sums(const unsigned char *qbytes, const u
     const uint32_t lane_off = (uint32_t)(l16 & 1) * 8u;
     const int chunk = l16 >> 1;
     while (p < p1) {
-        const int c = sc[p];
+        const int c = CA_IDX(sc[p], 0, 64, 61);
         double a[4] = {0.0, 0.0, 0.0, 0.0}, b[4] = {0.0, 0.0, 0.0, 0.0};
         for (;;) {
             const int qq = p + lane;
             const unsigned same = __ballot_sync(0xffffffffu, qq < p1 && sc[qq] == c);
             const int n = __ffs(~same) ? __ffs(~same) - 1 : 32;
-            const int rowl = (lane < n) ? perm[p + lane] : 0;
+            const int rowl = (lane < n) ? CA_IDX(perm[p + lane], 0, kMaxTileRows, 62) : 0;
             for (int j = 0; j < n; j += 4) {
                 const int r0 = __shfl_sync(0xffffffffu, rowl, (j + h) & 31);
                 const int r1 = __shfl_sync(0xffffffffu, rowl, (j + 2 + h) & 31);

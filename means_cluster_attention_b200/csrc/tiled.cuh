@@ -535,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
                     for (int w2 = 0; w2 < (KP + 31) / 32; ++w2) b3[w2] = 0u;
 #pragma unroll
                     for (int k = 0; k < KP; ++k) b3[k >> 5] |= (sv[k] <= thr3 ? 1u : 0u) << (k & 31);
-                    const int e = atomicAdd(&misc[0], 1);
+                    const int e = CA_IDX(atomicAdd(&misc[0], 1), 0, kTileQ, 63);
                     list[e] = (uint16_t)row;
 #pragma unroll
                     for (int w2 = 0; w2 < (KP + 31) / 32; ++w2) lmask[e * 2 + w2] = b3[w2];
@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     // exact re-measure of ambiguous tokens, one warp per token
     const int n_ref = misc[0];
     for (int e = warp; e < n_ref; e += kWarps) {
-        const int row = list[e];
+        const int row = CA_IDX(list[e], 0, Lt, 64);
         auto mu_at = [&](int k, int j) { return (double)mu[k * mu_ld + j]; };
         bool certain;
         int bk = tile::decide_candidates(qbytes, row, lmask[2 * e], KP > 32 ? lmask[2 * e + 1] : 0u, dead, mu_at, lane,
@@ -589,8 +589,8 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
         if (n_mv <= kMoverMax) {
             double *psum = P.part_sum;
             for (int e = warp; e < n_mv; e += kWarps) {
-                const int row = list[e];
-                const int co = cprev[row], cn = cs[row];
+                const int row = CA_IDX(list[e], 0, Lt, 65);
+                const int co = CA_IDX(cprev[row], 0, Kp, 66), cn = CA_IDX(cs[row], 0, Kp, 66);
                 const uint32_t w = *reinterpret_cast<const uint32_t *>(qbytes + swz(row, lane >> 2) + (lane & 3) * 4);
                 const double d0 = bf16_to_f64(w & 0xffffu), d1 = bf16_to_f64(w >> 16);
                 double *so = psum + ((cb + co) * P.n_tiles + tile) * kD;
@@ -918,7 +918,8 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
         x.w *= be;
         *reinterpret_cast<float4 *>(vc + (e >> 4) * fused::kVcStride + (e & 15) * 4) = x;
     }
-    for (int i = threadIdx.x; i < kWinQ; i += kThreads) cblk[i] = (qb + i < L) ? P.assign[head * L + qb + i] : 0;
+    for (int i = threadIdx.x; i < kWinQ; i += kThreads)
+        cblk[i] = (qb + i < L) ? CA_IDX(P.assign[head * L + qb + i], 0, K, 68) : 0;
     const int i0 = qb + warp * 16;
     uint32_t a[4][4];
 #pragma unroll
@@ -1154,7 +1155,7 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
     // reads its share of the row's score columns and writes half of its
     // output row.
     const int i = 32 * q4 + (tid & 31), qi = q0 + i;
-    const int ci = qi < L ? P.assign[head * L + qi] : 0;
+    const int ci = qi < L ? CA_IDX(P.assign[head * L + qi], 0, K, 67) : 0;
     const float4 *vrow = reinterpret_cast<const float4 *>(P.vcent + (head * K + ci) * kD) + 8 * wg;
     umma::tc_fence_before();
     __syncthreads();

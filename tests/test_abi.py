@@ -6,6 +6,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -140,3 +141,15 @@ def test_debug_error_hook_validates_code_on_host(lib):
     # else is rejected before a launch, so this needs no GPU
     for bad in (0, 1, 2, 3, 6, -1):
         assert lib.ca_debug_record_error(bad, None) == 1
+
+
+def test_checked_build_exports_every_header_symbol_and_is_selected_by_env():
+    path = build.build(checked=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (ca_[a-z0-9_]+)\b", out))
+    assert not [s for s in header_symbols() if s not in exported]
+    code = ("import os, sys; sys.path.insert(0, %r); from means_cluster_attention_b200 import _lib; "
+            "lib = _lib.load(); print(lib._name)") % ROOT
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                       env=dict(os.environ, CA_CHECKED="1"), check=True)
+    assert r.stdout.strip().endswith("libclusterattn_checked.so")
