@@ -65,10 +65,11 @@
  *     the centroid update in index order within each 1024-token block, the
  *     blocks in order), so any finite input is reproducible.  The bf16
  *     fused and tiled kernels add the member sums with fp64 atomics whose
- *     order varies, but the sums are
- *     exact (hence order-free) whenever the non-zero magnitudes of Q lie
- *     within 2^-27 .. 16; outside that range the last bit of a centroid may
- *     vary between runs.
+ *     order varies, but the sums are exact (hence order-free) whenever every
+ *     non-zero magnitude in Q is at least 2^-26 and, for each coordinate,
+ *     the magnitudes of one head's queries add up to less than 2^19 (for
+ *     instance |Q| < 16 with L <= 32768); outside that envelope the last
+ *     bit of a centroid may vary between runs.
  */
 #ifndef CLUSTERATTN_H_
 #define CLUSTERATTN_H_
@@ -213,8 +214,8 @@ const char *ca_version(void);
  * output the kernel must touch).  Kernel names: the fused one-CTA-per-head
  * kernel (bf16, L <= 512, K <= 64, floor(W/2) <= 16) is "fused_forward";
  * the tiled bf16 path (K <= 64, floor(W/2) <= 128) launches "tiled_init",
- * then per Lloyd iteration "tiled_dead", "tiled_assign" and
- * "tiled_update", then "tiled_centroid", "tiled_combine" and
+ * then per Lloyd iteration "tiled_assign" and "tiled_update", then
+ * "tiled_centroid", "tiled_combine" and
  * "tiled_window"; every other case runs the general path "kmeans_init",
  * "kmeans_assign", "kmeans_update", "centroid_attn", "centroid_combine" and
  * "window_blend". */

@@ -254,15 +254,13 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     using namespace ca;
     const int64_t NH = p.heads();
     const int L = p.L, K = p.K, Kp = tiled::kpad(K);
-    const int n_tiles = (L + tiled::kTileQ - 1) / tiled::kTileQ;
     const int n_chunks = (L + tiled::kChunk - 1) / tiled::kChunk;
     const float scale = 1.0f / sqrtf((float)p.d);
     Scratch s(st);
     float *mu = nullptr, *mm = nullptr, *cpart = nullptr, *vcent = nullptr;
     __nv_bfloat16 *hi = nullptr, *lo = nullptr;
-    uint32_t *hash = nullptr;
-    double *psum = nullptr;
-    int *pcnt = nullptr;
+    double *rsum = nullptr;
+    int *rcnt = nullptr;
     uint8_t *dead = nullptr;
     float *mstat = nullptr, *qnorm = nullptr;
     int32_t *assign = assign_out;
@@ -273,9 +271,8 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     CA_CUDA(s.get((void **)&hi, sizeof(__nv_bfloat16) * NH * Kp * kD));
     CA_CUDA(s.get((void **)&lo, sizeof(__nv_bfloat16) * NH * Kp * kD));
     CA_CUDA(s.get((void **)&mm, sizeof(float) * NH * Kp));
-    CA_CUDA(s.get((void **)&hash, sizeof(uint32_t) * NH * Kp));
-    CA_CUDA(s.get((void **)&psum, sizeof(double) * NH * n_tiles * Kp * kD));
-    CA_CUDA(s.get((void **)&pcnt, sizeof(int) * NH * n_tiles * Kp));
+    CA_CUDA(s.get((void **)&rsum, sizeof(double) * NH * Kp * kD));
+    CA_CUDA(s.get((void **)&rcnt, sizeof(int) * NH * Kp));
     CA_CUDA(s.get((void **)&cpart, sizeof(float) * NH * n_chunks * K * tiled::kPartLd));
     CA_CUDA(s.get((void **)&vcent, sizeof(float) * NH * K * kD));
     if (!assign) CA_CUDA(s.get((void **)&assign, sizeof(int32_t) * NH * L));
@@ -287,24 +284,24 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
 
     const double head_bytes = (double)NH * L * kD * sizeof(__nv_bfloat16);
 
-    tiled::MuParams mp{};
-    mp.q = q;
-    mp.part_sum = psum;
-    mp.part_cnt = pcnt;
-    mp.mu = mu;
-    mp.hi = hi;
-    mp.lo = lo;
-    mp.mm = mm;
-    mp.hash = hash;
-    mp.L = L;
-    mp.K = K;
-    mp.Kp = Kp;
-    mp.n_tiles = n_tiles;
-    mp.init = 1;
-    mp.cent_out = p.iters == 0 ? cent_out : nullptr;
+    tiled::UpdateParams up{};
+    up.q = q;
+    up.sum = rsum;
+    up.cnt = rcnt;
+    up.mu = mu;
+    up.hi = hi;
+    up.lo = lo;
+    up.mm = mm;
+    up.dead = dead;
+    up.mstat = mstat;
+    up.L = L;
+    up.K = K;
+    up.Kp = Kp;
+    up.init = 1;
+    up.cent_out = p.iters == 0 ? cent_out : nullptr;
     {
         Launch pl("tiled_init", st, 0.0);
-        tiled::tiled_mu_kernel<<<dim3(Kp, (unsigned)NH), 256, 0, st>>>(mp);
+        tiled::tiled_update_kernel<<<(unsigned)NH, tiled::kUpdThreads, 0, st>>>(up);
         pl.after();
     }
     CA_CUDA(cudaGetLastError());
@@ -322,35 +319,27 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     ap.qnorm = qnorm;
     ap.assign = assign;
     ap.hist_stride = (int64_t)p.iters * L;
-    ap.part_sum = psum;
-    ap.part_cnt = pcnt;
+    ap.sum = rsum;
+    ap.cnt = rcnt;
     ap.L = L;
     ap.K = K;
-    ap.n_tiles = n_tiles;
-    mp.init = 0;
+    up.init = 0;
+    const dim3 agrid((L + tiled::kTileQ - 1) / tiled::kTileQ, (unsigned)NH);
     for (int t = 0; t < p.iters; ++t) {
-        {
-            Launch pl("tiled_dead", st, 0.0);
-            CA_CUDA(launch_pdl(tiled::tiled_dead_kernel, dim3(Kp, (unsigned)NH), dim3(64), 0, st, K, Kp,
-                               (const float *)mu, (const float *)mm, (const uint32_t *)hash, dead, mstat));
-            pl.after();
-        }
-        CA_CUDA(cudaGetLastError());
         ap.hist = hist ? hist + (int64_t)t * L : nullptr;
         ap.first = t == 0;
         {
             Launch pl("tiled_assign", st, head_bytes);
-            const dim3 grid(n_tiles, (unsigned)NH);
             auto kern = Kp == 16 ? tiled::tiled_assign_kernel<16>
                                  : (Kp == 32 ? tiled::tiled_assign_kernel<32> : tiled::tiled_assign_kernel<64>);
-            CA_CUDA(launch_pdl(kern, grid, dim3(tiled::kThreads), alay.total, st, qmap, ap));
+            CA_CUDA(launch_pdl(kern, agrid, dim3(tiled::kThreads), alay.total, st, qmap, ap));
             pl.after();
         }
         CA_CUDA(cudaGetLastError());
-        mp.cent_out = t == p.iters - 1 ? cent_out : nullptr;
+        up.cent_out = t == p.iters - 1 ? cent_out : nullptr;
         {
             Launch pl("tiled_update", st, 0.0);
-            CA_CUDA(launch_pdl(tiled::tiled_mu_kernel, dim3(Kp, (unsigned)NH), dim3(256), 0, st, mp));
+            CA_CUDA(launch_pdl(tiled::tiled_update_kernel, dim3((unsigned)NH), dim3(tiled::kUpdThreads), 0, st, up));
             pl.after();
         }
         CA_CUDA(cudaGetLastError());

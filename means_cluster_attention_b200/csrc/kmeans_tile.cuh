@@ -252,5 +252,146 @@ __device__ __forceinline__ void member_sums(const unsigned char *qbytes, const u
     }
 }
 
+// Packed sum entry: query row in bits 0..9, cluster in bits 16..21, bit 30
+// for a padding entry (adds nothing), bit 31 for a subtracted row.
+constexpr uint32_t kEntPad = 0x40000000u, kEntNeg = 0x80000000u;
+
+// Counting sort of up to 32 * n_chunks entries by cluster into packed
+// entries ent[], every cluster's run padded with one padding entry to even
+// length (so the two halves of a warp always meet the same cluster).  cl(i)
+// is entry i's cluster (0xFF for none) and info(i) its row and sign bits;
+// cnt[] (Kp <= 64 entries) must be zero on entry.  *n_out receives the
+// padded length.  Each warp handles chunks warp and warp + nwarps.
+// Contains __syncthreads.
+template <typename Cl, typename Info>
+__device__ __forceinline__ void counting_sort_even(Cl cl, Info info, int n_chunks, int Kp, int *cnt, uint32_t *ent,
+                                                   int *n_out, int warp, int nwarps, int lane) {
+    int my_c[2], my_off[2];
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+        const int ch = warp + s2 * nwarps;
+        my_c[s2] = 0xFF;
+        my_off[s2] = 0;
+        if (ch < n_chunks) {
+            const int c = cl(ch * 32 + lane);
+            const unsigned peers = __match_any_sync(0xffffffffu, c);
+            const int leader = __ffs(peers) - 1;
+            int off = 0;
+            if (c != 0xFF && lane == leader) off = atomicAdd(&cnt[c], __popc(peers));
+            off = __shfl_sync(0xffffffffu, off, leader);
+            my_c[s2] = c;
+            my_off[s2] = off + __popc(peers & ((1u << lane) - 1u));
+        }
+    }
+    __syncthreads();
+    const int c0 = lane < Kp ? cnt[lane] : 0, c1 = lane + 32 < Kp ? cnt[lane + 32] : 0;
+    const int e0 = (c0 + 1) & ~1, e1 = (c1 + 1) & ~1;
+    int s0 = e0, s1 = e1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x0 = __shfl_up_sync(0xffffffffu, s0, o), x1 = __shfl_up_sync(0xffffffffu, s1, o);
+        if (lane >= o) {
+            s0 += x0;
+            s1 += x1;
+        }
+    }
+    const int tot0 = __shfl_sync(0xffffffffu, s0, 31);
+    const int b0 = s0 - e0, b1 = tot0 + s1 - e1;
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+        const int c = my_c[s2];
+        const int x0 = __shfl_sync(0xffffffffu, b0, c & 31), x1 = __shfl_sync(0xffffffffu, b1, c & 31);
+        if (c != 0xFF) {
+            const int i = (warp + s2 * nwarps) * 32 + lane;
+            const int pos = CA_IDX((c < 32 ? x0 : x1) + my_off[s2], 0, n_chunks * 32 + 64, 60);
+            ent[pos] = info(i) | ((uint32_t)c << 16);
+        }
+    }
+    const int total = tot0 + __shfl_sync(0xffffffffu, s1, 31);
+    if (warp == 0) {
+        if (c0 & 1) ent[CA_IDX(b0 + c0, 0, n_chunks * 32 + 64, 60)] = kEntPad | ((uint32_t)lane << 16);
+        if (c1 & 1) ent[CA_IDX(b1 + c1, 0, n_chunks * 32 + 64, 60)] = kEntPad | ((uint32_t)(lane + 32) << 16);
+        if (lane == 0) *n_out = total;
+    }
+    __syncthreads();
+}
+
+// Exact fp64 sums of signed query rows over the packed sorted entries
+// [p, p1) (p, p1 even) into a head's running sums gsum and counts gcnt in
+// global memory.  Each step takes two entries, one per half-warp, lane l
+// holding coordinates 4 (l mod 16) .. +3 (one 8-byte load); both entries
+// belong to the same cluster, so the walk never diverges.  A subtracted
+// row has the sign bits of its bf16 values flipped (exact).  When the
+// cluster changes, the run's sum goes out with two fp64 reductions
+// (red.global.add.f64) per lane: coordinate 4 l16 + i is kept at position
+// 16 i + l16 of its row of gsum, so each reduction instruction covers two
+// whole 128-byte lines; the run's signed count goes out with one integer
+// reduction.  When every partial state of the running sums is a multiple of
+// the smallest ulp among the added values and below 2^53 of those ulps,
+// every addition is exact and their order changes no bit.
+__device__ __forceinline__ void run_sums_red(const unsigned char *qbytes, const uint32_t *ent, int p, int p1,
+                                             double *gsum, int *gcnt, int lane) {
+    if (p >= p1) return;
+    const int h = lane >> 4, l16 = lane & 15;
+    const uint32_t lane_off = (uint32_t)(l16 & 1) * 8u;
+    const int chunk = l16 >> 1;
+    double a[4] = {0.0, 0.0, 0.0, 0.0}, b[4] = {0.0, 0.0, 0.0, 0.0};
+    int cnt = 0;
+    int c_cur = (int)((ent[p] >> 16) & 63u);
+    auto flush = [&](int c) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            a[i] += b[i];
+            a[i] += __shfl_xor_sync(0xffffffffu, a[i], 16);
+        }
+        double *row = gsum + c * kD;
+        atomicAdd(&row[32 * h + l16], h ? a[2] : a[0]);
+        atomicAdd(&row[32 * h + 16 + l16], h ? a[3] : a[1]);
+        const int t = cnt + __shfl_xor_sync(0xffffffffu, cnt, 16);
+        if (lane == 0 && t != 0) atomicAdd(&gcnt[c], t);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = b[i] = 0.0;
+        cnt = 0;
+    };
+    auto fetch = [&](uint32_t e) {
+        uint2 w = make_uint2(0u, 0u);
+        if (!(e & kEntPad)) {
+            w = *reinterpret_cast<const uint2 *>(qbytes + swz(CA_IDX((int)(e & 0x3FFu), 0, kMaxTileRows, 78), chunk) +
+                                                 lane_off);
+            const uint32_t f = (uint32_t)((int)e >> 31) & 0x80008000u;
+            w.x ^= f;
+            w.y ^= f;
+        }
+        return w;
+    };
+    auto delta = [](uint32_t e) { return (e & kEntPad) ? 0 : ((e & kEntNeg) ? -1 : 1); };
+    for (; p < p1; p += 4) {
+        const bool two = p + 2 < p1;  // uniform
+        const uint32_t e0 = ent[p + h];
+        const uint32_t e1 = two ? ent[p + 2 + h] : kEntPad | (e0 & (63u << 16));
+        const uint2 w0 = fetch(e0), w1 = fetch(e1);
+        const int c0 = (int)((e0 >> 16) & 63u), c1 = (int)((e1 >> 16) & 63u);
+        if (c0 != c_cur) {
+            flush(c_cur);
+            c_cur = c0;
+        }
+        a[0] += (double)__uint_as_float(w0.x << 16);
+        a[1] += (double)__uint_as_float(w0.x & 0xffff0000u);
+        a[2] += (double)__uint_as_float(w0.y << 16);
+        a[3] += (double)__uint_as_float(w0.y & 0xffff0000u);
+        cnt += delta(e0);
+        if (c1 != c_cur) {
+            flush(c_cur);
+            c_cur = c1;
+        }
+        b[0] += (double)__uint_as_float(w1.x << 16);
+        b[1] += (double)__uint_as_float(w1.x & 0xffff0000u);
+        b[2] += (double)__uint_as_float(w1.y << 16);
+        b[3] += (double)__uint_as_float(w1.y & 0xffff0000u);
+        cnt += delta(e1);
+    }
+    flush(c_cur);
+}
+
 }  // namespace tile
 }  // namespace ca

@@ -1,21 +1,21 @@
 // Tiled cluster-attention kernels for long sequences (bf16): a head is split
 // over several CTAs.
 //
-//   tiled_mu_kernel        (Kp, heads)     mu = strided init, or the update
+//   tiled_update_kernel    (heads)         mu = strided init, or the update
 //                                          mu_k = fp32(sum_k / max(1, count_k))
-//                                          from per-tile exact partial sums;
-//                                          also the bf16 hi/lo split, |mu|^2
-//                                          and a row hash for each centroid.
-//   tiled_dead_kernel      (Kp, heads)     marks centroids that are bitwise
+//                                          from the head's exact running sums;
+//                                          also the bf16 hi/lo split, |mu|^2,
+//                                          the centroids that are bitwise
 //                                          copies of a lower-index one (they
 //                                          can never win the argmin) and
-//                                          records max |mu|^2 per head.
+//                                          max |mu|^2.
 //   tiled_assign_kernel    (tiles, heads)  one Lloyd assignment for a tile of
 //                                          512 queries: TMA-staged queries,
 //                                          distances on tcgen05 (tensor-memory
 //                                          accumulators), certified argmin,
 //                                          exact fp64 re-measure of ambiguous
-//                                          tokens, the tile's exact member sums.
+//                                          tokens, the tile's exact share of
+//                                          the head's running member sums.
 //   tiled_centroid_kernel  (chunks, heads) partial softmax state of every
 //                                          centroid over 512 keys;
 //   tiled_combine_kernel   (K, heads)      combines the chunk states into
@@ -67,131 +67,109 @@ constexpr int kNTChunk = 6;   // key n-tiles per online-softmax step in the wind
 __host__ __device__ inline int kpad(int K) { return K <= 16 ? 16 : (K <= 32 ? 32 : 64); }
 
 // ---------------------------------------------------------------------------
-// Centroid set: mu^(0) or the update from per-tile partial sums.
-struct MuParams {
+// Centroid set of one head: mu^(0) or the update from the running sums.
+struct UpdateParams {
     const __nv_bfloat16 *q;
-    const double *part_sum;  // [NH][Kp][n_tiles][64]
-    const int *part_cnt;     // [NH][Kp][n_tiles]
+    double *sum;             // [NH][Kp][64] exact running member sums (coordinate j at 16 (j mod 4) + j / 4)
+    int *cnt;                // [NH][Kp] running member counts
     float *mu;               // [NH][Kp][64]
     __nv_bfloat16 *hi, *lo;  // [NH][Kp][64]
     float *mm;               // [NH][Kp] |mu_k|^2
-    uint32_t *hash;          // [NH][Kp]
+    uint8_t *dead;           // [NH][Kp] 1 for centroids that can never win
+    float *mstat;            // [NH][2] max over k < K of |mu_k|^2, and its square root
     float *cent_out;         // [NH][K][64] or null
-    int L, K, Kp, n_tiles, init;
+    int L, K, Kp, init;
 };
 
-// grid (Kp, NH), 256 threads: thread (g8, jp) adds tiles g8, g8+8, ... of
-// coordinates 2 jp and 2 jp + 1 of centroid k (16-byte loads); thread j of
-// the first 64 then adds the eight exact partial sums of coordinate j in
-// group order and finalises it.
-__global__ void __launch_bounds__(256) tiled_mu_kernel(MuParams P) {
-    __shared__ double2 red_s[8][32];
-    __shared__ int red_c[8];
-    __shared__ float red_sq[2];
-    __shared__ uint32_t red_h[2];
-    const int k = blockIdx.x, jp = threadIdx.x & 31, g8 = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int64_t head = blockIdx.y;
-    const int64_t kb = head * P.Kp + k;
+// grid (NH), 1024 threads.  mu_k = Q[floor(k L / K)] (init; the running sums
+// and counts are cleared for the first assignment) or fp32(sum_k /
+// max(1, count_k)); padding rows k >= K are zero.  Also the bf16 hi/lo
+// split, |mu_k|^2, the dead marks (a bitwise copy of a lower-index centroid
+// has the same distances and loses every tie; padding rows never win) and
+// max |mu_k|^2 for the assignment's error bound.
+constexpr int kUpdThreads = 1024;
+__global__ void __launch_bounds__(kUpdThreads) tiled_update_kernel(UpdateParams P) {
+    __shared__ float mus[64][kD + 1];
+    __shared__ uint32_t hs[64];
+    __shared__ float ms[64];
+    __shared__ uint8_t ds[64];
+    __shared__ int ns[64];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int K = P.K, Kp = P.Kp;
+    const int64_t head = blockIdx.x, hb = head * Kp;
     pdl_launch();
     pdl_wait();
-    double2 s = make_double2(0.0, 0.0);
-    int cnt = 0;
-    if (!P.init && k < P.K) {
-        for (int tt = g8; tt < P.n_tiles; tt += 8) {
-            const double2 v = reinterpret_cast<const double2 *>(P.part_sum + (kb * P.n_tiles + tt) * kD)[jp];
-            s.x += v.x;
-            s.y += v.y;
-            if (jp == 0) cnt += P.part_cnt[kb * P.n_tiles + tt];
+    if (tid < Kp) ns[tid] = P.init ? 0 : P.cnt[hb + tid];
+    // thread (k0, j) takes coordinate j of centroids k0, k0 + 16, ...: every
+    // load is issued before the first is used
+    constexpr int kPer = 64 * kD / kUpdThreads, kRows = kUpdThreads / kD, kUw = kUpdThreads / 32;
+    const int j = tid & (kD - 1), k0 = tid >> 6;
+    double sv[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int k = k0 + kRows * u;
+        sv[u] = 0.0;
+        if (k < K) {
+            if (P.init) {
+                const int64_t row = ((int64_t)k * P.L) / K;
+                sv[u] = (double)__bfloat162float(P.q[(head * P.L + row) * kD + j]);
+            } else {
+                sv[u] = P.sum[(hb + k) * kD + (j & 3) * 16 + (j >> 2)];
+            }
         }
     }
-    red_s[g8][jp] = s;
-    if (jp == 0) red_c[g8] = cnt;
     __syncthreads();
-    if (threadIdx.x >= 64) return;
-    // thread j (< 64) finalises coordinate j
-    const int j = threadIdx.x, wid = j >> 5;
-    float x = 0.f;
-    if (k < P.K) {
-        if (P.init) {
-            const int64_t row = ((int64_t)k * P.L) / P.K;
-            x = __bfloat162float(P.q[(head * P.L + row) * kD + j]);
-        } else {
-            double tot = 0.0;
 #pragma unroll
-            for (int g = 0; g < 8; ++g) tot += (j & 1) ? red_s[g][j >> 1].y : red_s[g][j >> 1].x;
-            int n = 0;
+    for (int u = 0; u < kPer; ++u) {
+        const int k = k0 + kRows * u;
+        if (k >= Kp) break;
+        const int64_t o = (hb + k) * kD + j;
+        float x = 0.f;
+        if (k < K) {
+            const int n = ns[k];
+            x = P.init ? (float)sv[u] : __double2float_rn(sv[u] / (double)(n > 1 ? n : 1));
+        }
+        if (P.init) P.sum[o] = 0.0;
+        mus[k][j] = x;
+        P.mu[o] = x;
+        const __nv_bfloat16 h = __float2bfloat16_rn(x);
+        P.hi[o] = h;
+        P.lo[o] = __float2bfloat16_rn(x - __bfloat162float(h));
+        if (P.cent_out && k < K) P.cent_out[(head * K + k) * kD + j] = x;
+    }
+    if (P.init && tid < Kp) P.cnt[hb + tid] = 0;
+    __syncthreads();
+    for (int k = warp; k < Kp; k += kUw) {
+        const float x0 = mus[k][2 * lane], x1 = mus[k][2 * lane + 1];
+        float sq = fmaf(x0, x0, x1 * x1);
+        uint32_t hv = __float_as_uint(x0) * (0x9E3779B1u + 4u * (uint32_t)lane) +
+                      __float_as_uint(x1) * (0x85EBCA77u + 4u * (uint32_t)lane) + (uint32_t)lane * 0xC2B2AE3Du;
 #pragma unroll
-            for (int g = 0; g < 8; ++g) n += red_c[g];
-            x = __double2float_rn(tot / (double)(n > 1 ? n : 1));
+        for (int off = 16; off > 0; off >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            hv += __shfl_xor_sync(0xffffffffu, hv, off);
+        }
+        if (lane == 0) {
+            ms[k] = sq;
+            hs[k] = hv;
+            ds[k] = k >= K ? 1 : 0;
+            P.mm[hb + k] = sq;
         }
     }
-    const int64_t o = kb * kD + j;
-    P.mu[o] = x;
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    P.hi[o] = h;
-    P.lo[o] = __float2bfloat16_rn(x - __bfloat162float(h));
-    if (P.cent_out && k < P.K) P.cent_out[(head * P.K + k) * kD + j] = x;
-    float sq = x * x;
-    uint32_t hv = __float_as_uint(x) * (0x9E3779B1u + 2u * (uint32_t)j) + (uint32_t)j * 0xC2B2AE3Du;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        sq += __shfl_xor_sync(0xffffffffu, sq, off);
-        hv += __shfl_xor_sync(0xffffffffu, hv, off);
-    }
-    if (lane == 0) {
-        red_sq[wid] = sq;
-        red_h[wid] = hv;
-    }
-    asm volatile("bar.sync 1, 64;");
-    if (j == 0) {
-        P.mm[kb] = red_sq[0] + red_sq[1];
-        P.hash[kb] = red_h[0] + red_h[1];
-    }
-}
-
-// Centroids that can never win: grid (Kp, NH), 64 threads.  CTA k marks
-// centroid k dead when it is a bitwise copy of a lower-index centroid (its
-// distances equal that centroid's and ties go to the lowest index) or a
-// padding row (k >= K); lower indices with the same row hash are compared
-// coordinate by coordinate, lowest first.  CTA 0 also records max_k |mu_k|^2
-// over k < K (a copy has its original's norm).
-__global__ void __launch_bounds__(64) tiled_dead_kernel(int K, int Kp, const float *__restrict__ mu,
-                                                        const float *__restrict__ mm,
-                                                        const uint32_t *__restrict__ hash, uint8_t *__restrict__ dead,
-                                                        float *__restrict__ mstat) {
-    const int k = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
-    const int64_t head = blockIdx.y, hb = head * Kp;
-    pdl_launch();
-    pdl_wait();
-    if (k == 0 && w == 1) {
+    __syncthreads();
+    if (warp == kUw - 1) {
         float mx = 0.f;
-        for (int k2 = lane; k2 < K; k2 += 32) mx = fmaxf(mx, mm[hb + k2]);
+        for (int k2 = lane; k2 < K; k2 += 32) mx = fmaxf(mx, ms[k2]);
         mx = warp_max(mx);
         if (lane == 0) {
-            mstat[head * 2 + 0] = mx;
-            mstat[head * 2 + 1] = sqrtf(mx);
+            P.mstat[head * 2 + 0] = mx;
+            P.mstat[head * 2 + 1] = sqrtf(mx);
         }
     }
-    if (k >= K) {
-        if (t == 0) dead[hb + k] = 1;
-        return;
-    }
-    const uint32_t hk = hash[hb + k];
-    const float x = mu[(hb + k) * kD + t];
-    // Both warps form the same candidate masks, so every barrier below is
-    // reached by all 64 threads; the barrier's vote is the same everywhere.
-    bool found = false;
-    for (int a0 = 0; a0 < k && !found; a0 += 32) {
-        const int a = a0 + lane;
-        unsigned cand = __ballot_sync(0xffffffffu, a < k && hash[hb + a] == hk);
-        while (cand && !found) {
-            const int b = a0 + __ffs(cand) - 1;
-            cand &= cand - 1u;
-            found = __syncthreads_and(__float_as_uint(mu[(hb + b) * kD + t]) == __float_as_uint(x)) != 0;
-        }
-    }
-    if (t == 0) dead[hb + k] = found ? 1 : 0;
+    __syncthreads();
+    mark_copies(K, hs, &mus[0][0], kD + 1, ds, ms, warp, kUw, lane);
+    __syncthreads();
+    if (tid < Kp) P.dead[hb + tid] = ds[tid];
 }
 
 // Floats per chunk state of the centroid attention: 64 accumulator values,
@@ -256,7 +234,9 @@ __global__ void __launch_bounds__(64) tiled_combine_kernel(int K, int n_chunks, 
 // Epilogue: every thread owns one token row of a block (tcgen05.ld), forms
 // s_k = |mu_k|^2 - 2 D_k, takes the minimum m1 and the set of k with
 // s_k <= m1 + 2E; a single member is the certified argmin, several send the
-// token to the exact fp64 re-measure.
+// token to the exact fp64 re-measure.  Sums: the tile's tokens (first
+// iteration) or its movers (later ones, signed) are sorted by cluster and
+// added run by run to the head's running sums with fp64 reductions.
 //
 // Error bound: the split leaves |mu - hi - lo| <= 2^-18 |mu| per coordinate;
 // the products are exact and even an accumulator that truncates every one of
@@ -266,22 +246,19 @@ __global__ void __launch_bounds__(64) tiled_combine_kernel(int K, int n_chunks, 
 // max|mu|^2) covers it threefold.
 struct AssignLayout {
     int Kp;
-    uint32_t q_off, r_off, mu_off, mm_off, dead_off, cnt_off, c_off, sc_off, cprev_off, list_off, lmask_off,
-        perm_off, misc_off, bar_off, total;
+    uint32_t q_off, r_off, mu_off, mm_off, dead_off, cnt_off, c_off, cprev_off, list_off, lmask_off, ent_off,
+        misc_off, bar_off, total;
     __host__ __device__ AssignLayout(int K) {
         Kp = kpad(K);
         uint32_t o = 0;
         q_off = o;  // 512 rows x 128 bytes, 1024-aligned (TMA / MMA swizzle)
         o += (uint32_t)kTileQ * 128u;
-        // Region R, reused in turn: the MMA's B operand [hi; lo] (2 Kp rows of
-        // 128 bytes, 1024-aligned) beside the fp32 centroids (rows padded to
-        // 65 floats) for the exact re-measure; then the tile's fp64 member
-        // sums [Kp][64].
+        // The MMA's B operand [hi; lo] (2 Kp rows of 128 bytes, 1024-aligned)
+        // beside the fp32 centroids (rows padded to 65 floats) for the exact
+        // re-measure.
         r_off = o;
         mu_off = o + 2u * (uint32_t)Kp * 128u;
-        const uint32_t r_a = 2u * (uint32_t)Kp * 128u + (uint32_t)Kp * 65u * 4u;
-        const uint32_t r_b = (uint32_t)Kp * 64u * 8u;
-        o += up(r_a > r_b ? r_a : r_b, 16);
+        o += up(2u * (uint32_t)Kp * 128u + (uint32_t)Kp * 65u * 4u, 16);
         mm_off = o;
         o += (uint32_t)Kp * 4u;
         dead_off = o;
@@ -290,16 +267,14 @@ struct AssignLayout {
         o += (uint32_t)Kp * 4u;
         c_off = o;
         o += (uint32_t)kTileQ;
-        sc_off = o;
-        o += (uint32_t)kTileQ;
         cprev_off = o;
         o += (uint32_t)kTileQ;
         list_off = o;
         o += (uint32_t)kTileQ * 2u;
         lmask_off = o;  // candidate bits of each listed token (two words)
         o += (uint32_t)kTileQ * 8u;
-        perm_off = o;
-        o += (uint32_t)kTileQ * 2u;
+        ent_off = o;  // packed sum entries sorted by cluster (runs padded to even length)
+        o += (uint32_t)(kTileQ + 64) * 4u;
         misc_off = o;
         o += 64;
         bar_off = o;  // two mbarriers and the tensor-memory address
@@ -319,15 +294,11 @@ struct AssignParams {
     int32_t *assign;     // [NH][L]
     int32_t *hist;       // [NH][iters][L] or null (already offset by the iteration)
     int64_t hist_stride; // iters * L
-    double *part_sum;    // [NH][Kp][n_tiles][64]
-    int *part_cnt;       // [NH][Kp][n_tiles]
-    int L, K, n_tiles;
-    int first;           // 1: first Lloyd iteration; 0: the slots hold the previous iteration's sums
+    double *sum;         // [NH][Kp][64] exact running member sums (red.global.add; coordinate j at 16 (j mod 4) + j / 4)
+    int *cnt;            // [NH][Kp] running member counts
+    int L, K;
+    int first;           // 1: first Lloyd iteration (the sums are clear); 0: they hold the previous assignment's
 };
-
-// Later iterations move at most this many tokens of a tile by exact fp64
-// subtract / add on the tile's slot; more movers recompute the tile's sums.
-constexpr int kMoverMax = 96;
 
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src));
@@ -354,17 +325,15 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     const uint32_t bar_tma = sbase + lay.bar_off, bar_mma = bar_tma + 8;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + lay.bar_off + 16);
     unsigned char *qbytes = smem + lay.q_off;
-    float *mu = reinterpret_cast<float *>(smem + lay.mu_off);        // [Kp][65] until the re-measure ends
-    double *ssum = reinterpret_cast<double *>(smem + lay.r_off);     // [Kp][64] after it
+    float *mu = reinterpret_cast<float *>(smem + lay.mu_off);        // [Kp][65]
     float *mm = reinterpret_cast<float *>(smem + lay.mm_off);
     int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
     uint8_t *dead = smem + lay.dead_off;
     uint8_t *cs = smem + lay.c_off;
-    uint8_t *sc = smem + lay.sc_off;
     uint8_t *cprev = smem + lay.cprev_off;
     uint16_t *list = reinterpret_cast<uint16_t *>(smem + lay.list_off);
     uint32_t *lmask = reinterpret_cast<uint32_t *>(smem + lay.lmask_off);
-    uint16_t *perm = reinterpret_cast<uint16_t *>(smem + lay.perm_off);
+    uint32_t *ent = reinterpret_cast<uint32_t *>(smem + lay.ent_off);
     int *misc = reinterpret_cast<int *>(smem + lay.misc_off);
     constexpr int mu_ld = 65;
 
@@ -571,58 +540,47 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
         P.assign[head * P.L + t0 + i] = cs[i];
         if (P.hist) P.hist[head * P.hist_stride + t0 + i] = cs[i];
     }
-    if (!P.first) {
-        // Later iterations list the tokens whose cluster changed; when they
-        // are few, only they move between the tile's member sums (exact fp64
-        // subtract / add on the slot) and counts.
-        for (int ch = warp; ch < kTileQ / 32; ch += kWarps) {
-            const int i = ch * 32 + lane;
-            const bool mv = i < Lt && cs[i] != cprev[i];
-            const unsigned bal = __ballot_sync(0xffffffffu, mv);
-            int base = 0;
-            if (lane == 0 && bal) base = atomicAdd(&misc[3], __popc(bal));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (mv) list[base + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)i;
-        }
-        __syncthreads();
-        const int n_mv = misc[3];
-        if (n_mv <= kMoverMax) {
-            double *psum = P.part_sum;
-            for (int e = warp; e < n_mv; e += kWarps) {
-                const int row = CA_IDX(list[e], 0, Lt, 65);
-                const int co = CA_IDX(cprev[row], 0, Kp, 66), cn = CA_IDX(cs[row], 0, Kp, 66);
-                const uint32_t w = *reinterpret_cast<const uint32_t *>(qbytes + swz(row, lane >> 2) + (lane & 3) * 4);
-                const double d0 = bf16_to_f64(w & 0xffffu), d1 = bf16_to_f64(w >> 16);
-                double *so = psum + ((cb + co) * P.n_tiles + tile) * kD;
-                double *sn = psum + ((cb + cn) * P.n_tiles + tile) * kD;
-                atomicAdd(&so[2 * lane], -d0);
-                atomicAdd(&so[2 * lane + 1], -d1);
-                atomicAdd(&sn[2 * lane], d0);
-                atomicAdd(&sn[2 * lane + 1], d1);
-                if (lane == 0) {
-                    atomicSub(&P.part_cnt[(cb + co) * P.n_tiles + tile], 1);
-                    atomicAdd(&P.part_cnt[(cb + cn) * P.n_tiles + tile], 1);
-                }
-            }
-            return;
-        }
+    // The tile's share of the head's running sums and counts: in the first
+    // iteration every token is added; later, every token whose cluster
+    // changed is subtracted from its old cluster and added to its new one.
+    double *gsum = P.sum + cb * kD;
+    int *gcnt = P.cnt + cb;
+    if (P.first) {
+        tile::counting_sort_even([&](int i) { return (int)cs[i]; }, [](int i) { return (uint32_t)i; }, kTileQ / 32, Kp,
+                                 cnt_s, ent, &misc[4], warp, kWarps, lane);
+        const int n2 = misc[4], seg = ((n2 >> 1) + kWarps - 1) / kWarps * 2;
+        tile::run_sums_red(qbytes, ent, warp * seg, min(n2, (warp + 1) * seg), gsum, gcnt, lane);
+        return;
     }
-    // Full member sums of the tile into shared memory (region R is free now
-    // that the MMA and the re-measure are done).
-    for (int e = threadIdx.x; e < Kp * kD / 2; e += kThreads)
-        reinterpret_cast<double2 *>(ssum)[e] = make_double2(0.0, 0.0);
-    tile::counting_sort(cs, kTileQ / 32, Kp, cnt_s, perm, sc, warp, kWarps, lane);
-    {
-        const int seg = (Lt + kWarps - 1) / kWarps;
-        tile::member_sums(qbytes, sc, perm, warp * seg, min(Lt, (warp + 1) * seg), ssum, lane);
+    for (int ch = warp; ch < kTileQ / 32; ch += kWarps) {
+        const int i = ch * 32 + lane;
+        const bool mv = i < Lt && cs[i] != cprev[i];
+        const unsigned bal = __ballot_sync(0xffffffffu, mv);
+        int base = 0;
+        if (lane == 0 && bal) base = atomicAdd(&misc[3], __popc(bal));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (mv) list[base + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)i;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < Kp * kD / 2; e += kThreads) {
-        const int kk = (2 * e) / kD, j = (2 * e) % kD;
-        *reinterpret_cast<double2 *>(P.part_sum + ((cb + kk) * P.n_tiles + tile) * kD + j) =
-            reinterpret_cast<const double2 *>(ssum)[e];
+    const int n_mv = misc[3];
+    // batches of up to 256 movers: entry e < m adds mover b + e to its new
+    // cluster, entry m + e subtracts it from its old one
+    for (int b = 0; b < n_mv; b += kTileQ / 2) {
+        const int m = min(kTileQ / 2, n_mv - b);
+        for (int kk = threadIdx.x; kk < Kp; kk += kThreads) cnt_s[kk] = 0;
+        __syncthreads();
+        auto row_of = [&](int e) { return CA_IDX((int)list[b + (e < m ? e : e - m)], 0, Lt, 65); };
+        auto cl = [&](int e) {
+            if (e >= 2 * m) return 0xFF;
+            const int row = row_of(e);
+            return CA_IDX((int)(e < m ? cs[row] : cprev[row]), 0, Kp, 66);
+        };
+        auto info = [&](int e) { return (uint32_t)row_of(e) | (e < m ? 0u : tile::kEntNeg); };
+        tile::counting_sort_even(cl, info, kTileQ / 32, Kp, cnt_s, ent, &misc[4], warp, kWarps, lane);
+        const int n2 = misc[4], seg = ((n2 >> 1) + kWarps - 1) / kWarps * 2;
+        tile::run_sums_red(qbytes, ent, warp * seg, min(n2, (warp + 1) * seg), gsum, gcnt, lane);
+        __syncthreads();
     }
-    for (int kk = threadIdx.x; kk < Kp; kk += kThreads) P.part_cnt[(cb + kk) * P.n_tiles + tile] = cnt_s[kk];
 }
 
 // ---------------------------------------------------------------------------
@@ -1203,18 +1161,21 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
         umma::tmem_ld_wait();
 #pragma unroll
         for (int t = 0; t < HALF; ++t) asm volatile("" : "+f"(v[t]));  // used only after the wait
+        // Scores outside [lo, hi] become -inf (their weight ex2(-inf) is
+        // +0).  A piece inside the band of every row of the warp (a
+        // warp-uniform test) needs no mask, so no branch diverges.
+        const int lo_w = __reduce_max_sync(0xffffffffu, lo), hi_w = __reduce_min_sync(0xffffffffu, hi);
 #pragma unroll
         for (int pc = 0; pc < NP; ++pc) {
             const int cb = cb0 + 16 * pc;
-            if (cb >= lo && cb + 15 <= hi) {
-#pragma unroll
-                for (int t = 0; t < 16; ++t) m = fmaxf(m, v[16 * pc + t]);
-            } else {
+            if (!(cb >= lo_w && cb + 15 <= hi_w)) {
 #pragma unroll
                 for (int t = 0; t < 16; ++t)
-                    if ((unsigned)(cb + t - lo) <= (unsigned)(hi - lo)) m = fmaxf(m, v[16 * pc + t]);
+                    if ((unsigned)(cb + t - lo) > (unsigned)(hi - lo)) v[16 * pc + t] = -INFINITY;
             }
         }
+#pragma unroll
+        for (int t = 0; t < HALF; ++t) m = fmaxf(m, v[t]);
     }
     red[wg * 128 + i] = m;
     __syncthreads();
@@ -1234,24 +1195,12 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
         for (int pc = 0; pc < NP; ++pc) {
             const int cb = cb0 + 16 * pc;
             uint32_t pk[8];
-            if (cb >= lo && cb + 15 <= hi) {
 #pragma unroll
-                for (int t = 0; t < 16; t += 2) {
-                    const float p0 = fused::ex2(fmaf(v[16 * pc + t], csc, -mc));
-                    const float p1 = fused::ex2(fmaf(v[16 * pc + t + 1], csc, -mc));
-                    l += p0 + p1;
-                    pk[t >> 1] = pack_bf16(p0, p1);
-                }
-            } else {
-#pragma unroll
-                for (int t = 0; t < 16; t += 2) {
-                    const bool in0 = (unsigned)(cb + t - lo) <= (unsigned)(hi - lo);
-                    const bool in1 = (unsigned)(cb + t + 1 - lo) <= (unsigned)(hi - lo);
-                    const float p0 = in0 ? fused::ex2(fmaf(v[16 * pc + t], csc, -mc)) : 0.f;
-                    const float p1 = in1 ? fused::ex2(fmaf(v[16 * pc + t + 1], csc, -mc)) : 0.f;
-                    l += p0 + p1;
-                    pk[t >> 1] = pack_bf16(p0, p1);
-                }
+            for (int t = 0; t < 16; t += 2) {
+                const float p0 = fused::ex2(fmaf(v[16 * pc + t], csc, -mc));
+                const float p1 = fused::ex2(fmaf(v[16 * pc + t + 1], csc, -mc));
+                l += p0 + p1;
+                pk[t >> 1] = pack_bf16(p0, p1);
             }
 #pragma unroll
             for (int q = 0; q < 2; ++q)
