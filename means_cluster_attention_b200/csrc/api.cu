@@ -145,7 +145,9 @@ ca_status ensure_kernel_attributes() {
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
@@ -345,20 +347,23 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         CA_CUDA(cudaGetLastError());
     }
 
-    const tiled::CentroidLayout clay(K);
-    tiled::CentroidParams cp{};
-    cp.k = k;
-    cp.v = v;
-    cp.hi = hi;
-    cp.part = cpart;
-    cp.L = L;
-    cp.K = K;
-    cp.n_chunks = n_chunks;
-    cp.scale = scale;
     {
+        CUtensorMap kmap256, vmap256;
+        ca_status ms = encode_rows_map(&kmap256, k, NH, L, 256);
+        if (ms == CA_OK) ms = encode_rows_map(&vmap256, v, NH, L, 256);
+        if (ms != CA_OK) return ms;
+        tiled::CentroidTcParams cp{};
+        cp.hi = hi;
+        cp.part = cpart;
+        cp.L = L;
+        cp.K = K;
+        cp.n_chunks = n_chunks;
+        cp.scale = scale;
+        const tiled::CentroidTcLayout clay(Kp);
+        auto kern = Kp == 16 ? tiled::tiled_centroid_tc_kernel<16>
+                             : (Kp == 32 ? tiled::tiled_centroid_tc_kernel<32> : tiled::tiled_centroid_tc_kernel<64>);
         Launch pl("tiled_centroid", st, 2.0 * head_bytes);
-        CA_CUDA(launch_pdl(tiled::tiled_centroid_kernel, dim3(n_chunks, (unsigned)NH), dim3(tiled::kThreads), clay.total,
-                           st, cp));
+        CA_CUDA(launch_pdl(kern, dim3(n_chunks, (unsigned)NH), dim3(256), clay.total, st, kmap256, vmap256, cp));
         pl.after();
     }
     CA_CUDA(cudaGetLastError());

@@ -16,8 +16,9 @@
 //                                          exact fp64 re-measure of ambiguous
 //                                          tokens, the tile's exact share of
 //                                          the head's running member sums.
-//   tiled_centroid_kernel  (chunks, heads) partial softmax state of every
-//                                          centroid over 512 keys;
+//   tiled_centroid_tc_kernel (chunks, heads) partial softmax state of every
+//                                          centroid over 512 keys on tcgen05
+//                                          (M = 64 tiles at two lane offsets);
 //   tiled_combine_kernel   (K, heads)      combines the chunk states into
 //                                          V_cent.
 //   tiled_window_tc_kernel (blocks, heads) clipped window attention for 128
@@ -58,8 +59,6 @@ constexpr int kThreads = 256;
 constexpr int kWarps = 8;
 constexpr int kTileQ = 512;   // queries per assignment tile
 constexpr int kChunk = 512;   // keys per centroid-attention CTA
-constexpr int kTile = 64;
-constexpr int kSlots = 5;
 constexpr int kWinQ = 128;    // queries per window CTA
 constexpr int kMaxR = 128;    // largest window radius floor(W/2)
 constexpr int kNTChunk = 6;   // key n-tiles per online-softmax step in the window
@@ -584,230 +583,304 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
 }
 
 // ---------------------------------------------------------------------------
-// Centroid attention over a chunk of up to 512 keys: the chunk's softmax
-// state (sum of exp-weighted V rows, running max in natural-log units, and
-// running denominator) for every centroid, in the layout of
-// centroid_attn_combine_kernel: part[head][chunk][K][64 + 2].
-struct CentroidLayout {
-    int Kp;
-    uint32_t slots_off, hi_off, ml_off, total;
-    __host__ __device__ CentroidLayout(int K) {
-        Kp = kpad(K);
+// Centroid attention over a chunk of up to 512 keys on tcgen05: the chunk's
+// softmax state of every centroid (sum of exp-weighted V rows, max in
+// natural-log units, denominator) in the layout tiled_combine_kernel reads.
+//
+// The chunk goes in two steps of 256 keys.  S = mu K^T runs as M = 64
+// tcgen05.mma tiles (rows = centroids) at tensor-memory lane offsets 0 and
+// 16, so the two tiles together fill all 128 lanes: tile o takes keys
+// [128 o, 128 o + 128) of the step.  Within a tile, G = 64 / KP groups of
+// rows each see their own 2 KP keys: the A operand of group g is a 64-row
+// window into a zero-padded copy of the centroids that holds them at rows
+// [g KP, (g + 1) KP) and zeros elsewhere, and the G products accumulate into
+// one [64 x 2 KP] tile.  Each row's softmax weights go to shared memory at
+// its own keys (block-diagonal P, zeros elsewhere), so one P V product per
+// tile gives every row the weighted sum over its own keys.  Two threads
+// (warpgroups) share a row: KP scores each.  Every thread folds its row's
+// step results into a running state; the rows of one centroid (tiles and
+// groups) are merged at the end.  K / V of the next step are loaded by TMA
+// while this one computes.
+struct CentroidTcLayout {
+    uint32_t z_off, k_off, v_off, p_off, red_off, bar_off, total;
+    __host__ __device__ CentroidTcLayout(int Kp) {
         uint32_t o = 0;
-        slots_off = o;
-        const uint32_t slots = (uint32_t)kSlots * 2u * kTile * 128u;
-        const uint32_t comb = (uint32_t)kWarps * 16u * 64u * 4u;
-        o += up(slots > comb ? slots : comb, 1024);
-        hi_off = o;
-        o += (uint32_t)Kp * 128u;
-        ml_off = o;
-        o += (uint32_t)kWarps * 16u * 2u * 4u;
-        total = up(o, 128);
+        z_off = o;  // (128 - Kp) rows of 128 bytes: zeros, the centroids at rows [64 - Kp, 64), zeros
+        o += up((uint32_t)(128 - Kp) * 128u, 1024);
+        k_off = o;  // 256 keys x 128 bytes
+        o += 256u * 128u;
+        v_off = o;
+        o += 256u * 128u;
+        p_off = o;  // P of tile o: 64 rows x 128 keys (two 64-key slabs of 8 KB), o = 0, 1
+        o += 2u * 16384u;
+        red_off = o;  // [2][128] half-row maxima, then [2][128] half-row sums
+        o += 2u * 2u * 128u * 4u;
+        bar_off = o;  // four mbarriers, the tensor-memory address
+        o += 48;
+        total = up(o, 128) + 1024;  // + slack to align the base to 1024 bytes
     }
 };
 
-struct CentroidParams {
-    const __nv_bfloat16 *k, *v;
-    const __nv_bfloat16 *hi;       // [NH][Kp][64] centroids rounded to bf16
-    float *part;                   // [NH][n_chunks][K][kPartLd]
+struct CentroidTcParams {
+    const __nv_bfloat16 *hi;  // [NH][Kp][64] centroids rounded to bf16
+    float *part;              // [NH][n_chunks][K][kPartLd]
     int L, K, n_chunks;
     float scale;
 };
 
-__global__ void __launch_bounds__(kThreads, 2) tiled_centroid_kernel(CentroidParams P) {
-    extern __shared__ __align__(1024) unsigned char smem[];
-    const CentroidLayout lay(P.K);
-    const int K = P.K, Kp = lay.Kp;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+template <int KP>
+__global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_constant__ CUtensorMap tmk,
+                                                                     const __grid_constant__ CUtensorMap tmv,
+                                                                     CentroidTcParams P) {
+    constexpr int G = 64 / KP;      // row groups per M = 64 tile
+    constexpr int N = 2 * KP;       // keys per group (S columns)
+    constexpr uint32_t kOCol = 128; // O columns [128, 192)
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const CentroidTcLayout lay(KP);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q = warp & 3, wg = warp >> 2;
+    const int L = P.L, K = P.K;
     const int chunk = blockIdx.x;
     const int64_t head = blockIdx.y;
-    const int k0 = chunk * kChunk;
-    const int Lc = min(kChunk, P.L - k0);
-    const int nT = (Lc + kTile - 1) / kTile;
-    const __nv_bfloat16 *kh = P.k + (head * P.L + k0) * kD;
-    const __nv_bfloat16 *vh = P.v + (head * P.L + k0) * kD;
-    const uint32_t sbase = smem_u32(smem);
-    const uint32_t slot_s = sbase + lay.slots_off, hi_s = sbase + lay.hi_off;
-    float *ml = reinterpret_cast<float *>(smem + lay.ml_off);
+    const int c0 = chunk * kChunk;
+    const int nsteps = min(2, (L - c0 + 255) / 256);
+    const uint32_t sb = smem_u32(smem);
+    const uint32_t z_s = sb + lay.z_off, k_s = sb + lay.k_off, v_s = sb + lay.v_off, p_s = sb + lay.p_off;
+    const uint32_t bar_k = sb + lay.bar_off, bar_v = bar_k + 8, bar_s = bar_k + 16, bar_o = bar_k + 24;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + lay.bar_off + 32);
+    float *red = reinterpret_cast<float *>(smem + lay.red_off);
 
     pdl_launch();
-    for (int s = 0; s < kSlots; ++s) {
-        if (s < nT) {
-            const uint32_t slot = slot_s + s * 2 * kTile * 128;
-            load_rows(slot, kh, s * kTile, kTile, Lc);
-            load_rows(slot + kTile * 128, vh, s * kTile, kTile, Lc);
-        }
-        cp_async_commit();
+    if (tid == 0) {
+        umma::mbar_init(bar_k, 1);
+        umma::mbar_init(bar_v, 1);
+        umma::mbar_init(bar_s, 1);
+        umma::mbar_init(bar_o, 1);
+        umma::mbar_init_fence();
+        umma::mbar_expect_tx(bar_k, 256u * 128u);
+        umma::tma_load_3d(k_s, &tmk, 0, c0, (int)head, bar_k);
+        umma::mbar_expect_tx(bar_v, 256u * 128u);
+        umma::tma_load_3d(v_s, &tmv, 0, c0, (int)head, bar_v);
     }
+    // P starts as zeros (each row later writes only its own keys)
+    for (int e = tid; e < 2 * 16384 / 16; e += 256)
+        asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};\n" ::"r"(p_s + (uint32_t)e * 16u), "r"(0u) : "memory");
     pdl_wait();  // the centroids come from the previous kernel
-    const int64_t cb = head * Kp;
-    for (int e = threadIdx.x; e < Kp * 8; e += kThreads) {
-        const int kk = e >> 3, ch = e & 7;
-        *reinterpret_cast<uint4 *>(smem + lay.hi_off + swz(kk, ch)) = *reinterpret_cast<const uint4 *>(P.hi + (cb + kk) * kD + ch * 8);
+    __syncwarp();
+    if (warp == 0) umma::tmem_alloc(smem_u32(tslot), 256u);
+    {
+        const __nv_bfloat16 *hh = P.hi + head * KP * kD;
+        for (int e = tid; e < (128 - KP) * 8; e += 256) {
+            const int row = e >> 3, ch = e & 7, kk = row - (64 - KP);
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            if (kk >= 0 && kk < KP) w = *reinterpret_cast<const uint4 *>(hh + kk * kD + ch * 8);
+            *reinterpret_cast<uint4 *>(smem + lay.z_off + swz(row, ch)) = w;
+        }
     }
+    umma::fence_proxy_async_smem();
+    umma::tc_fence_before();
     __syncthreads();
-    const int n_cm = Kp / 16, G = kWarps / n_cm, cm = warp / G, kb = warp % G, keys_w = kTile / G;
-    const float csc = P.scale * kLog2e;
-    // Scores use the centroids rounded once to bf16: the weights P are
-    // rounded to bf16 as well, and the error this adds to a logit
-    // (|mu| |K| 2^-9 / sqrt(d) at worst, far less on average) stays well
-    // below the output tolerance.
-    uint32_t ahi[4][4];
+    umma::tc_fence_after();
+    const uint32_t taddr = *tslot;
+
+    // This thread: tensor-memory lane tl = 32 q + lane holds row r of tile o.
+    const int tl = 32 * q + lane, o = lane >> 4, r = 16 * q + (lane & 15);
+    const int g = r / KP, kc = r % KP;  // row group, centroid
+    const int blk = o * G + g;          // key block of the row within a step
+    const float csc = P.scale * fused::kLog2e;
+    const uint32_t trow = taddr + ((uint32_t)(32 * q) << 16);
+    float m_run = -INFINITY, l_run = 0.f, acc[32];
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-        const int m = lane >> 3;
-        const int row = cm * 16 + (lane & 7) + ((m & 1) ? 8 : 0);
-        ldmatrix_x4(ahi[ks], hi_s + swz(row, 2 * ks + (m >> 1)));
-    }
-    float o_acc[8][4];
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+    bool ok = true;
+    int k_issued = 1, v_issued = 1;  // loads issued (completions waited so far: s for K, s for V)
+    for (int s = 0; s < nsteps; ++s) {
+        const uint32_t par = (uint32_t)s & 1u;
+        ok = __syncthreads_and(ok && umma::mbar_wait(bar_k, par));
+        if (!ok) break;
+        if (tid == 0) {
+            constexpr uint32_t idesc = umma::idesc_bf16_f32(64, N);
 #pragma unroll
-    for (int d = 0; d < 8; ++d)
+            for (int oo = 0; oo < 2; ++oo)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o_acc[d][e] = 0.f;
-    float rm[2] = {-INFINITY, -INFINITY}, rl[2] = {0.f, 0.f};
-    for (int tt = 0; tt < nT; ++tt) {
-        cp_async_wait<kSlots - 1>();
-        __syncthreads();
-        const uint32_t kt = slot_s + (tt % kSlots) * 2 * kTile * 128;
-        const uint32_t vt = kt + kTile * 128;
-        float sacc[4][4];
+                for (int gg = 0; gg < G; ++gg) {
+                    const uint32_t a0 = z_s + (uint32_t)((64 - KP) - gg * KP) * 128u;
+                    const uint32_t b0 = k_s + (uint32_t)((oo * G + gg) * N) * 128u;
 #pragma unroll
-        for (int n = 0; n < 4; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sacc[n][e] = 0.f;
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            if (n * 8 >= keys_w) break;
-            const int key0 = kb * keys_w + n * 8;
-#pragma unroll
-            for (int kp = 0; kp < 2; ++kp) {
-                uint32_t bk[4];
-                ldmatrix_x4(bk, kt + swz(key0 + (lane & 7), 4 * kp + (lane >> 3)));
-                mma_16816(sacc[n], ahi[2 * kp], bk[0], bk[1]);
-                mma_16816(sacc[n], ahi[2 * kp + 1], bk[2], bk[3]);
-            }
-        }
-        float tmax[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            if (n * 8 >= keys_w) break;
-            const int key = tt * kTile + kb * keys_w + n * 8 + 2 * t;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                if (key + (e & 1) >= Lc) sacc[n][e] = -INFINITY;
-            tmax[0] = fmaxf(tmax[0], fmaxf(sacc[n][0], sacc[n][1]));
-            tmax[1] = fmaxf(tmax[1], fmaxf(sacc[n][2], sacc[n][3]));
-        }
-        float corr[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 1));
-            tmax[h] = fmaxf(tmax[h], __shfl_xor_sync(0xffffffffu, tmax[h], 2));
-            const float mn = fmaxf(rm[h], tmax[h]);
-            corr[h] = (mn == -INFINITY) ? 1.f : ex2((rm[h] - mn) * csc);
-            rm[h] = mn;
-            rl[h] *= corr[h];
-        }
-#pragma unroll
-        for (int d = 0; d < 8; ++d) {
-            o_acc[d][0] *= corr[0];
-            o_acc[d][1] *= corr[0];
-            o_acc[d][2] *= corr[1];
-            o_acc[d][3] *= corr[1];
-        }
-        uint32_t pa[4][2];
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            pa[n][0] = pa[n][1] = 0u;
-            if (n * 8 >= keys_w) break;
-            float p[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float mh = rm[e >> 1];
-                p[e] = (mh == -INFINITY) ? 0.f : ex2((sacc[n][e] - mh) * csc);
-            }
-            rl[0] += p[0] + p[1];
-            rl[1] += p[2] + p[3];
-            pa[n][0] = pack_bf16(p[0], p[1]);
-            pa[n][1] = pack_bf16(p[2], p[3]);
-        }
-        if (keys_w == 8) {
-            const int key0 = kb * keys_w;
-#pragma unroll
-            for (int dq = 0; dq < 2; ++dq) {
-                uint32_t bv[4];
-                ldmatrix_x4_trans(bv, vt + swz(key0 + (lane & 7), 4 * dq + (lane >> 3)));
-#pragma unroll
-                for (int u = 0; u < 4; ++u) mma_1688(o_acc[4 * dq + u], pa[0][0], pa[0][1], bv[u]);
-            }
-        } else {
-#pragma unroll
-            for (int n2 = 0; n2 < 2; ++n2) {
-                if (n2 * 16 >= keys_w) break;
-                const uint32_t a4[4] = {pa[2 * n2][0], pa[2 * n2][1], pa[2 * n2 + 1][0], pa[2 * n2 + 1][1]};
-                const int key0 = kb * keys_w + n2 * 16;
-#pragma unroll
-                for (int dq = 0; dq < 4; ++dq) {
-                    uint32_t bv[4];
-                    const int m = lane >> 3;
-                    ldmatrix_x4_trans(bv, vt + swz(key0 + (lane & 7) + ((m & 1) ? 8 : 0), 2 * dq + (m >> 1)));
-                    mma_16816(o_acc[2 * dq], a4, bv[0], bv[1]);
-                    mma_16816(o_acc[2 * dq + 1], a4, bv[2], bv[3]);
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma::mma_bf16(taddr + ((uint32_t)(16 * oo) << 16), umma::desc_sw128(a0 + (uint32_t)ks * 32u),
+                                       umma::desc_sw128(b0 + (uint32_t)ks * 32u), idesc, gg > 0 || ks > 0);
                 }
+            umma::mma_commit(bar_s);
+        }
+        ok = __syncthreads_and(umma::mbar_wait(bar_s, par));
+        if (!ok) break;
+        umma::tc_fence_after();
+        // this thread's KP scores: columns [wg KP, wg KP + KP) of its row
+        float v[KP];
+#pragma unroll
+        for (int pc = 0; pc < KP / 16; ++pc) {
+            float t16[16];
+            umma::tmem_ld16(trow + (uint32_t)(wg * KP + 16 * pc), t16);
+#pragma unroll
+            for (int t = 0; t < 16; ++t) v[16 * pc + t] = t16[t];
+        }
+        umma::tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < KP; ++t) asm volatile("" : "+f"(v[t]));
+        const int key0 = c0 + 256 * s + blk * N + wg * KP;  // key of v[0]
+        if (c0 + 256 * (s + 1) > L) {  // keys past L (zero rows of the load) do not exist
+#pragma unroll
+            for (int t = 0; t < KP; ++t)
+                if (key0 + t >= L) v[t] = -INFINITY;
+        }
+        float m = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < KP; ++t) m = fmaxf(m, v[t]);
+        red[wg * 128 + tl] = m;
+        __syncthreads();
+        m = fmaxf(red[tl], red[128 + tl]);
+        const float mc = (m == -INFINITY) ? 0.f : m * csc;
+        float l = 0.f;
+        {
+            const uint32_t prow = p_s + (uint32_t)o * 16384u;
+            const int kb = g * N + wg * KP;  // first key column of this thread in the tile's P
+#pragma unroll
+            for (int c8 = 0; c8 < KP / 8; ++c8) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int t = 0; t < 8; t += 2) {
+                    const float p0 = fused::ex2(fmaf(v[8 * c8 + t], csc, -mc));
+                    const float p1 = fused::ex2(fmaf(v[8 * c8 + t + 1], csc, -mc));
+                    l += p0 + p1;
+                    pk[t >> 1] = pack_bf16(p0, p1);
+                }
+                const int col = kb + 8 * c8;
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(prow + (uint32_t)(col >> 6) * 8192u +
+                                                                              swz(r, (col & 63) >> 3)),
+                             "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                             : "memory");
             }
+        }
+        red[256 + wg * 128 + tl] = l;
+        umma::fence_proxy_async_smem();
+        umma::tc_fence_before();
+        __syncthreads();
+        umma::tc_fence_after();
+        if (tid == 0) {
+            // K of the next step into the buffer the S product has finished reading
+            if (s + 1 < nsteps) {
+                umma::mbar_expect_tx(bar_k, 256u * 128u);
+                umma::tma_load_3d(k_s, &tmk, 0, c0 + 256 * (s + 1), (int)head, bar_k);
+                ++k_issued;
+            }
+            if (umma::mbar_wait(bar_v, par)) {
+                constexpr uint32_t idesc = umma::idesc_bf16_f32_bmn(64, 64);
+#pragma unroll
+                for (int oo = 0; oo < 2; ++oo)
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        umma::mma_bf16(taddr + ((uint32_t)(16 * oo) << 16) + kOCol,
+                                       umma::desc_sw128(p_s + (uint32_t)oo * 16384u + (uint32_t)(ks >> 2) * 8192u +
+                                                        (uint32_t)(ks & 3) * 32u),
+                                       umma::desc_sw128(v_s + (uint32_t)(oo * 128 + ks * 16) * 128u), idesc, ks > 0);
+                umma::mma_commit(bar_o);
+            } else {
+                record_error(4, 45);
+            }
+        }
+        l = red[256 + tl] + red[384 + tl];
+        ok = __syncthreads_and(umma::mbar_wait(bar_o, par));
+        if (!ok) break;
+        umma::tc_fence_after();
+        float ov[32];
+        umma::tmem_ld32(trow + kOCol + (uint32_t)(32 * wg), ov);
+        umma::tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) asm volatile("" : "+f"(ov[t]));
+        if (m != -INFINITY) {
+            const float M = fmaxf(m_run, m);
+            const float a = (m_run == -INFINITY) ? 0.f : fused::ex2((m_run - M) * csc);
+            const float b = fused::ex2((m - M) * csc);
+#pragma unroll
+            for (int t = 0; t < 32; ++t) acc[t] = fmaf(acc[t], a, ov[t] * b);
+            l_run = fmaf(l_run, a, l * b);
+            m_run = M;
+        }
+        umma::tc_fence_before();
+        __syncthreads();
+        umma::tc_fence_after();
+        if (tid == 0 && s + 1 < nsteps) {
+            // V of the next step into the buffer the P V product has finished reading
+            umma::mbar_expect_tx(bar_v, 256u * 128u);
+            umma::tma_load_3d(v_s, &tmv, 0, c0 + 256 * (s + 1), (int)head, bar_v);
+            ++v_issued;
+        }
+    }
+    if (!ok && tid == 0) {
+        record_error(4, 44);
+        // no load may still be writing this block's shared memory when it
+        // exits: wait (bounded) for the last K and V loads issued
+        umma::mbar_wait(bar_k, (uint32_t)(k_issued - 1) & 1u);
+        umma::mbar_wait(bar_v, (uint32_t)(v_issued - 1) & 1u);
+    }
+    // Merge the rows of one centroid: the two tiles (lanes l and l ^ 16),
+    // then the G row groups (quadrants) through shared memory.
+    auto merge = [&](float m2, float l2, const float *a2) {
+        const float M = fmaxf(m_run, m2);
+        if (M == -INFINITY) return;
+        const float fa = (m_run == -INFINITY) ? 0.f : fused::ex2((m_run - M) * csc);
+        const float fb = (m2 == -INFINITY) ? 0.f : fused::ex2((m2 - M) * csc);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) acc[t] = fmaf(acc[t], fa, a2[t] * fb);
+        l_run = fmaf(l_run, fa, l2 * fb);
+        m_run = M;
+    };
+    {
+        float a2[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) a2[t] = __shfl_xor_sync(0xffffffffu, acc[t], 16);
+        const float m2 = __shfl_xor_sync(0xffffffffu, m_run, 16), l2 = __shfl_xor_sync(0xffffffffu, l_run, 16);
+        merge(m2, l2, a2);
+    }
+    if constexpr (G > 1) {
+        // rows of group g > 0 hand their state to group 0 through the (dead) P buffer
+        float *xs = reinterpret_cast<float *>(smem + lay.p_off);  // [G][wg][KP][34]
+        __syncthreads();
+        if (g > 0 && o == 0) {
+            float *dst = xs + (((g * 2 + wg) * KP) + kc) * 34;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) dst[t] = acc[t];
+            dst[32] = m_run;
+            dst[33] = l_run;
         }
         __syncthreads();
-        if (tt + kSlots < nT) {
-            load_rows(kt, kh, (tt + kSlots) * kTile, kTile, Lc);
-            load_rows(vt, vh, (tt + kSlots) * kTile, kTile, Lc);
-        }
-        cp_async_commit();
-    }
-    cp_async_wait<0>();
-    float *part = reinterpret_cast<float *>(smem + lay.slots_off);
+        if (g == 0 && o == 0) {
+#pragma unroll 1
+            for (int g2 = 1; g2 < G; ++g2) {
+                const float *src = xs + (((g2 * 2 + wg) * KP) + kc) * 34;
+                float a2[32];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        rl[h] += __shfl_xor_sync(0xffffffffu, rl[h], 1);
-        rl[h] += __shfl_xor_sync(0xffffffffu, rl[h], 2);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int d = 0; d < 8; ++d) {
-        float *p0 = part + (warp * 16 + g) * 64 + 8 * d + 2 * t;
-        float *p1 = part + (warp * 16 + g + 8) * 64 + 8 * d + 2 * t;
-        p0[0] = o_acc[d][0];
-        p0[1] = o_acc[d][1];
-        p1[0] = o_acc[d][2];
-        p1[1] = o_acc[d][3];
-    }
-    if (t == 0) {
-        ml[(warp * 16 + g) * 2 + 0] = rm[0];
-        ml[(warp * 16 + g) * 2 + 1] = rl[0];
-        ml[(warp * 16 + g + 8) * 2 + 0] = rm[1];
-        ml[(warp * 16 + g + 8) * 2 + 1] = rl[1];
-    }
-    __syncthreads();
-    float *outp = P.part + ((head * P.n_chunks + chunk) * (int64_t)K) * kPartLd;
-    for (int e = threadIdx.x; e < K * kPartLd; e += kThreads) {
-        const int row = e / kPartLd, col = e % kPartLd;
-        const int mt = row / 16, rr = row % 16;
-        float M = -INFINITY;
-        for (int w = mt * G; w < mt * G + G; ++w) M = fmaxf(M, ml[(w * 16 + rr) * 2]);
-        float val;
-        if (col >= kD + 2) {
-            val = 0.f;  // padding
-        } else if (col == kD) {
-            val = M * P.scale;  // running max in natural-log units
-        } else {
-            float acc = 0.f;
-            for (int w = mt * G; w < mt * G + G; ++w) {
-                const float mw = ml[(w * 16 + rr) * 2];
-                const float f = (mw == -INFINITY) ? 0.f : ex2((mw - M) * csc);
-                acc = fmaf(col == kD + 1 ? ml[(w * 16 + rr) * 2 + 1] : part[(w * 16 + rr) * 64 + col], f, acc);
+                for (int t = 0; t < 32; ++t) a2[t] = src[t];
+                merge(src[32], src[33], a2);
             }
-            val = acc;
         }
-        outp[e] = val;
+    }
+    if (ok && g == 0 && o == 0 && kc < K) {
+        float *dst = P.part + ((head * P.n_chunks + chunk) * K + kc) * kPartLd;
+#pragma unroll
+        for (int t = 0; t < 32; t += 4)
+            *reinterpret_cast<float4 *>(dst + 32 * wg + t) = make_float4(acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
+        if (wg == 0) {
+            dst[kD] = m_run * P.scale;
+            dst[kD + 1] = l_run;
+        }
+    }
+    umma::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        umma::tc_fence_after();
+        umma::tmem_dealloc(taddr, 256u);
     }
 }
 
