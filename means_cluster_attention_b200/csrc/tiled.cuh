@@ -253,11 +253,11 @@ struct AssignLayout {
         q_off = o;  // 512 rows x 128 bytes, 1024-aligned (TMA / MMA swizzle)
         o += (uint32_t)kTileQ * 128u;
         // The MMA's B operand [hi; lo] (2 Kp rows of 128 bytes, 1024-aligned)
-        // beside the fp32 centroids (rows padded to 65 floats) for the exact
-        // re-measure.
+        // beside the fp32 centroids (rows padded to 68 floats: 16-byte
+        // copies) for the exact decisions.
         r_off = o;
         mu_off = o + 2u * (uint32_t)Kp * 128u;
-        o += up(2u * (uint32_t)Kp * 128u + (uint32_t)Kp * 65u * 4u, 16);
+        o += up(2u * (uint32_t)Kp * 128u + (uint32_t)Kp * 68u * 4u, 16);
         mm_off = o;
         o += (uint32_t)Kp * 4u;
         dead_off = o;
@@ -276,8 +276,8 @@ struct AssignLayout {
         o += (uint32_t)(kTileQ + 64) * 4u;
         misc_off = o;
         o += 64;
-        bar_off = o;  // two mbarriers and the tensor-memory address
-        o += 32;
+        bar_off = o;  // five mbarriers (queries, the products of each 128-row block) and the tensor-memory address
+        o += 64;
         total = up(o, 128) + 1024;  // + slack to align the base to 1024 bytes
     }
 };
@@ -299,10 +299,6 @@ struct AssignParams {
     int first;           // 1: first Lloyd iteration (the sums are clear); 0: they hold the previous assignment's
 };
 
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src));
-}
-
 template <int KP>
 __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_constant__ CUtensorMap tmq,
                                                                     AssignParams P) {
@@ -321,10 +317,10 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
 
     const uint32_t sbase = smem_u32(smem);
     const uint32_t q_s = sbase + lay.q_off, b_s = sbase + lay.r_off;
-    const uint32_t bar_tma = sbase + lay.bar_off, bar_mma = bar_tma + 8;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + lay.bar_off + 16);
+    const uint32_t bar_tma = sbase + lay.bar_off, bar_mma = bar_tma + 8;  // bar_mma + 8 m: block m
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + lay.bar_off + 48);
     unsigned char *qbytes = smem + lay.q_off;
-    float *mu = reinterpret_cast<float *>(smem + lay.mu_off);        // [Kp][65]
+    float *mu = reinterpret_cast<float *>(smem + lay.mu_off);        // [Kp][68]
     float *mm = reinterpret_cast<float *>(smem + lay.mm_off);
     int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
     uint8_t *dead = smem + lay.dead_off;
@@ -334,14 +330,15 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     uint32_t *lmask = reinterpret_cast<uint32_t *>(smem + lay.lmask_off);
     uint32_t *ent = reinterpret_cast<uint32_t *>(smem + lay.ent_off);
     int *misc = reinterpret_cast<int *>(smem + lay.misc_off);
-    constexpr int mu_ld = 65;
+    constexpr int mu_ld = 68;
 
     pdl_launch();
     // The query tile is an input of the forward: its load starts before the
     // previous kernel (the centroid update) has finished.
     if (threadIdx.x == 0) {
         umma::mbar_init(bar_tma, 1);
-        umma::mbar_init(bar_mma, 1);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) umma::mbar_init(bar_mma + 8u * m, 1);
         umma::mbar_init_fence();
         const int nbox = Lt > 256 ? 2 : 1;
         umma::mbar_expect_tx(bar_tma, (uint32_t)nbox * 256u * 128u);
@@ -361,8 +358,8 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
         cp_async16(b_s + swz(kk, ch), P.hi + (cb + kk) * kD + ch * 8, 16);
         cp_async16(b_s + (uint32_t)Kp * 128u + swz(kk, ch), P.lo + (cb + kk) * kD + ch * 8, 16);
     }
-    for (int e = threadIdx.x; e < Kp * kD; e += kThreads)
-        cp_async4(smem_u32(mu + (e / kD) * mu_ld + e % kD), P.mu + cb * kD + e);
+    for (int e = threadIdx.x; e < Kp * (kD / 4); e += kThreads)
+        cp_async16(smem_u32(mu + (e >> 4) * mu_ld + (e & 15) * 4), P.mu + cb * kD + e * 4, 16);
     cp_async_commit();
     float qn_g[2] = {0.f, 0.f};
     const int wg = warp >> 2, q4 = warp & 3;
@@ -405,8 +402,12 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     const bool q_ok = __syncthreads_and(umma::mbar_wait(bar_tma, 0));
     if (threadIdx.x == 0) {
         if (q_ok) {
+            // each 128-row block commits to its own barrier; blocks 0 and 2
+            // (the first of each warpgroup) go first
             constexpr uint32_t idesc = umma::idesc_bf16_f32(128, KP);
-            for (int m = 0; m < nblk; ++m)
+            for (int mo = 0; mo < 4; ++mo) {
+                const int m = (mo >> 1) | ((mo & 1) << 1);  // 0, 2, 1, 3
+                if (m >= nblk) continue;
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
@@ -415,7 +416,8 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
                                        umma::desc_sw128(q_s + (uint32_t)m * 16384u + (uint32_t)ks * 32u),
                                        umma::desc_sw128(b_s + (uint32_t)part * (uint32_t)Kp * 128u + (uint32_t)ks * 32u),
                                        idesc, part > 0 || ks > 0);
-            umma::mma_commit(bar_mma);
+                umma::mma_commit(bar_mma + 8u * (uint32_t)m);
+            }
         } else {
             record_error(4, 30);
         }
@@ -446,14 +448,17 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
             }
         }
     }
-    const bool mma_ok = __syncthreads_and(q_ok && umma::mbar_wait(bar_mma, 0));
-    if (!mma_ok && q_ok && threadIdx.x == 0) record_error(4, 31);
-    umma::tc_fence_after();
-    if (mma_ok) {
+    if (q_ok) {
 #pragma unroll
         for (int mi = 0; mi < 2; ++mi) {
             const int m = 2 * wg + mi;
             if (m >= nblk) break;  // uniform across the warp
+            // this block's products (the warp waits as one)
+            if (!__all_sync(0xffffffffu, umma::mbar_wait(bar_mma + 8u * (uint32_t)m, 0))) {
+                if (lane == 0) record_error(4, 31);
+                break;
+            }
+            umma::tc_fence_after();
             const int row = m * 128 + q4 * 32 + lane;
             float sv[KP];
             const uint32_t ta = taddr + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(m * KP);
