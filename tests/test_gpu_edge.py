@@ -284,3 +284,38 @@ def test_tiled_exact_ties_between_distinct_centroids():
     np.testing.assert_array_equal(g["cent"], ref_cent)
     tokens = [i for i in range(L) if i not in rows]
     assert (ref_assign[0, 0, tokens] == 0).all()
+
+
+def test_tiled_many_movers_two_batches():
+    """More than 256 tokens of one 512-query tile change cluster in one
+    iteration, so the tile's running-sum update runs in two batches of signed
+    entries.  Rows 0 and 512 (the strided starting centroids for K = 2) are
+    the same near-zero row: centroid 1 starts as a copy and takes nothing, so
+    the first update leaves it empty (the zero vector) while centroid 0 moves
+    to the mean of all rows; in the second iteration the 300 near-zero rows
+    of the first tile move to centroid 1."""
+    from means_cluster_attention_b200 import _lib
+    from means_cluster_attention_b200.inputs import bf16_bits_to_f64, bf16_round_bits
+    L, K, iters = 1024, 2, 3
+    rng = np.random.default_rng(11)
+    q = np.zeros((1, 1, L, 64), dtype=np.float32)
+    q[0, 0, :300] = 0.01 * rng.standard_normal((300, 64), dtype=np.float32)
+    q[0, 0, 300:] = 0.1 * rng.standard_normal((L - 300, 64), dtype=np.float32)
+    q[0, 0, 300:, 0] += 10.0
+    q[0, 0, 512] = q[0, 0, 0]
+    x = {}
+    for name, a in (("q", q), ("k", rng.standard_normal(q.shape, dtype=np.float32)),
+                    ("v", rng.standard_normal(q.shape, dtype=np.float32))):
+        x[name] = bf16_round_bits(a)
+        x[name + "64"] = bf16_bits_to_f64(x[name])
+    _lib.profile_start("tiled_assign")
+    g = run_gpu(x, "bf16", K, iters, 8, 0.5, hist=True)
+    assert _lib.profile_stop().launches == iters
+    ref_out, ref_assign, ref_cent, ref_hist = oracle.forward(x["q64"], x["k64"], x["v64"], K=K, iters=iters,
+                                                             W=8, alpha=0.5, hist=True)
+    moved_in_tile0 = int((ref_hist[0, 0, 1, :512] != ref_hist[0, 0, 0, :512]).sum())
+    assert moved_in_tile0 > 256, moved_in_tile0
+    np.testing.assert_array_equal(g["hist"], ref_hist)
+    np.testing.assert_array_equal(g["assign"], ref_assign)
+    np.testing.assert_array_equal(g["cent"], ref_cent)
+    assert float(np.abs(g["out"] - ref_out).max()) <= TOL["bf16"]
