@@ -251,10 +251,25 @@ bool tiled_eligible(int dtype, const Problem &p) {
     return dtype == 1 && p.K <= 64 && p.W / 2 <= ca::tiled::kMaxR;
 }
 
+// The module's variants the tiled path runs (the defaults give the forward
+// of the pages' formulas): window radius r (floor(W / 2), or W with
+// window_mode), no local branch (O = gathered), the module's stride init,
+// empty clusters keeping their centroid, grouped key/value heads.
+struct TiledVariant {
+    int r = 0, local = 1, init_stride = 0, empty_keep = 0, H_kv = 0;
+    static TiledVariant plain(const Problem &p) {
+        TiledVariant tv;
+        tv.r = p.W / 2;
+        tv.H_kv = p.H;
+        return tv;
+    }
+};
+
 ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v, const Problem &p,
-                    __nv_bfloat16 *out, int32_t *assign_out, float *cent_out, int32_t *hist, cudaStream_t st) {
+                    __nv_bfloat16 *out, int32_t *assign_out, float *cent_out, int32_t *hist, cudaStream_t st,
+                    const TiledVariant &tv) {
     using namespace ca;
-    const int64_t NH = p.heads();
+    const int64_t NH = p.heads(), NH_kv = (int64_t)p.B * tv.H_kv;
     const int L = p.L, K = p.K, Kp = tiled::kpad(K);
     const int n_chunks = (L + tiled::kChunk - 1) / tiled::kChunk;
     const float scale = 1.0f / sqrtf((float)p.d);
@@ -300,6 +315,8 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     up.K = K;
     up.Kp = Kp;
     up.init = 1;
+    up.init_stride = tv.init_stride;
+    up.empty_keep = tv.empty_keep;
     up.cent_out = p.iters == 0 ? cent_out : nullptr;
     {
         Launch pl("tiled_init", st, 0.0);
@@ -349,8 +366,8 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
 
     {
         CUtensorMap kmap256, vmap256;
-        ca_status ms = encode_rows_map(&kmap256, k, NH, L, 256);
-        if (ms == CA_OK) ms = encode_rows_map(&vmap256, v, NH, L, 256);
+        ca_status ms = encode_rows_map(&kmap256, k, NH_kv, L, 256);
+        if (ms == CA_OK) ms = encode_rows_map(&vmap256, v, NH_kv, L, 256);
         if (ms != CA_OK) return ms;
         tiled::CentroidTcParams cp{};
         cp.hi = hi;
@@ -358,6 +375,8 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         cp.L = L;
         cp.K = K;
         cp.n_chunks = n_chunks;
+        cp.H = p.H;
+        cp.H_kv = tv.H_kv;
         cp.scale = scale;
         const tiled::CentroidTcLayout clay(Kp);
         auto kern = Kp == 16 ? tiled::tiled_centroid_tc_kernel<16>
@@ -384,8 +403,12 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     wp.out = out;
     wp.L = L;
     wp.K = K;
-    wp.r = p.W / 2;
-    wp.alpha = p.alpha;
+    // without the local branch the epilogue blends with alpha = 0: O is the
+    // gathered row exactly, and the window is the smallest one
+    wp.r = tv.local ? tv.r : 0;
+    wp.alpha = tv.local ? p.alpha : 0.f;
+    wp.H = p.H;
+    wp.H_kv = tv.H_kv;
     wp.scale = scale;
     if (wp.r <= 64) {
         // tensor-core window kernel: the key window [q0 - RP, q0 + 127 + RP]
@@ -393,8 +416,8 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         const tiled::WindowTcLayout tlay(RP);
         CUtensorMap kmap, vmap, q128, o128;
         ca_status ms = encode_rows_map(&q128, q, NH, L, 128);
-        if (ms == CA_OK) ms = encode_rows_map(&kmap, k, NH, L, tlay.NK);
-        if (ms == CA_OK) ms = encode_rows_map(&vmap, v, NH, L, tlay.NK);
+        if (ms == CA_OK) ms = encode_rows_map(&kmap, k, NH_kv, L, tlay.NK);
+        if (ms == CA_OK) ms = encode_rows_map(&vmap, v, NH_kv, L, tlay.NK);
         if (ms == CA_OK) ms = encode_rows_map(&o128, out, NH, L, 128);
         if (ms != CA_OK) return ms;
         Launch pl("tiled_window", st, 4.0 * head_bytes);
@@ -402,7 +425,7 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
                            dim3((L + 127) / 128, (unsigned)NH), dim3(256), tlay.total, st, q128, kmap, vmap, o128, wp));
         pl.after();
     } else {
-        const tiled::WindowLayout wlay(K, p.W / 2);
+        const tiled::WindowLayout wlay(K, wp.r);
         Launch pl("tiled_window", st, 4.0 * head_bytes);
         CA_CUDA(launch_pdl(tiled::tiled_window_kernel, dim3((L + tiled::kWinQ - 1) / tiled::kWinQ, (unsigned)NH),
                            dim3(tiled::kThreads), wlay.total, st, wp));
@@ -528,7 +551,7 @@ ca_status dispatch(const void *q, const void *k, const void *v, int dtype, const
     if (tiled_eligible(dtype, p)) {
         NvtxRange range("ca_forward tiled");
         return run_tiled((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, p,
-                         (__nv_bfloat16 *)out, assign_out, cent_out, hist, st);
+                         (__nv_bfloat16 *)out, assign_out, cent_out, hist, st, TiledVariant::plain(p));
     }
     NvtxRange range("ca_forward general");
     if (dtype == 0)
@@ -598,6 +621,20 @@ ca_status ca_forward_ex(const void *q, const void *k, const void *v, int dtype, 
     s = ensure_kernel_attributes();
     if (s != CA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
+    // bf16 with grouped key/value heads, the radius window, the stride init or
+    // kept empty centroids: the tiled kernels (key masks and the soft gather
+    // stay on the general path)
+    if (dtype == 1 && !o.key_valid && !o.gather_mode && K <= 64 && (!ex.var.local || ex.r <= ca::tiled::kMaxR)) {
+        TiledVariant tv;
+        tv.r = ex.r;
+        tv.local = ex.var.local;
+        tv.init_stride = ex.init_stride;
+        tv.empty_keep = ex.empty_keep;
+        tv.H_kv = H_kv;
+        NvtxRange range("ca_forward_ex tiled");
+        return run_tiled((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, p,
+                         (__nv_bfloat16 *)out, assign_out, centroids_out, assign_hist, st, tv);
+    }
     if (dtype == 0)
         return run_forward<float>((const float *)q, (const float *)k, (const float *)v, p, (float *)out,
                                   assign_out, centroids_out, assign_hist, st, &ex);

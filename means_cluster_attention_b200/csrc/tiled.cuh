@@ -78,6 +78,8 @@ struct UpdateParams {
     float *mstat;            // [NH][2] max over k < K of |mu_k|^2, and its square root
     float *cent_out;         // [NH][K][64] or null
     int L, K, Kp, init;
+    int init_stride;         // 1: mu_k = Q[k max(1, L / K)] (the module's stride) instead of Q[floor(k L / K)]
+    int empty_keep;          // 1: an empty cluster keeps its previous centroid instead of becoming zero
 };
 
 // grid (NH), 1024 threads.  mu_k = Q[floor(k L / K)] (init; the running sums
@@ -110,7 +112,7 @@ __global__ void __launch_bounds__(kUpdThreads) tiled_update_kernel(UpdateParams 
         sv[u] = 0.0;
         if (k < K) {
             if (P.init) {
-                const int64_t row = ((int64_t)k * P.L) / K;
+                const int64_t row = P.init_stride ? (int64_t)k * max(1, P.L / K) : ((int64_t)k * P.L) / K;
                 sv[u] = (double)__bfloat162float(P.q[(head * P.L + row) * kD + j]);
             } else {
                 sv[u] = P.sum[(hb + k) * kD + (j & 3) * 16 + (j >> 2)];
@@ -126,7 +128,8 @@ __global__ void __launch_bounds__(kUpdThreads) tiled_update_kernel(UpdateParams 
         float x = 0.f;
         if (k < K) {
             const int n = ns[k];
-            x = P.init ? (float)sv[u] : __double2float_rn(sv[u] / (double)(n > 1 ? n : 1));
+            x = P.init ? (float)sv[u]
+                       : ((P.empty_keep && n == 0) ? P.mu[o] : __double2float_rn(sv[u] / (double)(n > 1 ? n : 1)));
         }
         if (P.init) P.sum[o] = 0.0;
         mus[k][j] = x;
@@ -630,8 +633,15 @@ struct CentroidTcParams {
     const __nv_bfloat16 *hi;  // [NH][Kp][64] centroids rounded to bf16
     float *part;              // [NH][n_chunks][K][kPartLd]
     int L, K, n_chunks;
+    int H, H_kv;              // query head h reads key/value head kv_head(h) of the [B H_kv] tensors
     float scale;
 };
+
+// Key/value head of query head h when H query heads share H_kv key/value
+// heads per batch row (H_kv divides H).
+__host__ __device__ __forceinline__ int kv_head(int64_t h, int H, int H_kv) {
+    return (int)((h / H) * H_kv + (h % H) / (H / H_kv));
+}
 
 template <int KP>
 __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_constant__ CUtensorMap tmk,
@@ -647,6 +657,7 @@ __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_
     const int L = P.L, K = P.K;
     const int chunk = blockIdx.x;
     const int64_t head = blockIdx.y;
+    const int kvh = kv_head(head, P.H, P.H_kv);
     const int c0 = chunk * kChunk;
     const int nsteps = min(2, (L - c0 + 255) / 256);
     const uint32_t sb = smem_u32(smem);
@@ -663,9 +674,9 @@ __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_
         umma::mbar_init(bar_o, 1);
         umma::mbar_init_fence();
         umma::mbar_expect_tx(bar_k, 256u * 128u);
-        umma::tma_load_3d(k_s, &tmk, 0, c0, (int)head, bar_k);
+        umma::tma_load_3d(k_s, &tmk, 0, c0, kvh, bar_k);
         umma::mbar_expect_tx(bar_v, 256u * 128u);
-        umma::tma_load_3d(v_s, &tmv, 0, c0, (int)head, bar_v);
+        umma::tma_load_3d(v_s, &tmv, 0, c0, kvh, bar_v);
     }
     // P starts as zeros (each row later writes only its own keys)
     for (int e = tid; e < 2 * 16384 / 16; e += 256)
@@ -776,7 +787,7 @@ __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_
             // K of the next step into the buffer the S product has finished reading
             if (s + 1 < nsteps) {
                 umma::mbar_expect_tx(bar_k, 256u * 128u);
-                umma::tma_load_3d(k_s, &tmk, 0, c0 + 256 * (s + 1), (int)head, bar_k);
+                umma::tma_load_3d(k_s, &tmk, 0, c0 + 256 * (s + 1), kvh, bar_k);
                 ++k_issued;
             }
             if (umma::mbar_wait(bar_v, par)) {
@@ -818,7 +829,7 @@ __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_
         if (tid == 0 && s + 1 < nsteps) {
             // V of the next step into the buffer the P V product has finished reading
             umma::mbar_expect_tx(bar_v, 256u * 128u);
-            umma::tma_load_3d(v_s, &tmv, 0, c0 + 256 * (s + 1), (int)head, bar_v);
+            umma::tma_load_3d(v_s, &tmv, 0, c0 + 256 * (s + 1), kvh, bar_v);
             ++v_issued;
         }
     }
@@ -913,11 +924,12 @@ struct WindowLayout {
 };
 
 struct WindowParams {
-    const __nv_bfloat16 *q, *k, *v;
+    const __nv_bfloat16 *q, *k, *v;  // k, v: [B H_kv][L][64]
     const float *vcent;     // [NH][K][64]
     const int32_t *assign;  // [NH][L]
     __nv_bfloat16 *out;
     int L, K, r;
+    int H, H_kv;            // query head h reads key/value head kv_head(h)
     float alpha, scale;
 };
 
@@ -929,8 +941,9 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
     const int64_t head = blockIdx.y;
     const int qb = blockIdx.x * kWinQ;
     const __nv_bfloat16 *qh = P.q + head * (int64_t)L * kD;
-    const __nv_bfloat16 *kh = P.k + head * (int64_t)L * kD;
-    const __nv_bfloat16 *vh = P.v + head * (int64_t)L * kD;
+    const int64_t kvh = kv_head(head, P.H, P.H_kv);
+    const __nv_bfloat16 *kh = P.k + kvh * (int64_t)L * kD;
+    const __nv_bfloat16 *vh = P.v + kvh * (int64_t)L * kD;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t kw_s = sbase + lay.k_off, vw_s = sbase + lay.v_off;
     float *vc = reinterpret_cast<float *>(smem + lay.vc_off);
@@ -1181,8 +1194,9 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
         umma::mbar_init_fence();
         umma::mbar_expect_tx(bar_ld, (uint32_t)(128 + 2 * NK) * 128u);
         umma::tma_load_3d(q_s, &tmq, 0, q0, (int)head, bar_ld);
-        umma::tma_load_3d(k_s, &tmk, 0, kb0, (int)head, bar_ld);
-        umma::tma_load_3d(v_s, &tmv, 0, kb0, (int)head, bar_ld);
+        const int kvh = kv_head(head, P.H, P.H_kv);
+        umma::tma_load_3d(k_s, &tmk, 0, kb0, kvh, bar_ld);
+        umma::tma_load_3d(v_s, &tmv, 0, kb0, kvh, bar_ld);
     }
     pdl_wait();  // V_cent and the assignments come from earlier kernels
     __syncwarp();

@@ -119,3 +119,23 @@ def test_default_options_take_the_fast_path():
     _lib.profile_start("fused_forward")
     _run("bf16", xq, xk, 16, 3, 32, 0.5)
     assert _lib.profile_stop().launches == 1
+
+
+@pytest.mark.parametrize("modes,H_kv,W", [
+    (dict(window_mode=1), 0, 60),                                # radius 60: tensor-core window
+    (dict(window_mode=1), 0, 100),                               # radius 100: mma.sync window
+    (dict(window_mode=1), 0, 5000),                              # W >= L: no local branch
+    (dict(empty_mode=1), 0, 40),
+    (dict(init_mode=1), 0, 40),
+    ({}, 2, 40),                                                 # grouped key/value heads
+    (dict(window_mode=1, empty_mode=1, init_mode=1), 2, 33),
+])
+def test_variants_on_the_tiled_kernels(modes, H_kv, W):
+    # bf16 variants without key masks or the soft gather run the tiled
+    # tensor-core kernels: several query tiles, key chunks and window blocks.
+    from means_cluster_attention_b200 import _lib
+    xq, xk = _case("bf16", 1, 4, 1500, 24, 3, W, 0.5, seed=71 + W, H_kv=H_kv or None,
+                   gmm=bool(modes.get("empty_mode")))
+    _lib.profile_start("tiled_assign")
+    _check("bf16", xq, xk, 24, 3, W, 0.5, H_kv=H_kv, **modes)
+    assert _lib.profile_stop().launches == 3, "the tiled path did not run"
