@@ -145,12 +145,17 @@ ca_status ensure_kernel_attributes() {
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_assign_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(centroid_attn_partial_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
@@ -257,6 +262,7 @@ bool tiled_eligible(int dtype, const Problem &p) {
 // empty clusters keeping their centroid, grouped key/value heads.
 struct TiledVariant {
     int r = 0, local = 1, init_stride = 0, empty_keep = 0, H_kv = 0;
+    const uint8_t *key_valid = nullptr;  // [B][L] key-padding mask (radius <= 64 or no local branch)
     static TiledVariant plain(const Problem &p) {
         TiledVariant tv;
         tv.r = p.W / 2;
@@ -278,12 +284,13 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     __nv_bfloat16 *hi = nullptr, *lo = nullptr;
     double *rsum = nullptr;
     int *rcnt = nullptr;
-    uint8_t *dead = nullptr;
+    uint8_t *dead = nullptr, *any_valid = nullptr;
     float *mstat = nullptr, *qnorm = nullptr;
     int32_t *assign = assign_out;
     CA_CUDA(s.get((void **)&mu, sizeof(float) * NH * Kp * kD));
     CA_CUDA(s.get((void **)&mstat, sizeof(float) * NH * 2));
     CA_CUDA(s.get((void **)&dead, sizeof(uint8_t) * NH * Kp));
+    if (tv.key_valid) CA_CUDA(s.get((void **)&any_valid, sizeof(uint8_t) * NH));
     CA_CUDA(s.get((void **)&qnorm, sizeof(float) * NH * L));
     CA_CUDA(s.get((void **)&hi, sizeof(__nv_bfloat16) * NH * Kp * kD));
     CA_CUDA(s.get((void **)&lo, sizeof(__nv_bfloat16) * NH * Kp * kD));
@@ -317,6 +324,9 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     up.init = 1;
     up.init_stride = tv.init_stride;
     up.empty_keep = tv.empty_keep;
+    up.key_valid = tv.key_valid;
+    up.any_valid = any_valid;
+    up.H = p.H;
     up.cent_out = p.iters == 0 ? cent_out : nullptr;
     {
         Launch pl("tiled_init", st, 0.0);
@@ -378,9 +388,13 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         cp.H = p.H;
         cp.H_kv = tv.H_kv;
         cp.scale = scale;
-        const tiled::CentroidTcLayout clay(Kp);
-        auto kern = Kp == 16 ? tiled::tiled_centroid_tc_kernel<16>
-                             : (Kp == 32 ? tiled::tiled_centroid_tc_kernel<32> : tiled::tiled_centroid_tc_kernel<64>);
+        cp.key_valid = tv.key_valid;
+        cp.any_valid = any_valid;
+        const tiled::CentroidTcLayout clay(Kp, tv.key_valid != nullptr);
+        const bool msk = tv.key_valid != nullptr;
+        auto kern = Kp == 16 ? (msk ? tiled::tiled_centroid_tc_kernel<16, true> : tiled::tiled_centroid_tc_kernel<16, false>)
+                    : Kp == 32 ? (msk ? tiled::tiled_centroid_tc_kernel<32, true> : tiled::tiled_centroid_tc_kernel<32, false>)
+                               : (msk ? tiled::tiled_centroid_tc_kernel<64, true> : tiled::tiled_centroid_tc_kernel<64, false>);
         Launch pl("tiled_centroid", st, 2.0 * head_bytes);
         CA_CUDA(launch_pdl(kern, dim3(n_chunks, (unsigned)NH), dim3(256), clay.total, st, kmap256, vmap256, cp));
         pl.after();
@@ -410,10 +424,11 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     wp.H = p.H;
     wp.H_kv = tv.H_kv;
     wp.scale = scale;
+    wp.key_valid = tv.key_valid;
     if (wp.r <= 64) {
         // tensor-core window kernel: the key window [q0 - RP, q0 + 127 + RP]
         const int RP = wp.r <= 32 ? 32 : 64;
-        const tiled::WindowTcLayout tlay(RP);
+        const tiled::WindowTcLayout tlay(RP, tv.key_valid != nullptr);
         CUtensorMap kmap, vmap, q128, o128;
         ca_status ms = encode_rows_map(&q128, q, NH, L, 128);
         if (ms == CA_OK) ms = encode_rows_map(&kmap, k, NH_kv, L, tlay.NK);
@@ -421,7 +436,10 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         if (ms == CA_OK) ms = encode_rows_map(&o128, out, NH, L, 128);
         if (ms != CA_OK) return ms;
         Launch pl("tiled_window", st, 4.0 * head_bytes);
-        CA_CUDA(launch_pdl(RP == 32 ? tiled::tiled_window_tc_kernel<32> : tiled::tiled_window_tc_kernel<64>,
+        const bool msk = tv.key_valid != nullptr;
+        auto wkern = RP == 32 ? (msk ? tiled::tiled_window_tc_kernel<32, true> : tiled::tiled_window_tc_kernel<32, false>)
+                              : (msk ? tiled::tiled_window_tc_kernel<64, true> : tiled::tiled_window_tc_kernel<64, false>);
+        CA_CUDA(launch_pdl(wkern,
                            dim3((L + 127) / 128, (unsigned)NH), dim3(256), tlay.total, st, q128, kmap, vmap, o128, wp));
         pl.after();
     } else {
@@ -621,11 +639,13 @@ ca_status ca_forward_ex(const void *q, const void *k, const void *v, int dtype, 
     s = ensure_kernel_attributes();
     if (s != CA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
-    // bf16 with grouped key/value heads, the radius window, the stride init or
-    // kept empty centroids: the tiled kernels (key masks and the soft gather
-    // stay on the general path)
-    if (dtype == 1 && !o.key_valid && !o.gather_mode && K <= 64 && (!ex.var.local || ex.r <= ca::tiled::kMaxR)) {
+    // bf16 with grouped key/value heads, the radius window, the stride init,
+    // kept empty centroids or key masks (window radius <= 64 then): the tiled
+    // kernels (the soft gather stays on the general path)
+    const int r_max = o.key_valid ? 64 : ca::tiled::kMaxR;  // masks: the tensor-core window kernel only
+    if (dtype == 1 && !o.gather_mode && K <= 64 && (!ex.var.local || ex.r <= r_max)) {
         TiledVariant tv;
+        tv.key_valid = o.key_valid;
         tv.r = ex.r;
         tv.local = ex.var.local;
         tv.init_stride = ex.init_stride;

@@ -80,6 +80,9 @@ struct UpdateParams {
     int L, K, Kp, init;
     int init_stride;         // 1: mu_k = Q[k max(1, L / K)] (the module's stride) instead of Q[floor(k L / K)]
     int empty_keep;          // 1: an empty cluster keeps its previous centroid instead of becoming zero
+    const uint8_t *key_valid;  // [B][L] key-padding mask or null
+    uint8_t *any_valid;        // [NH] written in init mode: 1 when the head has a valid key
+    int H;                     // query heads per batch row
 };
 
 // grid (NH), 1024 threads.  mu_k = Q[floor(k L / K)] (init; the running sums
@@ -128,8 +131,12 @@ __global__ void __launch_bounds__(kUpdThreads) tiled_update_kernel(UpdateParams 
         float x = 0.f;
         if (k < K) {
             const int n = ns[k];
-            x = P.init ? (float)sv[u]
-                       : ((P.empty_keep && n == 0) ? P.mu[o] : __double2float_rn(sv[u] / (double)(n > 1 ? n : 1)));
+            if (P.init)
+                x = (float)sv[u];
+            else if (n == 0 && P.empty_keep)  // the previous centroid is read only in this mode
+                x = P.mu[o];
+            else
+                x = __double2float_rn(sv[u] / (double)(n > 1 ? n : 1));
         }
         if (P.init) P.sum[o] = 0.0;
         mus[k][j] = x;
@@ -140,6 +147,13 @@ __global__ void __launch_bounds__(kUpdThreads) tiled_update_kernel(UpdateParams 
         if (P.cent_out && k < K) P.cent_out[(head * K + k) * kD + j] = x;
     }
     if (P.init && tid < Kp) P.cnt[hb + tid] = 0;
+    if (P.init && P.key_valid) {
+        const uint8_t *kv = P.key_valid + (head / P.H) * P.L;
+        int mine = 0;
+        for (int jj = tid; jj < P.L; jj += kUpdThreads) mine |= kv[jj];
+        mine = __syncthreads_or(mine);
+        if (tid == 0) P.any_valid[head] = mine ? 1 : 0;
+    }
     __syncthreads();
     for (int k = warp; k < Kp; k += kUw) {
         const float x0 = mus[k][2 * lane], x1 = mus[k][2 * lane + 1];
@@ -610,8 +624,8 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
 // groups) are merged at the end.  K / V of the next step are loaded by TMA
 // while this one computes.
 struct CentroidTcLayout {
-    uint32_t z_off, k_off, v_off, p_off, red_off, bar_off, total;
-    __host__ __device__ CentroidTcLayout(int Kp) {
+    uint32_t z_off, k_off, v_off, p_off, red_off, km_off, bar_off, total;
+    __host__ __device__ CentroidTcLayout(int Kp, bool mask) {
         uint32_t o = 0;
         z_off = o;  // (128 - Kp) rows of 128 bytes: zeros, the centroids at rows [64 - Kp, 64), zeros
         o += up((uint32_t)(128 - Kp) * 128u, 1024);
@@ -623,6 +637,8 @@ struct CentroidTcLayout {
         o += 2u * 16384u;
         red_off = o;  // [2][128] half-row maxima, then [2][128] half-row sums
         o += 2u * 2u * 128u * 4u;
+        km_off = o;  // key mask of the chunk (masked calls)
+        o += mask ? 512u : 0u;
         bar_off = o;  // four mbarriers, the tensor-memory address
         o += 48;
         total = up(o, 128) + 1024;  // + slack to align the base to 1024 bytes
@@ -635,15 +651,19 @@ struct CentroidTcParams {
     int L, K, n_chunks;
     int H, H_kv;              // query head h reads key/value head kv_head(h) of the [B H_kv] tensors
     float scale;
+    const uint8_t *key_valid;  // [B][L] key-padding mask or null: invalid keys take no weight
+    const uint8_t *any_valid;  // [NH]: 0 when the head has no valid key (every key then weighs the same)
 };
 
 // Key/value head of query head h when H query heads share H_kv key/value
 // heads per batch row (H_kv divides H).
 __host__ __device__ __forceinline__ int kv_head(int64_t h, int H, int H_kv) {
-    return (int)((h / H) * H_kv + (h % H) / (H / H_kv));
+    if (H_kv == H) return (int)h;  // no grouping (B H < 2^16)
+    const int hh = (int)h;
+    return (hh / H) * H_kv + (hh % H) / (H / H_kv);
 }
 
-template <int KP>
+template <int KP, bool MASK>
 __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                      const __grid_constant__ CUtensorMap tmv,
                                                                      CentroidTcParams P) {
@@ -652,7 +672,7 @@ __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_
     constexpr uint32_t kOCol = 128; // O columns [128, 192)
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const CentroidTcLayout lay(KP);
+    const CentroidTcLayout lay(KP, MASK);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q = warp & 3, wg = warp >> 2;
     const int L = P.L, K = P.K;
     const int chunk = blockIdx.x;
@@ -677,6 +697,11 @@ __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_
         umma::tma_load_3d(k_s, &tmk, 0, c0, kvh, bar_k);
         umma::mbar_expect_tx(bar_v, 256u * 128u);
         umma::tma_load_3d(v_s, &tmv, 0, c0, kvh, bar_v);
+    }
+    uint8_t *kmask = smem + lay.km_off;
+    if constexpr (MASK) {
+        const uint8_t *kv = P.key_valid + (head / P.H) * L;
+        for (int c = tid; c < kChunk; c += 256) kmask[c] = c0 + c < L ? kv[c0 + c] : 0;
     }
     // P starts as zeros (each row later writes only its own keys)
     for (int e = tid; e < 2 * 16384 / 16; e += 256)
@@ -745,6 +770,14 @@ __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_
 #pragma unroll
         for (int t = 0; t < KP; ++t) asm volatile("" : "+f"(v[t]));
         const int key0 = c0 + 256 * s + blk * N + wg * KP;  // key of v[0]
+        if constexpr (MASK) {
+            // an invalid key takes no weight; a head without a valid key
+            // weighs every key the same
+            const bool any = P.any_valid[head] != 0;
+#pragma unroll
+            for (int t = 0; t < KP; ++t)
+                if (key0 + t < L) v[t] = any ? (kmask[key0 + t - c0] ? v[t] : -INFINITY) : 0.f;
+        }
         if (c0 + 256 * (s + 1) > L) {  // keys past L (zero rows of the load) do not exist
 #pragma unroll
             for (int t = 0; t < KP; ++t)
@@ -931,6 +964,7 @@ struct WindowParams {
     int L, K, r;
     int H, H_kv;            // query head h reads key/value head kv_head(h)
     float alpha, scale;
+    const uint8_t *key_valid;  // [B][L] key-padding mask or null (tensor-core kernel only)
 };
 
 __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams P) {
@@ -1152,19 +1186,20 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
 //                       rounded once to bf16, one 128-byte row per thread.
 struct WindowTcLayout {
     int NK;
-    uint32_t qk_off, v_off, red_off, bar_off, total;
-    __host__ __device__ WindowTcLayout(int RP) {
+    uint32_t qk_off, v_off, red_off, km_off, bar_off, total;
+    __host__ __device__ WindowTcLayout(int RP, bool mask) {
         NK = 128 + 2 * RP;
         qk_off = 0;  // Q (16 KB) then K (NK rows); afterwards P (NK / 64 blocks of 16 KB)
         const uint32_t qk = 16384u + (uint32_t)NK * 128u, pb = (uint32_t)NK / 64u * 16384u;
         v_off = up(qk > pb ? qk : pb, 1024);
         red_off = v_off + (uint32_t)NK * 128u;  // [4][128] floats: partial row maxima and sums
-        bar_off = red_off + 4u * 128u * 4u;
+        km_off = red_off + 4u * 128u * 4u;      // key mask of the window, then [2][128] row flags (masked calls)
+        bar_off = km_off + (mask ? up((uint32_t)NK + 256u, 16) : 0u);
         total = up(bar_off + 32u, 128) + 1024;  // + slack to align the base to 1024 bytes
     }
 };
 
-template <int RP>
+template <int RP, bool MASK>
 __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                                                                   const __grid_constant__ CUtensorMap tmk,
                                                                   const __grid_constant__ CUtensorMap tmv,
@@ -1174,7 +1209,7 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
     constexpr int NC = RP / 16 + 1;    // 32-column chunks of one warp quarter's window
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const WindowTcLayout lay(RP);
+    const WindowTcLayout lay(RP, MASK);
     const int tid = threadIdx.x, warp = tid >> 5, wg = warp >> 2, q4 = warp & 3;
     const int L = P.L, K = P.K, r = P.r;
     const int64_t head = blockIdx.y;
@@ -1197,6 +1232,11 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
         const int kvh = kv_head(head, P.H, P.H_kv);
         umma::tma_load_3d(k_s, &tmk, 0, kb0, kvh, bar_ld);
         umma::tma_load_3d(v_s, &tmv, 0, kb0, kvh, bar_ld);
+    }
+    uint8_t *kmask = smem + lay.km_off, *rowflag = kmask + NK;
+    if constexpr (MASK) {  // the window's key mask (an input: before the wait)
+        const uint8_t *kv = P.key_valid + (head / P.H) * L;
+        for (int c = tid; c < NK; c += 256) kmask[c] = (kb0 + c >= 0 && kb0 + c < L) ? kv[kb0 + c] : 0;
     }
     pdl_wait();  // V_cent and the assignments come from earlier kernels
     __syncwarp();
@@ -1266,6 +1306,25 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
                     if ((unsigned)(cb + t - lo) > (unsigned)(hi - lo)) v[16 * pc + t] = -INFINITY;
             }
         }
+        if constexpr (MASK) {
+            // Invalid keys take no weight; a row whose window holds no valid
+            // key weighs its window's keys the same (scores 0).
+            int mine = 0;
+#pragma unroll
+            for (int t = 0; t < HALF; ++t) mine |= (v[t] != -INFINITY && kmask[cb0 + t]) ? 1 : 0;
+            rowflag[wg * 128 + i] = (uint8_t)mine;
+        }
+    }
+    if constexpr (MASK) {
+        __syncthreads();
+        const bool any = (rowflag[i] | rowflag[128 + i]) != 0;
+        if (s_ok) {
+#pragma unroll
+            for (int t = 0; t < HALF; ++t)
+                if (v[t] != -INFINITY) v[t] = any ? (kmask[cb0 + t] ? v[t] : -INFINITY) : 0.f;
+        }
+    }
+    if (s_ok) {
 #pragma unroll
         for (int t = 0; t < HALF; ++t) m = fmaxf(m, v[t]);
     }
@@ -1334,6 +1393,10 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
         for (int u = 0; u < 8; ++u) {
             w[2 * u] = pack_bf16(fmaf(f, o[4 * u + 0], be * g[u].x), fmaf(f, o[4 * u + 1], be * g[u].y));
             w[2 * u + 1] = pack_bf16(fmaf(f, o[4 * u + 2], be * g[u].z), fmaf(f, o[4 * u + 3], be * g[u].w));
+        }
+        if (MASK && qi < L && !P.key_valid[(head / P.H) * L + qi]) {  // an invalid query's row is zero
+#pragma unroll
+            for (int u = 0; u < 16; ++u) w[u] = 0u;
         }
         // the output tile, 128-byte swizzled over the dead P block 0, then
         // one TMA store (rows past L are clipped)

@@ -139,3 +139,21 @@ def test_variants_on_the_tiled_kernels(modes, H_kv, W):
     _lib.profile_start("tiled_assign")
     _check("bf16", xq, xk, 24, 3, W, 0.5, H_kv=H_kv, **modes)
     assert _lib.profile_stop().launches == 3, "the tiled path did not run"
+
+
+@pytest.mark.parametrize("W,modes", [(40, {}), (128, {}), (30, dict(window_mode=1)), (5000, dict(window_mode=1))])
+def test_key_padding_mask_on_the_tiled_kernels(W, modes):
+    # Several key chunks and window blocks per head: right, left and scattered
+    # padding, and one batch row with no valid key at all (every key then
+    # weighs the same in both softmaxes, and every output row is zero).
+    from means_cluster_attention_b200 import _lib
+    B, L = 4, 1500
+    xq, xk = _case("bf16", B, 2, L, 20, 3, W, 0.5, seed=91 + W)
+    valid = np.ones((B, L), dtype=bool)
+    valid[0, 1100:] = False
+    valid[1, :613] = False
+    valid[2, ::3] = False
+    valid[3, :] = False
+    _lib.profile_start("tiled_assign")
+    _check("bf16", xq, xk, 20, 3, W, 0.5, key_valid=valid, **modes)
+    assert _lib.profile_stop().launches == 3, "the tiled path did not run"
