@@ -138,11 +138,12 @@ typedef struct {
 
 /* ca_forward_trace with the variants of ca_options (opt may be NULL).  Calls
  * whose options are all defaults take the same kernels as ca_forward_trace.
- * bf16 calls with K <= 64 that do not use the soft gather (grouped key/value
- * heads, the radius window with radius <= 128 or no local branch, the stride
- * init, kept empty centroids, key_valid with a window radius <= 64 or no
- * local branch, alone or together) run the tiled tensor-core kernels; every
- * other option runs the general multi-kernel path. */
+ * bf16 calls with K <= 64 (grouped key/value heads, the radius window with
+ * radius <= 128 or no local branch, the stride init, kept empty centroids,
+ * key_valid with a window radius <= 64, the soft gather with a window radius
+ * <= 32, or no local branch with either; alone or together) run the tiled
+ * tensor-core kernels; every other option runs the general multi-kernel
+ * path. */
 ca_status ca_forward_ex(const void *q, const void *k, const void *v, int dtype, int B, int H,
                         int L, int d, int K, int iters, int W, float alpha, const ca_options *opt,
                         void *out, int32_t *assign_out, float *centroids_out, int32_t *assign_hist,

@@ -152,10 +152,12 @@ ca_status ensure_kernel_attributes() {
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_centroid_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<32, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<64, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<32, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<64, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<32, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    CA_CUDA(cudaFuncSetAttribute(tiled::tiled_window_tc_kernel<32, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(kmeans_assign_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(centroid_attn_partial_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
@@ -263,6 +265,7 @@ bool tiled_eligible(int dtype, const Problem &p) {
 struct TiledVariant {
     int r = 0, local = 1, init_stride = 0, empty_keep = 0, H_kv = 0;
     const uint8_t *key_valid = nullptr;  // [B][L] key-padding mask (radius <= 64 or no local branch)
+    int soft = 0;                        // soft gather (radius <= 32 or no local branch)
     static TiledVariant plain(const Problem &p) {
         TiledVariant tv;
         tv.r = p.W / 2;
@@ -425,10 +428,12 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     wp.H_kv = tv.H_kv;
     wp.scale = scale;
     wp.key_valid = tv.key_valid;
+    wp.hi = hi;
+    wp.Kp = Kp;
     if (wp.r <= 64) {
         // tensor-core window kernel: the key window [q0 - RP, q0 + 127 + RP]
         const int RP = wp.r <= 32 ? 32 : 64;
-        const tiled::WindowTcLayout tlay(RP, tv.key_valid != nullptr);
+        const tiled::WindowTcLayout tlay(RP, tv.key_valid != nullptr, tv.soft != 0);
         CUtensorMap kmap, vmap, q128, o128;
         ca_status ms = encode_rows_map(&q128, q, NH, L, 128);
         if (ms == CA_OK) ms = encode_rows_map(&kmap, k, NH_kv, L, tlay.NK);
@@ -437,8 +442,9 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         if (ms != CA_OK) return ms;
         Launch pl("tiled_window", st, 4.0 * head_bytes);
         const bool msk = tv.key_valid != nullptr;
-        auto wkern = RP == 32 ? (msk ? tiled::tiled_window_tc_kernel<32, true> : tiled::tiled_window_tc_kernel<32, false>)
-                              : (msk ? tiled::tiled_window_tc_kernel<64, true> : tiled::tiled_window_tc_kernel<64, false>);
+        auto wkern = tv.soft ? (msk ? tiled::tiled_window_tc_kernel<32, true, true> : tiled::tiled_window_tc_kernel<32, false, true>)
+                     : RP == 32 ? (msk ? tiled::tiled_window_tc_kernel<32, true, false> : tiled::tiled_window_tc_kernel<32, false, false>)
+                                : (msk ? tiled::tiled_window_tc_kernel<64, true, false> : tiled::tiled_window_tc_kernel<64, false, false>);
         CA_CUDA(launch_pdl(wkern,
                            dim3((L + 127) / 128, (unsigned)NH), dim3(256), tlay.total, st, q128, kmap, vmap, o128, wp));
         pl.after();
@@ -640,12 +646,14 @@ ca_status ca_forward_ex(const void *q, const void *k, const void *v, int dtype, 
     if (s != CA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
     // bf16 with grouped key/value heads, the radius window, the stride init,
-    // kept empty centroids or key masks (window radius <= 64 then): the tiled
-    // kernels (the soft gather stays on the general path)
-    const int r_max = o.key_valid ? 64 : ca::tiled::kMaxR;  // masks: the tensor-core window kernel only
-    if (dtype == 1 && !o.gather_mode && K <= 64 && (!ex.var.local || ex.r <= r_max)) {
+    // kept empty centroids, key masks (window radius <= 64 then) or the soft
+    // gather (radius <= 32): the tiled kernels
+    // masks: the tensor-core window kernel; the soft gather: its radius-32 form
+    const int r_max = o.gather_mode ? 32 : (o.key_valid ? 64 : ca::tiled::kMaxR);
+    if (dtype == 1 && K <= 64 && (!ex.var.local || ex.r <= r_max)) {
         TiledVariant tv;
         tv.key_valid = o.key_valid;
+        tv.soft = o.gather_mode;
         tv.r = ex.r;
         tv.local = ex.var.local;
         tv.init_stride = ex.init_stride;

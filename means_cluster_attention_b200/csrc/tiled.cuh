@@ -965,6 +965,8 @@ struct WindowParams {
     int H, H_kv;            // query head h reads key/value head kv_head(h)
     float alpha, scale;
     const uint8_t *key_valid;  // [B][L] key-padding mask or null (tensor-core kernel only)
+    const __nv_bfloat16 *hi;   // [NH][Kp][64] final centroids rounded to bf16 (soft gather)
+    int Kp;
 };
 
 __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams P) {
@@ -1186,20 +1188,31 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_window_kernel(WindowParams 
 //                       rounded once to bf16, one 128-byte row per thread.
 struct WindowTcLayout {
     int NK;
-    uint32_t qk_off, v_off, red_off, km_off, bar_off, total;
-    __host__ __device__ WindowTcLayout(int RP, bool mask) {
+    uint32_t qk_off, v_off, red_off, km_off, mu_off, vc_off, p2_off, red2_off, bar_off, total;
+    __host__ __device__ WindowTcLayout(int RP, bool mask, bool soft) {
         NK = 128 + 2 * RP;
         qk_off = 0;  // Q (16 KB) then K (NK rows); afterwards P (NK / 64 blocks of 16 KB)
         const uint32_t qk = 16384u + (uint32_t)NK * 128u, pb = (uint32_t)NK / 64u * 16384u;
         v_off = up(qk > pb ? qk : pb, 1024);
         red_off = v_off + (uint32_t)NK * 128u;  // [4][128] floats: partial row maxima and sums
         km_off = red_off + 4u * 128u * 4u;      // key mask of the window, then [2][128] row flags (masked calls)
-        bar_off = km_off + (mask ? up((uint32_t)NK + 256u, 16) : 0u);
+        uint32_t o = km_off + (mask ? up((uint32_t)NK + 256u, 16) : 0u);
+        // soft gather: the centroids (B of S2 = Q mu^T), V_cent in bf16 (B of
+        // G = P2 V_cent, N-major), the weights P2, and their row maxima / sums
+        mu_off = vc_off = p2_off = red2_off = o;
+        if (soft) {
+            mu_off = up(o, 1024);
+            vc_off = mu_off + 64u * 128u;
+            p2_off = vc_off + 64u * 128u;
+            red2_off = p2_off + 128u * 128u;
+            o = red2_off + 4u * 128u * 4u;
+        }
+        bar_off = o;
         total = up(bar_off + 32u, 128) + 1024;  // + slack to align the base to 1024 bytes
     }
 };
 
-template <int RP, bool MASK>
+template <int RP, bool MASK, bool SOFT>
 __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                                                                   const __grid_constant__ CUtensorMap tmk,
                                                                   const __grid_constant__ CUtensorMap tmv,
@@ -1207,9 +1220,12 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
                                                                   WindowParams P) {
     constexpr int NK = 128 + 2 * RP;
     constexpr int NC = RP / 16 + 1;    // 32-column chunks of one warp quarter's window
+    // soft gather: S2 = Q mu^T in tensor-memory columns [NK, NK + 64), which
+    // exist only for the radius-32 window
+    static_assert(!SOFT || NK + 64 <= 256, "the soft gather needs the radius-32 window");
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const WindowTcLayout lay(RP, MASK);
+    const WindowTcLayout lay(RP, MASK, SOFT);
     const int tid = threadIdx.x, warp = tid >> 5, wg = warp >> 2, q4 = warp & 3;
     const int L = P.L, K = P.K, r = P.r;
     const int64_t head = blockIdx.y;
@@ -1245,7 +1261,24 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
     // reads its share of the row's score columns and writes half of its
     // output row.
     const int i = 32 * q4 + (tid & 31), qi = q0 + i;
-    const int ci = qi < L ? CA_IDX(P.assign[head * L + qi], 0, K, 67) : 0;
+    const int ci = (qi < L && !SOFT) ? CA_IDX(P.assign[head * L + qi], 0, K, 67) : 0;
+    if constexpr (SOFT) {
+        // centroids (rows >= K zero) and V_cent rounded to bf16, as 128-byte
+        // swizzled rows for the two soft-gather products
+        for (int e = tid; e < 64 * 8; e += 256) {
+            const int kk = e >> 3, ch = e & 7;
+            uint4 wm = make_uint4(0u, 0u, 0u, 0u), wv = wm;
+            if (kk < K) {
+                wm = *reinterpret_cast<const uint4 *>(P.hi + (head * P.Kp + kk) * kD + ch * 8);
+                const float4 *src = reinterpret_cast<const float4 *>(P.vcent + (head * K + kk) * kD + ch * 8);
+                const float4 a = src[0], b = src[1];
+                wv = make_uint4(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w), pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
+            }
+            *reinterpret_cast<uint4 *>(smem + lay.mu_off + swz(kk, ch)) = wm;
+            *reinterpret_cast<uint4 *>(smem + lay.vc_off + swz(kk, ch)) = wv;
+        }
+        umma::fence_proxy_async_smem();
+    }
     const float4 *vrow = reinterpret_cast<const float4 *>(P.vcent + (head * K + ci) * kD) + 8 * wg;
     umma::tc_fence_before();
     __syncthreads();
@@ -1260,6 +1293,13 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
             for (int ks = 0; ks < 4; ++ks)
                 umma::mma_bf16(taddr, umma::desc_sw128(q_s + (uint32_t)ks * 32u), umma::desc_sw128(k_s + (uint32_t)ks * 32u),
                                idesc, ks > 0);
+            if constexpr (SOFT) {
+                constexpr uint32_t idesc2 = umma::idesc_bf16_f32(128, 64);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma::mma_bf16(taddr + (uint32_t)NK, umma::desc_sw128(q_s + (uint32_t)ks * 32u),
+                                   umma::desc_sw128(sb + lay.mu_off + (uint32_t)ks * 32u), idesc2, ks > 0);
+            }
             umma::mma_commit(bar_s);
         } else {
             record_error(4, 40);
@@ -1328,6 +1368,21 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
 #pragma unroll
         for (int t = 0; t < HALF; ++t) m = fmaxf(m, v[t]);
     }
+    float *red2 = reinterpret_cast<float *>(smem + lay.red2_off);  // soft gather: [2][128] maxima, then sums
+    if constexpr (SOFT) {
+        // this thread's 32 centroid scores of the row (centroids 32 wg ..)
+        float m2 = -INFINITY;
+        if (s_ok) {
+            float s2[32];
+            umma::tmem_ld32(trow + (uint32_t)(NK + 32 * wg), s2);
+            umma::tmem_ld_wait();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) asm volatile("" : "+f"(s2[t]));
+#pragma unroll
+            for (int t = 0; t < 32; ++t) m2 = fmaxf(m2, 32 * wg + t < K ? s2[t] : -INFINITY);
+        }
+        red2[wg * 128 + i] = m2;
+    }
     red[wg * 128 + i] = m;
     __syncthreads();
     m = fmaxf(red[i], red[128 + i]);
@@ -1360,6 +1415,32 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
                              : "memory");
         }
     }
+    if constexpr (SOFT) {
+        const float m2 = fmaxf(red2[i], red2[128 + i]), mc2 = m2 * csc;
+        float l2 = 0.f;
+        if (s_ok) {
+            float s2[32];
+            umma::tmem_ld32(trow + (uint32_t)(NK + 32 * wg), s2);
+            umma::tmem_ld_wait();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) asm volatile("" : "+f"(s2[t]));
+            uint32_t pk[16];
+#pragma unroll
+            for (int t = 0; t < 32; t += 2) {
+                const float p0 = 32 * wg + t < K ? fused::ex2(fmaf(s2[t], csc, -mc2)) : 0.f;
+                const float p1 = 32 * wg + t + 1 < K ? fused::ex2(fmaf(s2[t + 1], csc, -mc2)) : 0.f;
+                l2 += p0 + p1;
+                pk[t >> 1] = pack_bf16(p0, p1);
+            }
+            const uint32_t p2_s = sb + lay.p2_off;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"r"(p2_s + swz(i, 4 * wg + q)), "r"(pk[4 * q]),
+                             "r"(pk[4 * q + 1]), "r"(pk[4 * q + 2]), "r"(pk[4 * q + 3])
+                             : "memory");
+        }
+        red2[256 + wg * 128 + i] = l2;
+    }
     red[256 + wg * 128 + i] = l;
     umma::fence_proxy_async_smem();
     umma::tc_fence_before();
@@ -1371,20 +1452,40 @@ __global__ void __launch_bounds__(256, 2) tiled_window_tc_kernel(const __grid_co
         for (int ks = 0; ks < NK / 16; ++ks)
             umma::mma_bf16(taddr, umma::desc_sw128(p_s + (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u),
                            umma::desc_sw128(v_s + (uint32_t)ks * 2048u), idesc, ks > 0);
+        if constexpr (SOFT) {
+            // G = P2 V_cent into columns [64, 128) (their scores were read)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                umma::mma_bf16(taddr + 64u, umma::desc_sw128(sb + lay.p2_off + (uint32_t)ks * 32u),
+                               umma::desc_sw128(sb + lay.vc_off + (uint32_t)ks * 2048u), idesc, ks > 0);
+        }
         umma::mma_commit(bar_o);
     }
     // this thread's half of the token's V_cent row
     float4 g[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) g[u] = __ldg(vrow + u);
+    for (int u = 0; u < 8; ++u) g[u] = SOFT ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(vrow + u);
     l = red[256 + i] + red[384 + i];
     const bool o_ok = __syncthreads_and(s_ok && umma::mbar_wait(bar_o, 0));
     if (!o_ok && s_ok && tid == 0) record_error(4, 42);
     umma::tc_fence_after();
     if (o_ok) {
-        const float be = 1.f - P.alpha, f = l > 0.f ? P.alpha / l : 0.f;
+        float be = 1.f - P.alpha;
+        const float f = l > 0.f ? P.alpha / l : 0.f;
         float o[32];
         umma::tmem_ld32(trow + (uint32_t)(32 * wg), o);
+        if constexpr (SOFT) {
+            // the soft gather G / l2 takes the place of V_cent[c_i]
+            float gs[32];
+            umma::tmem_ld32(trow + (uint32_t)(64 + 32 * wg), gs);
+            umma::tmem_ld_wait();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) asm volatile("" : "+f"(gs[t]));
+#pragma unroll
+            for (int u = 0; u < 8; ++u) g[u] = make_float4(gs[4 * u], gs[4 * u + 1], gs[4 * u + 2], gs[4 * u + 3]);
+            const float l2 = red2[256 + i] + red2[384 + i];
+            be = l2 > 0.f ? be / l2 : 0.f;
+        }
         umma::tmem_ld_wait();
 #pragma unroll
         for (int t = 0; t < 32; ++t) asm volatile("" : "+f"(o[t]));

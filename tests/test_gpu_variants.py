@@ -157,3 +157,21 @@ def test_key_padding_mask_on_the_tiled_kernels(W, modes):
     _lib.profile_start("tiled_assign")
     _check("bf16", xq, xk, 20, 3, W, 0.5, key_valid=valid, **modes)
     assert _lib.profile_stop().launches == 3, "the tiled path did not run"
+
+
+@pytest.mark.parametrize("K,W,modes,masked", [(64, 64, {}, False), (9, 40, {}, True), (33, 5000, dict(window_mode=1), False),
+                                              (20, 30, dict(window_mode=1), True)])
+def test_soft_gather_on_the_tiled_kernels(K, W, modes, masked):
+    # The soft gather softmax(Q_i mu^T / sqrt(d)) V_cent inside the tensor-core
+    # window kernel (radius <= 32 or no local branch), with and without masks.
+    from means_cluster_attention_b200 import _lib
+    B, L = 2, 1500
+    xq, xk = _case("bf16", B, 3, L, K, 3, W, 0.4, seed=7 * K + W)
+    valid = None
+    if masked:
+        valid = np.ones((B, L), dtype=bool)
+        valid[0, 900:] = False
+        valid[1, ::4] = False
+    _lib.profile_start("tiled_assign")
+    _check("bf16", xq, xk, K, 3, W, 0.4, key_valid=valid, gather_mode=1, **modes)
+    assert _lib.profile_stop().launches == 3, "the tiled path did not run"
