@@ -373,6 +373,53 @@ def parity_check(w, x, dev_inputs, n_heads):
             "tolerance": 2e-3 if w.dtype == "f32" else 2e-2, "oracle_seconds": round(dt, 2)}
 
 
+def time_variants(args, w, dev_inputs, flush):
+    """Step times of the module's variants (ca_forward_ex) on workload w, on
+    the same device inputs: grouped key/value heads (H_kv = H / 4), the
+    module's radius window (radius = W), key padding (the last 10% of every
+    batch row invalid), the soft gather, and all of them together.  Each is
+    timed like the headline (L2 flushed before every step, CUDA events around
+    the forward), after its own warm-up; correctness of every variant is
+    covered by the GPU tests against the oracle."""
+    import torch
+    import means_cluster_attention_b200 as ca
+    q, k, v = dev_inputs
+    B, H, L, d = q.shape
+    hkv = max(1, H // 4)
+    kg, vg = k[:, :hkv].contiguous(), v[:, :hkv].contiguous()
+    valid = torch.ones((B, L), dtype=torch.uint8, device=q.device)
+    valid[:, L - L // 10:] = 0
+    cases = {
+        "gqa_hkv_h_over_4": (q, kg, vg, w.W, {}),
+        "radius_window_W": (q, k, v, w.W // 2, dict(window_mode=1)),
+        "key_padding_10pct": (q, k, v, w.W, dict(key_valid=valid)),
+        "soft_gather": (q, k, v, w.W, dict(gather_mode=1)),
+        "all_together": (q, kg, vg, w.W // 2, dict(window_mode=1, key_valid=valid, gather_mode=1)),
+    }
+    out = {}
+    for name, (qq, kk, vv, W, opts) in cases.items():
+        def step():
+            ca.forward_ex(qq, kk, vv, w.K, w.iters, W, w.alpha, **opts)
+        for _ in range(args.warmup):
+            step()
+            flush.zero_()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s_ev.record()
+            step()
+            e_ev.record()
+            ms.append((s_ev, e_ev))
+        torch.cuda.synchronize()
+        t = sum(a.elapsed_time(b) for a, b in ms) / len(ms)
+        out[name] = {"ms_per_step": t, "value": w.tokens / (t / 1e3), "unit": UNIT,
+                     "window_arg_W": W, "options": sorted(opts)}
+    ca.sync_status()
+    return {"workload": w.name, **out}
+
+
 def run_ours(args, w):
     import torch
     import means_cluster_attention_b200 as ca
@@ -435,6 +482,9 @@ def run_ours(args, w):
     }
     if others:
         line["other_workloads"] = others
+    if not args.no_variants and "l4k_gmm_bf16" in extra_inputs:
+        ow, _, odev = extra_inputs["l4k_gmm_bf16"]
+        line["variants"] = time_variants(args, ow, odev, flush)
     if pg:
         line["config"]["parallelism"] = f"replicas x{ws} (independent heads, no collective)"
     if rank == 0 and ws == 1 and not args.no_parity:
@@ -466,6 +516,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-parity", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the step times of the module's variants (on l4k_gmm_bf16)")
     ap.add_argument("--also", default=DEFAULT_ALSO,
                     help="comma-separated workloads timed beside the headline ('' for none)")
     args = ap.parse_args()
