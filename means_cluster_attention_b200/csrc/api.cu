@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>
@@ -131,6 +132,8 @@ struct Scratch {
 // Every kernel that takes dynamic shared memory may use up to 227 KB of it.
 // The attribute is per device and per function; it is set once per device,
 // under a lock, before the first launch there.
+static std::atomic<int> g_sm_count[64];  // multiprocessors of each device (set with the attributes)
+
 ca_status ensure_kernel_attributes() {
     using namespace ca;
     static std::mutex mu;
@@ -164,8 +167,19 @@ ca_status ensure_kernel_attributes() {
     CA_CUDA(cudaFuncSetAttribute(centroid_attn_partial_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(window_blend_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
     CA_CUDA(cudaFuncSetAttribute(window_blend_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+    int n_sm = 0;
+    CA_CUDA(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+    g_sm_count[dev].store(n_sm);
     done[dev] = true;
     return CA_OK;
+}
+
+// Multiprocessors of the current device (ensure_kernel_attributes ran).
+int sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    const int n = g_sm_count[dev].load();
+    return n > 0 ? n : 148;
 }
 
 // The fused one-CTA-per-head kernel handles bf16 heads with L <= 512,
@@ -280,7 +294,12 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
     using namespace ca;
     const int64_t NH = p.heads(), NH_kv = (int64_t)p.B * tv.H_kv;
     const int L = p.L, K = p.K, Kp = tiled::kpad(K);
-    const int n_chunks = (L + tiled::kChunk - 1) / tiled::kChunk;
+    // Keys per centroid-attention CTA: long chunks (fewer partial states to
+    // combine, each CTA's set-up spread over more steps) as long as the grid
+    // still gives every multiprocessor a CTA.
+    int chunk_keys = tiled::kMaxChunk;
+    while (chunk_keys > 512 && NH * ((L + chunk_keys - 1) / chunk_keys) < sm_count()) chunk_keys /= 2;
+    const int n_chunks = (L + chunk_keys - 1) / chunk_keys;
     const float scale = 1.0f / sqrtf((float)p.d);
     Scratch s(st);
     float *mu = nullptr, *mm = nullptr, *cpart = nullptr, *vcent = nullptr;
@@ -388,6 +407,7 @@ ca_status run_tiled(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_b
         cp.L = L;
         cp.K = K;
         cp.n_chunks = n_chunks;
+        cp.chunk_keys = chunk_keys;
         cp.H = p.H;
         cp.H_kv = tv.H_kv;
         cp.scale = scale;

@@ -58,7 +58,7 @@ using fused::up;
 constexpr int kThreads = 256;
 constexpr int kWarps = 8;
 constexpr int kTileQ = 512;   // queries per assignment tile
-constexpr int kChunk = 512;   // keys per centroid-attention CTA
+constexpr int kMaxChunk = 2048;  // most keys per centroid-attention CTA (a multiple of 256)
 constexpr int kWinQ = 128;    // queries per window CTA
 constexpr int kMaxR = 128;    // largest window radius floor(W/2)
 constexpr int kNTChunk = 6;   // key n-tiles per online-softmax step in the window
@@ -638,7 +638,7 @@ struct CentroidTcLayout {
         red_off = o;  // [2][128] half-row maxima, then [2][128] half-row sums
         o += 2u * 2u * 128u * 4u;
         km_off = o;  // key mask of the chunk (masked calls)
-        o += mask ? 512u : 0u;
+        o += mask ? (uint32_t)kMaxChunk : 0u;
         bar_off = o;  // four mbarriers, the tensor-memory address
         o += 48;
         total = up(o, 128) + 1024;  // + slack to align the base to 1024 bytes
@@ -649,6 +649,7 @@ struct CentroidTcParams {
     const __nv_bfloat16 *hi;  // [NH][Kp][64] centroids rounded to bf16
     float *part;              // [NH][n_chunks][K][kPartLd]
     int L, K, n_chunks;
+    int chunk_keys;           // keys per CTA: a multiple of 256, at most kMaxChunk
     int H, H_kv;              // query head h reads key/value head kv_head(h) of the [B H_kv] tensors
     float scale;
     const uint8_t *key_valid;  // [B][L] key-padding mask or null: invalid keys take no weight
@@ -678,8 +679,8 @@ __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_
     const int chunk = blockIdx.x;
     const int64_t head = blockIdx.y;
     const int kvh = kv_head(head, P.H, P.H_kv);
-    const int c0 = chunk * kChunk;
-    const int nsteps = min(2, (L - c0 + 255) / 256);
+    const int c0 = chunk * P.chunk_keys;
+    const int nsteps = min(P.chunk_keys / 256, (L - c0 + 255) / 256);
     const uint32_t sb = smem_u32(smem);
     const uint32_t z_s = sb + lay.z_off, k_s = sb + lay.k_off, v_s = sb + lay.v_off, p_s = sb + lay.p_off;
     const uint32_t bar_k = sb + lay.bar_off, bar_v = bar_k + 8, bar_s = bar_k + 16, bar_o = bar_k + 24;
@@ -701,7 +702,7 @@ __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_
     uint8_t *kmask = smem + lay.km_off;
     if constexpr (MASK) {
         const uint8_t *kv = P.key_valid + (head / P.H) * L;
-        for (int c = tid; c < kChunk; c += 256) kmask[c] = c0 + c < L ? kv[c0 + c] : 0;
+        for (int c = tid; c < P.chunk_keys; c += 256) kmask[c] = c0 + c < L ? kv[c0 + c] : 0;
     }
     // P starts as zeros (each row later writes only its own keys)
     for (int e = tid; e < 2 * 16384 / 16; e += 256)

@@ -175,3 +175,21 @@ def test_soft_gather_on_the_tiled_kernels(K, W, modes, masked):
     _lib.profile_start("tiled_assign")
     _check("bf16", xq, xk, K, 3, W, 0.4, key_valid=valid, gather_mode=1, **modes)
     assert _lib.profile_stop().launches == 3, "the tiled path did not run"
+
+
+@pytest.mark.parametrize("masked,modes", [(False, {}), (True, {}), (True, dict(gather_mode=1))])
+def test_long_centroid_chunks(masked, modes):
+    # 80 heads of 2600 keys: the centroid attention takes 2048-key chunks
+    # (80 x 2 CTAs fill a 148-multiprocessor device), the second one ragged
+    # (552 keys); with a scattered and a trailing key mask.
+    from means_cluster_attention_b200 import _lib
+    B, H, L = 2, 40, 2600
+    xq, xk = _case("bf16", B, H, L, 20, 2, 64, 0.5, seed=131 + len(modes) + masked)
+    valid = None
+    if masked:
+        valid = np.ones((B, L), dtype=bool)
+        valid[0, 2300:] = False
+        valid[1, ::5] = False
+    _lib.profile_start("tiled_centroid")
+    _check("bf16", xq, xk, 20, 2, 64, 0.5, key_valid=valid, **modes)
+    assert _lib.profile_stop().launches == 1, "the tiled path did not run"
