@@ -637,8 +637,8 @@ struct CentroidTcLayout {
         o += 2u * 16384u;
         red_off = o;  // [2][128] half-row maxima, then [2][128] half-row sums
         o += 2u * 2u * 128u * 4u;
-        km_off = o;  // key mask of the chunk (masked calls)
-        o += mask ? (uint32_t)kMaxChunk : 0u;
+        km_off = o;  // key mask of the chunk, one bit per key (masked calls)
+        o += mask ? (uint32_t)kMaxChunk / 8u : 0u;
         bar_off = o;  // four mbarriers, the tensor-memory address
         o += 48;
         total = up(o, 128) + 1024;  // + slack to align the base to 1024 bytes
@@ -699,10 +699,18 @@ __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_
         umma::mbar_expect_tx(bar_v, 256u * 128u);
         umma::tma_load_3d(v_s, &tmv, 0, c0, kvh, bar_v);
     }
-    uint8_t *kmask = smem + lay.km_off;
+    uint8_t *kmask = smem + lay.km_off;  // bit (c & 7) of byte c / 8: key c0 + c is valid
     if constexpr (MASK) {
         const uint8_t *kv = P.key_valid + (head / P.H) * L;
-        for (int c = tid; c < P.chunk_keys; c += 256) kmask[c] = c0 + c < L ? kv[c0 + c] : 0;
+        for (int b = tid; b < P.chunk_keys / 8; b += 256) {
+            uint32_t bits = 0u;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int c = c0 + 8 * b + j;
+                bits |= (c < L && kv[c] != 0) ? 1u << j : 0u;
+            }
+            kmask[b] = (uint8_t)bits;
+        }
     }
     // P starts as zeros (each row later writes only its own keys)
     for (int e = tid; e < 2 * 16384 / 16; e += 256)
@@ -775,9 +783,12 @@ __global__ void __launch_bounds__(256, 2) tiled_centroid_tc_kernel(const __grid_
             // an invalid key takes no weight; a head without a valid key
             // weighs every key the same
             const bool any = P.any_valid[head] != 0;
+            // this thread's KP keys start at a multiple of KP within the
+            // chunk: their bits are whole bytes of the mask
+            const uint8_t *mrow = kmask + ((key0 - c0) >> 3);
 #pragma unroll
             for (int t = 0; t < KP; ++t)
-                if (key0 + t < L) v[t] = any ? (kmask[key0 + t - c0] ? v[t] : -INFINITY) : 0.f;
+                if (key0 + t < L) v[t] = any ? (((mrow[t >> 3] >> (t & 7)) & 1u) ? v[t] : -INFINITY) : 0.f;
         }
         if (c0 + 256 * (s + 1) > L) {  // keys past L (zero rows of the load) do not exist
 #pragma unroll
