@@ -58,6 +58,7 @@ using fused::up;
 constexpr int kThreads = 256;
 constexpr int kWarps = 8;
 constexpr int kTileQ = 512;   // queries per assignment tile
+constexpr int kDirectMovers = 16;  // up to this many movers per tile skip the sort
 constexpr int kMaxChunk = 2048;  // most keys per centroid-attention CTA (a multiple of 256)
 constexpr int kWinQ = 128;    // queries per window CTA
 constexpr int kMaxR = 128;    // largest window radius floor(W/2)
@@ -584,6 +585,29 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     }
     __syncthreads();
     const int n_mv = misc[3];
+    if (n_mv <= kDirectMovers) {
+        // few movers: each warp subtracts its movers' rows from their old
+        // clusters and adds them to their new ones directly (lane l:
+        // coordinates 2l and 2l + 1); the sums are exact, so this changes
+        // no bit of them
+        for (int e = warp; e < n_mv; e += kWarps) {
+            const int row = CA_IDX((int)list[e], 0, Lt, 79);
+            const int cn = CA_IDX((int)cs[row], 0, Kp, 80), co = CA_IDX((int)cprev[row], 0, Kp, 81);
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(qbytes + swz(row, lane >> 2) + (lane & 3) * 4);
+            const double x0 = (double)bf16lo(w), x1 = (double)bf16hi(w);
+            const int j0 = 2 * lane, j1 = 2 * lane + 1;
+            const int o0 = (j0 & 3) * 16 + (j0 >> 2), o1 = (j1 & 3) * 16 + (j1 >> 2);
+            atomicAdd(gsum + cn * kD + o0, x0);
+            atomicAdd(gsum + cn * kD + o1, x1);
+            atomicAdd(gsum + co * kD + o0, -x0);
+            atomicAdd(gsum + co * kD + o1, -x1);
+            if (lane == 0) {
+                atomicAdd(gcnt + cn, 1);
+                atomicAdd(gcnt + co, -1);
+            }
+        }
+        return;
+    }
     // batches of up to 256 movers: entry e < m adds mover b + e to its new
     // cluster, entry m + e subtracts it from its old one
     for (int b = 0; b < n_mv; b += kTileQ / 2) {
