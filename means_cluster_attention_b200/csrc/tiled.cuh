@@ -17,8 +17,9 @@
 //                                          tokens, the tile's exact share of
 //                                          the head's running member sums.
 //   tiled_centroid_tc_kernel (chunks, heads) partial softmax state of every
-//                                          centroid over 512 keys on tcgen05
-//                                          (M = 64 tiles at two lane offsets);
+//                                          centroid over a chunk of 512 to
+//                                          2048 keys on tcgen05 (M = 64 tiles
+//                                          at two lane offsets);
 //   tiled_combine_kernel   (K, heads)      combines the chunk states into
 //                                          V_cent.
 //   tiled_window_tc_kernel (blocks, heads) clipped window attention for 128
@@ -629,11 +630,11 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
 }
 
 // ---------------------------------------------------------------------------
-// Centroid attention over a chunk of up to 512 keys on tcgen05: the chunk's
-// softmax state of every centroid (sum of exp-weighted V rows, max in
-// natural-log units, denominator) in the layout tiled_combine_kernel reads.
+// Centroid attention over a chunk of up to kMaxChunk keys on tcgen05: the
+// chunk's softmax state of every centroid (sum of exp-weighted V rows, max
+// in natural-log units, denominator) in the layout tiled_combine_kernel reads.
 //
-// The chunk goes in two steps of 256 keys.  S = mu K^T runs as M = 64
+// The chunk goes in steps of 256 keys.  S = mu K^T runs as M = 64
 // tcgen05.mma tiles (rows = centroids) at tensor-memory lane offsets 0 and
 // 16, so the two tiles together fill all 128 lanes: tile o takes keys
 // [128 o, 128 o + 128) of the step.  Within a tile, G = 64 / KP groups of
