@@ -247,25 +247,29 @@ __global__ void __launch_bounds__(64) tiled_combine_kernel(int K, int n_chunks, 
 //
 // Q tile: two TMA loads of 256 rows (128-byte swizzle) into shared memory.
 // Distances: one thread issues tcgen05.mma for each 128-token block,
-// D = Q [128 x 64] . (hi + lo)^T [64 x Kp] accumulated in fp32 in tensor
-// memory (4 k-steps with hi, then 4 with lo, into the same accumulator).
-// Epilogue: every thread owns one token row of a block (tcgen05.ld), forms
-// s_k = |mu_k|^2 - 2 D_k, takes the minimum m1 and the set of k with
-// s_k <= m1 + 2E; a single member is the certified argmin, several send the
-// token to the exact fp64 re-measure.  Sums: the tile's tokens (first
+// D = Q [128 x 64] . (hi + lo)^T [64 x Kp] - |mu|^2 / 2 accumulated in fp32
+// in tensor memory (4 k-steps with hi, then 4 with lo, then one whose A is a
+// column of ones and whose B holds -|mu_k|^2 / 2 split into three bf16 terms,
+// -inf for centroids that can never win), so s_k = |mu_k|^2 - 2 D_k needs no
+// arithmetic: s_k <= m1 + 2E is D_k >= max_k D_k - E.
+// Epilogue: every thread owns one token row of a block (tcgen05.ld), takes
+// the maximum of D and the set of k with D_k >= max D - E; a single member
+// is the certified argmin, several send the token to the exact fp64
+// re-measure.  Sums: the tile's tokens (first
 // iteration) or its movers (later ones, signed) are sorted by cluster and
 // added run by run to the head's running sums with fp64 reductions.
 //
-// Error bound: the split leaves |mu - hi - lo| <= 2^-18 |mu| per coordinate;
-// the products are exact and even an accumulator that truncates every one of
-// the 128 additions stays within 128 * 2^-23 (1 + 2^-8) |Q| |mu| of the
-// exact dot product, so |s_k error| <= 2^-14.6 (|Q| |mu_k| + |mu_k|^2) with
-// the fp32 |mu_k|^2 and the final fma included; E = 2^-13 (|Q| max|mu| +
-// max|mu|^2) covers it threefold.
+// Error bound: the split leaves |mu - hi - lo| <= 2^-18 |mu| per coordinate
+// (2^-17 |Q| |mu| in s); the products are exact and even an accumulator that
+// truncates every one of the 131 additions stays within 131 * 2^-23
+// (1 + 2^-8) (|Q| |mu| + |mu|^2 / 2) of the exact value (2^-14.97 (...) in
+// s); the fp32 |mu_k|^2 and its three-term split add under 2^-20 |mu_k|^2.
+// So |s_k error| <= 2^-14.6 (|Q| |mu_k| + |mu_k|^2), and E = 2^-13 (|Q|
+// max|mu| + max|mu|^2) covers it threefold.
 struct AssignLayout {
     int Kp;
-    uint32_t q_off, r_off, mu_off, mm_off, dead_off, cnt_off, c_off, cprev_off, list_off, lmask_off, ent_off,
-        misc_off, bar_off, total;
+    uint32_t q_off, r_off, mu_off, ones_off, mb_off, dead_off, cnt_off, c_off, cprev_off, list_off,
+        lmask_off, ent_off, misc_off, bar_off, total;
     __host__ __device__ AssignLayout(int K) {
         Kp = kpad(K);
         uint32_t o = 0;
@@ -277,8 +281,13 @@ struct AssignLayout {
         r_off = o;
         mu_off = o + 2u * (uint32_t)Kp * 128u;
         o += up(2u * (uint32_t)Kp * 128u + (uint32_t)Kp * 68u * 4u, 16);
-        mm_off = o;
-        o += (uint32_t)Kp * 4u;
+        // The |mu|^2 step's operands, K-major without swizzle (8-row x 16-byte
+        // core matrices): A = 8 rows [1 1 1 0 ...] read for all 128 rows, B =
+        // the Kp rows [h m l 0 ...] of -|mu_k|^2 / 2 = h + m + l.
+        ones_off = o;
+        o += 256u;
+        mb_off = o;
+        o += (uint32_t)Kp / 8u * 256u;
         dead_off = o;
         o += up((uint32_t)Kp, 16);
         cnt_off = o;
@@ -340,7 +349,6 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + lay.bar_off + 48);
     unsigned char *qbytes = smem + lay.q_off;
     float *mu = reinterpret_cast<float *>(smem + lay.mu_off);        // [Kp][68]
-    float *mm = reinterpret_cast<float *>(smem + lay.mm_off);
     int *cnt_s = reinterpret_cast<int *>(smem + lay.cnt_off);
     uint8_t *dead = smem + lay.dead_off;
     uint8_t *cs = smem + lay.c_off;
@@ -399,9 +407,25 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
     }
     for (int kk = threadIdx.x; kk < Kp; kk += kThreads) {
         const uint8_t dd = P.dead[cb + kk];
-        mm[kk] = dd ? INFINITY : P.mm[cb + kk];
         dead[kk] = dd;
         cnt_s[kk] = 0;
+        // -|mu_k|^2 / 2 as three bf16 terms (-inf: this centroid never wins)
+        uint32_t w0 = 0xFF80u, w1 = 0u;  // bf16 -inf, then zeros
+        if (!dd) {
+            const float v = -0.5f * P.mm[cb + kk];
+            const __nv_bfloat16 h = __float2bfloat16_rn(v);
+            const float r1 = v - __bfloat162float(h);
+            const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+            const __nv_bfloat16 l = __float2bfloat16_rn(r1 - __bfloat162float(m));
+            w0 = (uint32_t)__bfloat16_as_ushort(h) | ((uint32_t)__bfloat16_as_ushort(m) << 16);
+            w1 = (uint32_t)__bfloat16_as_ushort(l);
+        }
+        *reinterpret_cast<uint4 *>(smem + lay.mb_off + (kk >> 3) * 256 + (kk & 7) * 16) = make_uint4(w0, w1, 0u, 0u);
+        *reinterpret_cast<uint4 *>(smem + lay.mb_off + (kk >> 3) * 256 + 128 + (kk & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (threadIdx.x < 16) {  // 8 rows [1 1 1 0 0 0 0 0 | 0 ... 0]
+        const uint4 w = threadIdx.x < 8 ? make_uint4(0x3F803F80u, 0x3F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4 *>(smem + lay.ones_off + threadIdx.x * 16) = w;
     }
     for (int i = threadIdx.x; i < kTileQ; i += kThreads) cs[i] = i < Lt ? 0 : 0xFF;
     if (threadIdx.x == 0) {
@@ -435,6 +459,8 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
                                        umma::desc_sw128(q_s + (uint32_t)m * 16384u + (uint32_t)ks * 32u),
                                        umma::desc_sw128(b_s + (uint32_t)part * (uint32_t)Kp * 128u + (uint32_t)ks * 32u),
                                        idesc, part > 0 || ks > 0);
+                umma::mma_bf16(taddr + (uint32_t)(m * KP), umma::desc_kmajor_plain(sbase + lay.ones_off, 128u, 0u),
+                               umma::desc_kmajor_plain(sbase + lay.mb_off, 128u, 256u), idesc, true);
                 umma::mma_commit(bar_mma + 8u * (uint32_t)m);
             }
         } else {
@@ -490,25 +516,21 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
             }
             umma::tmem_ld_wait();
             if (row < Lt) {
-                float m1a = INFINITY, m1b = INFINITY;
+                // sv[k] = D_k = Q.mu_k - |mu_k|^2 / 2 = -s_k / 2
+                float m1a = -INFINITY, m1b = -INFINITY;
 #pragma unroll
-                for (int k4 = 0; k4 < KP / 4; ++k4) {
-                    const float4 m4 = reinterpret_cast<const float4 *>(mm)[k4];
-                    sv[4 * k4 + 0] = fmaf(-2.f, sv[4 * k4 + 0], m4.x);
-                    sv[4 * k4 + 1] = fmaf(-2.f, sv[4 * k4 + 1], m4.y);
-                    sv[4 * k4 + 2] = fmaf(-2.f, sv[4 * k4 + 2], m4.z);
-                    sv[4 * k4 + 3] = fmaf(-2.f, sv[4 * k4 + 3], m4.w);
-                    m1a = fminf(m1a, fminf(sv[4 * k4 + 0], sv[4 * k4 + 1]));
-                    m1b = fminf(m1b, fminf(sv[4 * k4 + 2], sv[4 * k4 + 3]));
+                for (int k2 = 0; k2 < KP / 2; ++k2) {
+                    m1a = fmaxf(m1a, sv[2 * k2]);
+                    m1b = fmaxf(m1b, sv[2 * k2 + 1]);
                 }
-                const float m1 = fminf(m1a, m1b);
+                const float dmax = fmaxf(m1a, m1b);
                 const float E = kEps * fmaf(qn[mi], mun_max, mm_max);
-                const float thr = m1 + 2.f * E;
+                const float thr = dmax - E;  // s_k <= m1 + 2E
                 uint32_t bits[(KP + 31) / 32];
 #pragma unroll
                 for (int w2 = 0; w2 < (KP + 31) / 32; ++w2) bits[w2] = 0u;
 #pragma unroll
-                for (int k = 0; k < KP; ++k) bits[k >> 5] |= (sv[k] <= thr ? 1u : 0u) << (k & 31);
+                for (int k = 0; k < KP; ++k) bits[k >> 5] |= (sv[k] >= thr ? 1u : 0u) << (k & 31);
                 int c = -1, n = 0;
 #pragma unroll
                 for (int w2 = (KP + 31) / 32 - 1; w2 >= 0; --w2) {
@@ -521,12 +543,12 @@ __global__ void __launch_bounds__(kThreads, 2) tiled_assign_kernel(const __grid_
                     // every k with s_k <= m1 + 3E, so any other centroid is
                     // worse than the fp32 winner by at least E in exact
                     // arithmetic
-                    const float thr3 = m1 + 3.f * E;
+                    const float thr3 = dmax - 1.5f * E;
                     uint32_t b3[(KP + 31) / 32];
 #pragma unroll
                     for (int w2 = 0; w2 < (KP + 31) / 32; ++w2) b3[w2] = 0u;
 #pragma unroll
-                    for (int k = 0; k < KP; ++k) b3[k >> 5] |= (sv[k] <= thr3 ? 1u : 0u) << (k & 31);
+                    for (int k = 0; k < KP; ++k) b3[k >> 5] |= (sv[k] >= thr3 ? 1u : 0u) << (k & 31);
                     const int e = CA_IDX(atomicAdd(&misc[0], 1), 0, kTileQ, 63);
                     list[e] = (uint16_t)row;
 #pragma unroll

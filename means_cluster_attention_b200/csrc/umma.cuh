@@ -93,6 +93,17 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
            | ((uint64_t)2 << 61);               // 128-byte swizzle
 }
 
+// Shared-memory matrix descriptor of a K-major operand without swizzle:
+// core matrices of 8 rows x 16 bytes (rows 16 bytes apart), lbo bytes
+// between core matrices adjacent in K, sbo bytes between groups of 8 rows
+// (0: every group reads the same 8 rows).
+__device__ __forceinline__ uint64_t desc_kmajor_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4)      // start address, 16-byte units
+           | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16)
+           | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32)
+           | ((uint64_t)1 << 46);                   // descriptor version for sm_100; no swizzle
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B (both K-major) and an
 // fp32 accumulator, for an M x N tile.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
