@@ -8,7 +8,9 @@
 // aligned): 16-byte chunk c of row r sits at r * 128 + ((c ^ (r & 7)) << 4).
 // This is what a TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes, what swz()
 // in mma.cuh addresses, and what the SWIZZLE_128B shared-memory matrix
-// descriptor of tcgen05.mma reads.
+// descriptor of tcgen05.mma reads.  The one exception is the assignment's
+// K = 16 step that adds -|mu|^2 / 2: its two small operands are K-major
+// without swizzle (desc_kmajor_plain).
 #pragma once
 
 #include <stdint.h>
